@@ -1,0 +1,157 @@
+/*
+ * tri_attn.h -- C ABI of the B200 (sm_100a) gated triangle self-attention library.
+ *
+ * The operation. Triangle attention lets an AlphaFold-family model use a third
+ * residue k when it reasons about the pair (i, j); its cost grows cubically
+ * with the crop size, and its backward returns gradients for query, key, value
+ * and pair bias ("TurboPairFormer accelera fino a 1,73x l'addestramento di
+ * OpenFold3 nei test", section "Dove si impiega il tempo"). The gate is fused
+ * into the attention op ("HelixFold: An Efficient Implementation of AlphaFold2
+ * using PaddlePaddle", proposed methods: fused gated self-attention), and the
+ * N^3*H logits are computed tile by tile in on-chip memory and never stored
+ * ("MegaFold: Efficient Training of Next-Generation 3D Attention Protein Models
+ * on Cross-Platform GPUs", tool 1, EvoFlash-3D). For each attention row r, head
+ * h and query x, with c the head dimension:
+ *
+ *   s_y   = c^-1/2 <q[r,x,h,:], k[r,y,h,:]> + bias[h,x,y] + mu(r,y)
+ *   lse   = log sum_y exp(s_y)
+ *   out   = sigmoid(gate[r,x,h,:]) * sum_y exp(s_y - lse) v[r,y,h,:]
+ *
+ * mu(r,y) = 0 if mask[r*mask_row_stride + y] != 0, else -infinity. A row whose
+ * keys are all masked yields out = 0 and lse = -infinity and adds nothing to
+ * any gradient.
+ *
+ * Variants. STARTING (around the starting node): row r = i, query x = j, key
+ * y = k; pair tensors are read at [r, x] / [r, y] and the bias at [h, x, y].
+ * ENDING (around the ending node) runs the same computation on the transposed
+ * pair layout: pair tensors are read and written at [x, r] / [y, r], the bias
+ * at [h, y, x], and dbias is returned in the bias's own storage layout. The
+ * mask and lse are always in the variant's own frame (row, key) / (row, head,
+ * query).
+ *
+ * Layout (all row-major, c fastest, no padding):
+ *   q, k, v, gate, out, dout, dq, dk, dv, dgate : [N, N, H, c]
+ *   bias, dbias                                 : [H, N, N]
+ *   lse                                         : float32 [N, H, N]
+ *   mask                                        : uint8, row stride
+ *                                                 mask_row_stride (0: one key
+ *                                                 mask [N] shared by every row;
+ *                                                 N: a full [N, N] mask); NULL
+ *                                                 means every key takes part.
+ *
+ * Types. dtype BF16: every tensor above except lse and mask is bfloat16;
+ * contractions run on the tensor cores with fp32 accumulation, softmax and
+ * gate arithmetic in fp32; dbias is accumulated in fp32 over all rows and
+ * rounded once. dtype F32: every tensor is float32 and all arithmetic is fp32
+ * on the CUDA cores (no TF32).
+ *
+ * Ownership and threading. Every pointer is a caller-owned device pointer,
+ * 16-byte aligned, to contiguous memory. The library allocates no device
+ * memory and keeps no state between calls: scratch space is the caller's
+ * workspace. Outputs are overwritten, never accumulated into. Calls only
+ * enqueue work on the given stream and return without synchronising; results
+ * are ready once the stream reaches them. Repeated calls on identical inputs
+ * give bit-identical outputs (all reductions run in a fixed order, no
+ * floating-point atomics). Concurrent calls must use distinct workspaces.
+ *
+ * Errors. Argument checks happen on the host before anything is enqueued; a
+ * call that returns anything but TRI_ATTN_OK has enqueued nothing, except
+ * TRI_ATTN_ERR_CUDA, which reports a failed launch. Device-side failures (a
+ * bounded wait that ran out) never trap: the kernel records the failure in the
+ * workspace status word, fills the affected lse entries with NaN and returns;
+ * tri_attn_read_status() reports it.
+ */
+#ifndef TRI_ATTN_H
+#define TRI_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *tri_attn_stream_t;
+
+typedef enum {
+    TRI_ATTN_OK = 0,
+    TRI_ATTN_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size or enum */
+    TRI_ATTN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (see limits)    */
+    TRI_ATTN_ERR_WORKSPACE = 3,    /* workspace missing or too small            */
+    TRI_ATTN_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed         */
+    TRI_ATTN_ERR_TIMEOUT = 5,      /* device: a bounded wait ran out            */
+    TRI_ATTN_ERR_BOUNDS = 6        /* device: an index check failed             */
+} tri_attn_status;
+
+typedef enum { TRI_ATTN_F32 = 0, TRI_ATTN_BF16 = 1 } tri_attn_dtype;
+typedef enum { TRI_ATTN_STARTING = 0, TRI_ATTN_ENDING = 1 } tri_attn_variant;
+
+/*
+ * Problem description. Limits: N >= 0; H >= 1; N * N * H * c < 2^31 * 64.
+ * BF16 needs c == 32 and N % 8 == 0 (the bias rows are moved by TMA, whose row
+ * pitch must be a multiple of 16 bytes). F32 needs 1 <= c <= 64.
+ */
+typedef struct {
+    int64_t N;                /* residues: the pair tensors are N x N           */
+    int32_t H;                /* heads                                          */
+    int32_t c;                /* head dimension                                 */
+    int32_t dtype;            /* tri_attn_dtype                                 */
+    int32_t variant;          /* tri_attn_variant                               */
+    int64_t mask_row_stride;  /* 0 or N (ignored when mask is NULL)             */
+} tri_attn_problem;
+
+/* Library version, (major << 16) | minor. */
+int tri_attn_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *tri_attn_status_string(tri_attn_status status);
+
+/*
+ * Workspace the forward needs, in bytes (a status word, plus a transposed copy
+ * of the bias for the ENDING variant). Writes *bytes; fails only on an invalid
+ * problem.
+ */
+tri_attn_status tri_attn_fwd_workspace_size(const tri_attn_problem *prob, size_t *bytes);
+
+/*
+ * Forward. Reads q, k, v, bias, gate (and mask); writes out and lse. The
+ * workspace must hold at least tri_attn_fwd_workspace_size() bytes, 256-byte
+ * aligned; its contents on entry do not matter.
+ */
+tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
+                             const void *v, const void *bias, const void *gate,
+                             const uint8_t *mask, void *out, float *lse, void *workspace,
+                             size_t workspace_bytes, tri_attn_stream_t stream);
+
+/* Workspace the backward needs for this problem, in bytes. */
+tri_attn_status tri_attn_bwd_workspace_size(const tri_attn_problem *prob, size_t *bytes);
+
+/*
+ * Backward of L = sum(dout * out). Reads the forward's inputs and its outputs
+ * out and lse (as written by tri_attn_fwd on the same inputs) and dout; writes
+ * dq, dk, dv, dgate (pair layout of the inputs) and dbias ([H, N, N], summed
+ * over all N attention rows). The probabilities are recomputed from lse once
+ * per tile and reused for all four gradients of that tile. Workspace as for
+ * the forward, at least tri_attn_bwd_workspace_size() bytes.
+ */
+tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const void *k,
+                             const void *v, const void *bias, const void *gate,
+                             const uint8_t *mask, const void *out, const float *lse,
+                             const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                             void *dgate, void *workspace, size_t workspace_bytes,
+                             tri_attn_stream_t stream);
+
+/*
+ * Device status word of the last call that used this workspace: synchronises
+ * the stream, copies the word to the host and stores a tri_attn_status in
+ * *device_status. Returns TRI_ATTN_ERR_CUDA if the copy itself fails.
+ */
+tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_status,
+                                     tri_attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_ATTN_H */

@@ -1,0 +1,85 @@
+"""Shared helpers of the GPU tests: run the CUDA path through the binding and
+compare it with the oracle in the variant frame."""
+
+import numpy as np
+import torch
+
+import triangle_attention_b200 as ta
+from tri_inputs import ENDING, STARTING
+
+# Tolerances. fp32 path: relative L2 1e-5 on every output. bf16 path: relative
+# L2 1e-2 on out, dq, dk, dv, dgate and dbias, max-abs 2e-2 on out. lse is
+# computed in fp32 from exactly representable logits; its error is set by the
+# hardware exp2/log2 approximations (~2^-22 relative), so 1e-3 absolute is
+# loose for both paths.
+F32_REL = 1e-5
+BF16_REL = 1e-2
+BF16_OUT_ABS = 2e-2
+LSE_ABS = 1e-3
+
+
+def rel_l2(a, b) -> float:
+    a = np.asarray(a, dtype=np.float64).ravel()
+    b = np.asarray(b, dtype=np.float64).ravel()
+    den = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
+
+
+def np64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def variant_frame(t: torch.Tensor, variant: int) -> torch.Tensor:
+    """Pair tensor in storage layout -> [row, query, H, c] of the variant."""
+    return t if variant == STARTING else t.transpose(0, 1)
+
+
+def to_device(d: dict, device) -> dict:
+    out = {}
+    for k, v in d.items():
+        out[k] = v.to(device).contiguous() if torch.is_tensor(v) else v
+    return out
+
+
+def run_cuda(d: dict, variant: int, backward: bool = True, device="cuda:0"):
+    g = to_device(d, device)
+    out, lse = ta.fwd(g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], variant)
+    res = {"out": out, "lse": lse}
+    if backward:
+        dq, dk, dv, db, dg = ta.bwd(g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], out,
+                                    lse, g["dout"], variant)
+        res.update(dq=dq, dk=dk, dv=dv, dbias=db, dgate=dg)
+    torch.cuda.synchronize()
+    return res
+
+
+def assert_close(name, got, ref, rel, max_abs=None):
+    err = rel_l2(got, ref)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    assert err <= rel, f"{name}: relative L2 error {err:.3e} > {rel:.1e}"
+    if max_abs is not None:
+        m = float(np.max(np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))))
+        assert m <= max_abs, f"{name}: max abs error {m:.3e} > {max_abs:.1e}"
+    return err
+
+
+def compare_rows(res, ref_fwd, ref_bwd, rows, variant, dtype):
+    """Compare the CUDA results on the listed attention rows (variant frame)."""
+    rel = F32_REL if dtype == "f32" else BF16_REL
+    out_abs = None if dtype == "f32" else BF16_OUT_ABS
+    errs = {}
+    o_ref, l_ref = ref_fwd
+    out = np64(variant_frame(res["out"], variant))[rows]
+    lse = np64(res["lse"])[rows]
+    errs["out"] = assert_close("out", out, o_ref, rel, out_abs)
+    fin = np.isfinite(l_ref)
+    assert np.array_equal(np.isfinite(lse), fin), "lse: -inf pattern differs"
+    if fin.any():
+        m = float(np.max(np.abs(lse[fin] - l_ref[fin])))
+        assert m <= LSE_ABS, f"lse: max abs error {m:.3e}"
+        errs["lse_abs"] = m
+    if ref_bwd is not None:
+        for name, ref in zip(("dq", "dk", "dv", "dgate"), ref_bwd[:4]):
+            got = np64(variant_frame(res[name], variant))[rows]
+            errs[name] = assert_close(name, got, ref, rel)
+    return errs

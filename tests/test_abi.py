@@ -1,0 +1,141 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import triangle_attention_b200 as ta
+from triangle_attention_b200 import build as tbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+def declared_functions():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(tri_attn_\w+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tbuild.build()
+    return ta.lib()
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("tri_attn_fwd", "tri_attn_bwd", "tri_attn_fwd_workspace_size",
+                     "tri_attn_bwd_workspace_size", "tri_attn_read_status",
+                     "tri_attn_status_string", "tri_attn_version"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} is declared but not exported"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.tri_attn_version() >> 16 == 1
+    for code in range(7):
+        assert lib.tri_attn_status_string(code).decode() == ta.STATUS[code]
+    assert lib.tri_attn_status_string(99).decode() == "unknown status"
+
+
+def P(N=64, H=4, c=32, dtype=ta.BF16, variant=ta.STARTING, stride=0):
+    return ta.Problem(N, H, c, dtype, variant, stride)
+
+
+def ws_size(lib, prob, which="fwd"):
+    n = ctypes.c_size_t(0)
+    f = lib.tri_attn_fwd_workspace_size if which == "fwd" else lib.tri_attn_bwd_workspace_size
+    rc = f(ctypes.byref(prob), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_sizes(lib):
+    rc, n = ws_size(lib, P())
+    assert rc == 0 and n >= 256
+    rc, ne = ws_size(lib, P(variant=ta.ENDING))
+    assert rc == 0 and ne >= n + 2 * 4 * 64 * 64       # transposed bias copy
+    rc, nb = ws_size(lib, P(N=768), "bwd")
+    assert rc == 0
+    pair = 768 * 768 * 4 * 32
+    # dU (bf16) + D + three sets of fp32 partials over 6 tiles
+    assert nb >= 2 * pair + 4 * 768 * 768 * 4 + 3 * 6 * 4 * pair
+    rc, nf = ws_size(lib, P(N=32, dtype=ta.F32), "bwd")
+    assert rc == 0 and nf > 0
+
+
+@pytest.mark.parametrize("prob,code", [
+    (P(N=-1), 1), (P(H=0), 1), (P(c=0), 1), (P(dtype=7), 1), (P(variant=2), 1),
+    (P(stride=5), 1), (P(c=64), 2), (P(N=60), 2), (P(dtype=ta.F32, c=65), 2),
+])
+def test_invalid_problems(lib, prob, code):
+    rc, _ = ws_size(lib, prob)
+    assert rc == code
+    rc, _ = ws_size(lib, prob, "bwd")
+    assert rc == code
+
+
+def test_null_problem_and_null_size(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.tri_attn_fwd_workspace_size(None, ctypes.byref(n)) == 1
+    assert lib.tri_attn_fwd_workspace_size(ctypes.byref(P()), None) == 1
+
+
+def test_host_side_rejections_before_any_launch(lib):
+    """These return before any CUDA call, so they run without a GPU."""
+    prob = P()
+    fake = ctypes.c_void_p(4096)          # 256-aligned, never dereferenced
+    z = None
+    args = [fake] * 5 + [z] + [fake, fake]
+    # missing workspace
+    assert lib.tri_attn_fwd(ctypes.byref(prob), *args, z, 0, z) == 3
+    # misaligned workspace
+    assert lib.tri_attn_fwd(ctypes.byref(prob), *args, ctypes.c_void_p(4100), 1 << 20, z) == 3
+    # too small a workspace
+    assert lib.tri_attn_fwd(ctypes.byref(prob), *args, fake, 16, z) == 3
+    # null and misaligned tensors
+    bad = [fake] * 5 + [z] + [z, fake]
+    assert lib.tri_attn_fwd(ctypes.byref(prob), *bad, fake, 1 << 30, z) == 1
+    mis = [ctypes.c_void_p(4098)] + [fake] * 4 + [z] + [fake, fake]
+    assert lib.tri_attn_fwd(ctypes.byref(prob), *mis, fake, 1 << 30, z) == 1
+    # backward: invalid problem, then missing workspace
+    bargs = [fake] * 5 + [z] + [fake] * 8
+    assert lib.tri_attn_bwd(ctypes.byref(P(c=7)), *bargs, fake, 1 << 40, z) == 2
+    assert lib.tri_attn_bwd(ctypes.byref(prob), *bargs, z, 0, z) == 3
+    # N = 0 is a valid no-op
+    zero = P(N=0)
+    assert lib.tri_attn_fwd(ctypes.byref(zero), *args, fake, 1 << 20, z) == 0
+    assert lib.tri_attn_bwd(ctypes.byref(zero), *bargs, fake, 1 << 20, z) == 0
+
+
+def test_read_status_rejects_null(lib):
+    v = ctypes.c_int32(0)
+    assert lib.tri_attn_read_status(None, ctypes.byref(v), None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ta, "_lib", None)
+    monkeypatch.setattr(ta, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ta.lib()
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "triangle_attention_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.lower().replace("oracle/", ""), f

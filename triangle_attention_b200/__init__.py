@@ -1,0 +1,200 @@
+"""Thin Python binding of libtri_attn.so (gated triangle self-attention, B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. PyTorch supplies device memory and the current stream. If the shared
+library is missing or cannot be loaded, every entry point raises; there is no
+CPU fallback.
+
+Entry points (names follow the C ABI in include/tri_attn.h):
+    fwd(q, k, v, bias, gate, mask=None, variant=STARTING) -> (out, lse)
+    bwd(q, k, v, bias, gate, mask, out, lse, dout, variant) -> (dq, dk, dv, dbias, dgate)
+    fwd_workspace_size / bwd_workspace_size / read_status
+    TriangleAttention: torch.autograd.Function over fwd/bwd.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+STARTING = 0
+ENDING = 1
+F32 = 0
+BF16 = 1
+
+STATUS = {
+    0: "ok", 1: "invalid argument", 2: "unsupported problem", 3: "workspace missing or too small",
+    4: "CUDA call failed", 5: "device wait timed out", 6: "device index check failed",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtri_attn.so")
+_lib = None
+
+
+class TriAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, 'unknown status')} ({code})")
+        self.code = code
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int32), ("c", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("variant", ctypes.c_int32),
+                ("mask_row_stride", ctypes.c_int64)]
+
+
+def lib():
+    """The loaded library; raises if it was not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m triangle_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        PP = ctypes.POINTER(Problem)
+        sz = ctypes.c_size_t
+        L.tri_attn_version.restype = ctypes.c_int
+        L.tri_attn_status_string.argtypes = [ctypes.c_int]
+        L.tri_attn_status_string.restype = ctypes.c_char_p
+        L.tri_attn_fwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
+        L.tri_attn_bwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
+        L.tri_attn_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, sz, P]
+        L.tri_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
+        for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
+                  L.tri_attn_bwd, L.tri_attn_read_status):
+            f.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def problem(q: torch.Tensor, mask: Optional[torch.Tensor], variant: int) -> Problem:
+    if q.dim() != 4 or q.shape[0] != q.shape[1]:
+        raise ValueError(f"pair tensors must be [N, N, H, c], got {tuple(q.shape)}")
+    N, _, H, c = q.shape
+    stride = 0
+    if mask is not None:
+        if mask.dim() == 1:
+            stride = 0
+        elif mask.dim() == 2:
+            stride = N
+        else:
+            raise ValueError("mask must be [N] (shared by every row) or [N, N]")
+    return Problem(N, H, c, _dtype_code(q), variant, stride)
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise TriAttnError(code, where)
+
+
+def fwd_workspace_size(prob: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tri_attn_fwd_workspace_size(ctypes.byref(prob), ctypes.byref(n)),
+           "tri_attn_fwd_workspace_size")
+    return n.value
+
+
+def bwd_workspace_size(prob: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tri_attn_bwd_workspace_size(ctypes.byref(prob), ctypes.byref(n)),
+           "tri_attn_bwd_workspace_size")
+    return n.value
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A device buffer for the library's scratch (torch allocations are
+    256-byte aligned)."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("every tensor must be contiguous")
+
+
+def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=None, ws=None,
+        stream=None):
+    """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N]."""
+    _contig(q, k, v, bias, gate, mask)
+    prob = problem(q, mask, variant)
+    N, _, H, _ = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((N, H, N), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(fwd_workspace_size(prob), q.device)
+    _check(lib().tri_attn_fwd(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
+                              _p(mask), _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream)),
+           "tri_attn_fwd")
+    return out, lse
+
+
+def bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, grads=None, ws=None,
+        stream=None):
+    """Backward. Returns (dq, dk, dv, dbias, dgate) in the inputs' dtype."""
+    _contig(q, k, v, bias, gate, mask, out, lse, dout)
+    prob = problem(q, mask, variant)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty_like(bias), torch.empty_like(gate))
+    dq, dk, dv, dbias, dgate = grads
+    if ws is None:
+        ws = workspace(bwd_workspace_size(prob), q.device)
+    _check(lib().tri_attn_bwd(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
+                              _p(mask), _p(out), _p(lse), _p(dout), _p(dq), _p(dk), _p(dv),
+                              _p(dbias), _p(dgate), _p(ws), ws.numel(), _stream(stream)),
+           "tri_attn_bwd")
+    return dq, dk, dv, dbias, dgate
+
+
+def read_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device status word of the last
+    call that used this workspace (0 = ok)."""
+    v = ctypes.c_int32(0)
+    _check(lib().tri_attn_read_status(_p(ws), ctypes.byref(v), _stream(stream)),
+           "tri_attn_read_status")
+    return v.value
+
+
+class TriangleAttention(torch.autograd.Function):
+    """out = TriangleAttention.apply(q, k, v, bias, gate, mask, variant)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, bias, gate, mask=None, variant=STARTING):
+        out, lse = fwd(q, k, v, bias, gate, mask, variant)
+        ctx.save_for_backward(q, k, v, bias, gate, out, lse)
+        ctx.mask = mask
+        ctx.variant = variant
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, bias, gate, out, lse = ctx.saved_tensors
+        dq, dk, dv, dbias, dgate = bwd(q, k, v, bias, gate, ctx.mask, out, lse,
+                                       dout.contiguous(), ctx.variant)
+        return dq, dk, dv, dbias, dgate, None, None

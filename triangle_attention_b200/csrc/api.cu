@@ -1,0 +1,408 @@
+// C ABI of the library (declared in include/tri_attn.h): argument checks,
+// workspace carving, TMA tensor-map encoding and dispatch to the kernels.
+// Nothing here allocates device memory or keeps state between calls.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/tri_attn.h"
+#include "bf16.cuh"
+#include "common.cuh"
+
+namespace {
+
+using tri::Frame;
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kMaxN = 1 << 16;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tri_attn_status check_problem(const tri_attn_problem *p) {
+  if (!p) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->N < 0 || p->N > kMaxN || p->H < 1 || p->H > 4096 || p->c < 1)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->dtype != TRI_ATTN_F32 && p->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->variant != TRI_ATTN_STARTING && p->variant != TRI_ATTN_ENDING)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->mask_row_stride != 0 && p->mask_row_stride != p->N) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->dtype == TRI_ATTN_BF16 && (p->c != 32 || p->N % 8 != 0)) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (p->dtype == TRI_ATTN_F32 && p->c > 64) return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
+Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status) {
+  Frame f;
+  f.N = (int)p->N;
+  f.H = p->H;
+  f.c = p->c;
+  f.variant = p->variant;
+  const int64_t N = p->N, H = p->H, C = p->c;
+  if (p->variant == TRI_ATTN_STARTING) {
+    f.sR = N * H * C;
+    f.sX = H * C;
+    f.bX = N;
+    f.bY = 1;
+  } else {
+    f.sR = H * C;
+    f.sX = N * H * C;
+    f.bX = 1;
+    f.bY = N;
+  }
+  f.mask = mask;
+  f.mask_stride = mask ? p->mask_row_stride : 0;
+  f.status = status;
+  return f;
+}
+
+size_t elem_size(const tri_attn_problem *p) { return p->dtype == TRI_ATTN_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------- workspace layout --
+
+struct Carver {
+  char *base;
+  size_t off = 0;
+  explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+  void *take(size_t bytes) {
+    void *p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+int64_t mask_rows(const tri_attn_problem *p, bool has_mask) {
+  return (has_mask && p->mask_row_stride == p->N) ? p->N : 1;
+}
+
+int64_t mask_words_per_row(const tri_attn_problem *p) { return ((p->N + 127) / 128) * 4; }
+
+struct FwdWs {
+  int32_t *status;
+  uint32_t *mask_bits;
+  __nv_bfloat16 *biasT;
+};
+
+// Worst case over the mask argument (a per-row mask needs N rows of bits).
+size_t carve_fwd(const tri_attn_problem *p, void *ws, bool per_row_mask, FwdWs *out) {
+  Carver c(ws);
+  FwdWs w{};
+  w.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
+  if (p->dtype == TRI_ATTN_BF16) {
+    const int64_t rows = per_row_mask ? p->N : 1;
+    w.mask_bits = static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
+    if (p->variant == TRI_ATTN_ENDING)
+      w.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * p->N * p->N));
+  }
+  if (out) *out = w;
+  return c.off;
+}
+
+struct BwdWs {
+  FwdWs fw;
+  void *du;
+  float *D;
+  float *part_dq, *part_dk, *part_dv, *part_db;
+  int ntile, ngroups;
+};
+
+size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, BwdWs *out) {
+  Carver c(ws);
+  BwdWs w{};
+  w.fw.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
+  const size_t pair = (size_t)p->N * p->N * p->H * p->c;
+  const size_t nn = (size_t)p->N * p->N;
+  if (p->dtype == TRI_ATTN_BF16) {
+    const int64_t rows = per_row_mask ? p->N : 1;
+    w.fw.mask_bits =
+        static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
+    if (p->variant == TRI_ATTN_ENDING)
+      w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
+    tri::bwd_bf16_plan((int)p->N, p->H, &w.ntile, &w.ngroups);
+    w.du = c.take(2 * pair);
+  } else {
+    tri::f32_bwd_plan(make_frame(p, nullptr, nullptr), &w.ntile, &w.ngroups);
+    w.du = c.take(4 * pair);
+  }
+  w.D = static_cast<float *>(c.take(4 * nn * p->H));
+  w.part_dq = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
+  w.part_dk = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
+  w.part_dv = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
+  w.part_db = w.ngroups > 1 ? static_cast<float *>(c.take(4 * nn * p->H * (size_t)w.ngroups))
+                            : nullptr;
+  if (out) *out = w;
+  return c.off;
+}
+
+// ------------------------------------------------------------ tensor maps --
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// A pair tensor [.., .., H, 32] bf16 seen through the frame; dimensions by
+// increasing stride (c, h, then the smaller of x/r), box = one 128 x 32 tile.
+bool encode_pair(CUtensorMap *m, const void *base, int64_t N, int64_t H, int64_t sR, int64_t sX,
+                 bool x_inner) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[4] = {32, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)N};
+  cuuint64_t strides[3] = {64, (cuuint64_t)((x_inner ? sX : sR) * 2),
+                           (cuuint64_t)((x_inner ? sR : sX) * 2)};
+  cuuint32_t box[4] = {32, 1, x_inner ? 128u : 1u, x_inner ? 1u : 128u};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Bias [H, N, N] bf16 in the variant frame (y fastest), box 64 keys x 128 queries.
+bool encode_bias(CUtensorMap *m, const void *base, int64_t N, int64_t H) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H};
+  cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(N * N * 2)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+tri_attn_status cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+}
+
+#define TRI_CHECK_PTR(p)                                   \
+  do {                                                     \
+    if (!(p) || !aligned16(p)) return TRI_ATTN_ERR_INVALID_ARG; \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int tri_attn_version(void) { return (1 << 16) | 0; }
+
+const char *tri_attn_status_string(tri_attn_status s) {
+  switch (s) {
+    case TRI_ATTN_OK: return "ok";
+    case TRI_ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case TRI_ATTN_ERR_UNSUPPORTED: return "unsupported problem";
+    case TRI_ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case TRI_ATTN_ERR_CUDA: return "CUDA call failed";
+    case TRI_ATTN_ERR_TIMEOUT: return "device wait timed out";
+    case TRI_ATTN_ERR_BOUNDS: return "device index check failed";
+  }
+  return "unknown status";
+}
+
+tri_attn_status tri_attn_fwd_workspace_size(const tri_attn_problem *prob, size_t *bytes) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!bytes) return TRI_ATTN_ERR_INVALID_ARG;
+  *bytes = carve_fwd(prob, nullptr, true, nullptr);
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status tri_attn_bwd_workspace_size(const tri_attn_problem *prob, size_t *bytes) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!bytes) return TRI_ATTN_ERR_INVALID_ARG;
+  *bytes = carve_bwd(prob, nullptr, true, nullptr);
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
+                             const void *v, const void *bias, const void *gate,
+                             const uint8_t *mask, void *out, float *lse, void *workspace,
+                             size_t workspace_bytes, tri_attn_stream_t stream_) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return TRI_ATTN_ERR_WORKSPACE;
+  const bool per_row = mask && prob->mask_row_stride == prob->N;
+  FwdWs w;
+  if (workspace_bytes < carve_fwd(prob, workspace, per_row, &w)) return TRI_ATTN_ERR_WORKSPACE;
+  if (prob->N == 0) return TRI_ATTN_OK;
+  TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
+  TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse);
+  const Frame f = make_frame(prob, mask, w.status);
+
+  if (prob->dtype == TRI_ATTN_F32) {
+    cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
+    if (e == cudaSuccess)
+      e = tri::launch_f32_fwd(f, static_cast<const float *>(q), static_cast<const float *>(k),
+                              static_cast<const float *>(v), static_cast<const float *>(bias),
+                              static_cast<const float *>(gate), static_cast<float *>(out), lse,
+                              stream);
+    return cuda_status(e);
+  }
+
+  const int64_t words = mask_words_per_row(prob);
+  const int64_t rows = mask_rows(prob, mask != nullptr);
+  const bool x_inner = prob->variant == TRI_ATTN_STARTING;
+  tri::FwdMaps maps;
+  const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.biasT : bias;
+  if (!encode_pair(&maps.q, q, prob->N, prob->H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.k, k, prob->N, prob->H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.v, v, prob->N, prob->H, f.sR, f.sX, x_inner) ||
+      !encode_bias(&maps.bias, bias_frame, prob->N, prob->H))
+    return TRI_ATTN_ERR_CUDA;
+  tri::FwdArgs a;
+  a.N = f.N;
+  a.H = f.H;
+  a.x_inner = x_inner ? 1 : 0;
+  a.scale = 1.0f / sqrtf((float)prob->c);
+  a.sR = f.sR;
+  a.sX = f.sX;
+  a.gate = static_cast<const __nv_bfloat16 *>(gate);
+  a.out = static_cast<__nv_bfloat16 *>(out);
+  a.lse = lse;
+  a.mask_bits = w.mask_bits;
+  a.mask_bits_stride = rows > 1 ? words : 0;
+  a.status = w.status;
+  cudaError_t e = tri::launch_mask_bits(f, w.mask_bits, rows, words, w.status, stream);
+  if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
+    e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.biasT, f.N, f.H,
+                                   stream);
+  if (e == cudaSuccess) e = tri::launch_fwd_bf16(maps, a, stream);
+  return cuda_status(e);
+}
+
+tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const void *k,
+                             const void *v, const void *bias, const void *gate,
+                             const uint8_t *mask, const void *out, const float *lse,
+                             const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                             void *dgate, void *workspace, size_t workspace_bytes,
+                             tri_attn_stream_t stream_) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
+    return TRI_ATTN_ERR_WORKSPACE;
+  const bool per_row = mask && prob->mask_row_stride == prob->N;
+  BwdWs w;
+  if (workspace_bytes < carve_bwd(prob, workspace, per_row, &w)) return TRI_ATTN_ERR_WORKSPACE;
+  if (prob->N == 0) return TRI_ATTN_OK;
+  TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
+  TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse); TRI_CHECK_PTR(dout);
+  TRI_CHECK_PTR(dq); TRI_CHECK_PTR(dk); TRI_CHECK_PTR(dv); TRI_CHECK_PTR(dbias);
+  TRI_CHECK_PTR(dgate);
+  const Frame f = make_frame(prob, mask, w.fw.status);
+
+  if (prob->dtype == TRI_ATTN_F32) {
+    tri::F32BwdScratch s;
+    s.du = static_cast<float *>(w.du);
+    s.D = w.D;
+    s.part_dq = w.part_dq;
+    s.part_dk = w.part_dk;
+    s.part_dv = w.part_dv;
+    s.part_db = w.part_db;
+    s.ntile = w.ntile;
+    s.ngroups = w.ngroups;
+    cudaError_t e = cudaMemsetAsync(w.fw.status, 0, sizeof(int32_t), stream);
+    if (e == cudaSuccess)
+      e = tri::launch_f32_bwd(
+          f, static_cast<const float *>(q), static_cast<const float *>(k),
+          static_cast<const float *>(v), static_cast<const float *>(bias),
+          static_cast<const float *>(gate), static_cast<const float *>(out), lse,
+          static_cast<const float *>(dout), static_cast<float *>(dq), static_cast<float *>(dk),
+          static_cast<float *>(dv), static_cast<float *>(dbias), static_cast<float *>(dgate), s,
+          stream);
+    return cuda_status(e);
+  }
+
+  const int64_t words = mask_words_per_row(prob);
+  const int64_t rows = mask_rows(prob, mask != nullptr);
+  const bool x_inner = prob->variant == TRI_ATTN_STARTING;
+  const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.fw.biasT : bias;
+  const int64_t N = prob->N, H = prob->H;
+  tri::BwdMaps maps;
+  if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.v, v, N, H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.du, w.du, N, H, N * H * 32, H * 32, true) ||
+      !encode_bias(&maps.bias, bias_frame, N, H))
+    return TRI_ATTN_ERR_CUDA;
+  tri::BwdArgs a;
+  a.N = f.N;
+  a.H = f.H;
+  a.x_inner = x_inner ? 1 : 0;
+  a.scale = 1.0f / sqrtf((float)prob->c);
+  a.lse = lse;
+  a.D = w.D;
+  a.mask_bits = w.fw.mask_bits;
+  a.mask_bits_stride = rows > 1 ? words : 0;
+  a.part_dq = w.part_dq;
+  a.part_dk = w.part_dk;
+  a.part_dv = w.part_dv;
+  a.part_db = w.part_db;
+  a.dbias = static_cast<__nv_bfloat16 *>(dbias);
+  a.bX = f.bX;
+  a.bY = f.bY;
+  a.ngroups = w.ngroups;
+  a.rows_per_group = (f.N + w.ngroups - 1) / w.ngroups;
+  a.status = w.fw.status;
+
+  cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, stream);
+  if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
+    e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.fw.biasT, f.N,
+                                   f.H, stream);
+  if (e == cudaSuccess)
+    e = tri::launch_bwd_pre_bf16(f, static_cast<const __nv_bfloat16 *>(gate),
+                                 static_cast<const __nv_bfloat16 *>(out),
+                                 static_cast<const __nv_bfloat16 *>(dout),
+                                 static_cast<__nv_bfloat16 *>(w.du), w.D,
+                                 static_cast<__nv_bfloat16 *>(dgate), stream);
+  if (e == cudaSuccess) e = tri::launch_bwd_bf16(maps, a, stream);
+  const float scale = 1.0f / sqrtf((float)prob->c);
+  if (e == cudaSuccess)
+    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dq, w.ntile, scale,
+                                               static_cast<__nv_bfloat16 *>(dq), stream);
+  if (e == cudaSuccess)
+    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dk, w.ntile, scale,
+                                               static_cast<__nv_bfloat16 *>(dk), stream);
+  if (e == cudaSuccess)
+    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dv, w.ntile, 1.0f,
+                                               static_cast<__nv_bfloat16 *>(dv), stream);
+  if (e == cudaSuccess && w.ngroups > 1)
+    e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, w.ngroups,
+                                               static_cast<__nv_bfloat16 *>(dbias), stream);
+  return cuda_status(e);
+}
+
+tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_status,
+                                     tri_attn_stream_t stream_) {
+  if (!workspace || !device_status) return TRI_ATTN_ERR_INVALID_ARG;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int32_t v = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return TRI_ATTN_ERR_CUDA;
+  *device_status = v;
+  return TRI_ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// Launch interfaces of the bf16 tcgen05 kernels (forward, backward) and of
+// the small preparation kernels they share.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace tri {
+
+// ------------------------------------------------------------------ forward --
+// Pair-tensor maps list their dimensions by increasing stride: (c, h, x, r)
+// when the query index has the smaller stride (x_inner = 1, starting node),
+// else (c, h, r, x); the box is 32 channels x 1 head x 128 queries x 1 row, so
+// a tile lands in shared memory as 128 rows of 64 bytes (64-byte swizzle).
+// The bias map is (y, x, h) in the variant frame, box (64, 128, 1), 128-byte
+// swizzle.
+struct FwdMaps {
+  CUtensorMap q, k, v;
+  CUtensorMap bias;
+};
+
+struct FwdArgs {
+  int N, H;
+  int x_inner;                       // dimension order of the pair maps (see above)
+  float scale;                       // c^-1/2
+  int64_t sR, sX;                    // pair strides of the variant frame (elements)
+  const __nv_bfloat16 *gate;
+  __nv_bfloat16 *out;
+  float *lse;
+  const uint32_t *mask_bits;         // [rows][ceil(N/128)*4] key bits, 0 beyond N
+  int64_t mask_bits_stride;          // words per attention row (0: shared by all rows)
+  int32_t *status;
+};
+
+int fwd_bf16_rows_per_cta();
+cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream);
+
+// ----------------------------------------------------------------- backward --
+struct BwdMaps {
+  CUtensorMap q, k, v;   // as for the forward
+  CUtensorMap du;        // dU = dout * sigmoid(g), compact variant frame, dims (c, h, x, r)
+  CUtensorMap bias;
+};
+
+struct BwdArgs {
+  int N, H;
+  int x_inner;
+  float scale;
+  const float *lse;                  // [N, H, N] natural log
+  const float *D;                    // [N, H, N] sum_c dout * out
+  const uint32_t *mask_bits;
+  int64_t mask_bits_stride;
+  float *part_dq;                    // [nyb][N, N, H, 32] compact variant frame
+  float *part_dk;                    // [nxb][...]
+  float *part_dv;                    // [nxb][...]
+  float *part_db;                    // [ngroups][H, N, N] variant frame (ngroups > 1)
+  __nv_bfloat16 *dbias;              // final dbias (ngroups == 1)
+  int64_t bX, bY;                    // dbias strides of the variant frame
+  int ngroups, rows_per_group;
+  int32_t *status;
+};
+
+void bwd_bf16_plan(int N, int H, int *nxb, int *ngroups);
+cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream_t stream);
+
+// ------------------------------------------------------------ preparation --
+// Packs the key mask of every attention row into bits (0 beyond N) and resets
+// the status word. rows = N for a per-row mask, 1 for a shared one.
+cudaError_t launch_mask_bits(const Frame &f, uint32_t *bits, int64_t rows, int64_t words_per_row,
+                             int32_t *status, cudaStream_t stream);
+// biasT[h][x][y] = bias[h][y][x] (bf16), for the ending-node variant.
+cudaError_t launch_bias_transpose(const __nv_bfloat16 *bias, __nv_bfloat16 *biasT, int N, int H,
+                                  cudaStream_t stream);
+// du (compact variant frame, bf16) = dout * sigmoid(g); D = sum_c dout * out;
+// dgate (storage layout) = dout * out * (1 - sigmoid(g)).
+cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
+                                const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
+                                __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
+                                cudaStream_t stream);
+
+}  // namespace tri

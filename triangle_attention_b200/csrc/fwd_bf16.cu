@@ -1,0 +1,426 @@
+// bf16 forward of gated triangle self-attention on sm_100a (tcgen05 + TMA).
+//
+// Work unit: one CTA owns (query tile of 128, head h, group of R attention
+// rows). The N^3*H logits never leave the chip: for each key tile the CTA
+// stages the 128x128 pair-bias tile once by TMA (shared by all R rows, since
+// the bias does not depend on the row) and then, row by row, computes
+// S = Q K^T on the tensor cores into tensor memory, turns it into
+// probabilities with an online softmax, and accumulates O += P V in tensor
+// memory. The probabilities never exist as a whole: each tile is produced and
+// consumed on chip ("MegaFold: Efficient Training of Next-Generation 3D
+// Attention Protein Models on Cross-Platform GPUs", tool 1, EvoFlash-3D). The
+// sigmoid gate, the key mask and the log-sum-exp save are fused into the same
+// kernel ("HelixFold: An Efficient Implementation of AlphaFold2 using
+// PaddlePaddle", proposed methods: fused gated self-attention).
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      tensor-memory allocator and MMA issuer (one elected lane)
+//   warps 2..5  softmax / epilogue warpgroup: thread = query row of the tile
+//               (tensor-memory lane), so row max and row sum are thread-local.
+//
+// Tensor memory (512 columns): S ping-pong buffers at columns 0 and 128 (the
+// bf16 probabilities overwrite the first 64 columns of their S buffer and feed
+// the PV MMA straight from tensor memory); O accumulators of the R rows at
+// 256 + 32*rr.
+#include <cmath>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "bf16.cuh"
+#include "ptx.cuh"
+
+namespace tri {
+namespace {
+
+constexpr int kBM = 128;          // queries per tile
+constexpr int kBN = 128;          // keys per tile
+constexpr int kC = 32;            // head dimension
+constexpr int kRows = 8;          // attention rows per CTA
+constexpr int kStages = 4;        // K/V pipeline depth
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kPairTileBytes = kBM * kC * 2;   // 8 KB
+constexpr uint32_t kBiasTileBytes = kBM * kBN * 2;  // 32 KB (two 16 KB halves)
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct __align__(8) FwdSmem {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t bias_full[2];
+  uint64_t bias_empty[2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[kRows];
+  uint64_t o_final;
+  uint64_t teardown;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kRows * kPairTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kPairTileBytes;
+constexpr uint32_t kOffB = kOffV + kStages * kPairTileBytes;
+constexpr uint32_t kOffCtl = kOffB + 2 * kBiasTileBytes;
+constexpr uint32_t kSmemBytes = kOffCtl + sizeof(FwdSmem) + 1024;  // +1024 for alignment
+
+// Bounded wait on an mbarrier that also gives up once another role aborted.
+// Warp-uniform when every lane of the warp calls it.
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
+                                         volatile uint32_t *abort_flag, int32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t polls = 1; polls < kWaitMaxPolls; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+    }
+  }
+  *abort_flag = 1u;
+  report_status(status, kStatusTimeout);
+  return false;
+}
+
+__device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity,
+                                              volatile uint32_t *abort_flag, int32_t *status) {
+  const bool ok = wait_bar(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
+                const FwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  FwdSmem &ctl = *reinterpret_cast<FwdSmem *>(smem + kOffCtl);
+  volatile uint32_t *abort_flag = &ctl.abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int N = a.N;
+  const int xb = blockIdx.x, h = blockIdx.y;
+  const int r0 = blockIdx.z * kRows;
+  const int nrows = min(kRows, N - r0);
+  const int nkb = (N + kBN - 1) / kBN;
+  const int T = nkb * nrows;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl.kv_full[s], 1);
+      mbar_init(&ctl.kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl.bias_full[b], 1);
+      mbar_init(&ctl.bias_empty[b], 128);
+      mbar_init(&ctl.s_full[b], 1);
+      mbar_init(&ctl.p_full[b], 128);
+    }
+    for (int rr = 0; rr < kRows; ++rr) mbar_init(&ctl.o_done[rr], 1);
+    mbar_init(&ctl.o_final, 1);
+    mbar_init(&ctl.teardown, 1);
+    ctl.abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_b);
+      int armed_kv[kStages];
+      int armed_b[2] = {-1, -1};
+      for (int s = 0; s < kStages; ++s) armed_kv[s] = -1;
+      bool ok = true;
+      mbar_arrive_expect_tx(&ctl.q_full, nrows * kPairTileBytes);
+      for (int rr = 0; rr < nrows; ++rr) {
+        uint8_t *dst = smem + kOffQ + rr * kPairTileBytes;
+        if (a.x_inner)
+          tma_load_4d(dst, &tm_q, &ctl.q_full, 0, h, xb * kBM, r0 + rr);
+        else
+          tma_load_4d(dst, &tm_q, &ctl.q_full, 0, h, r0 + rr, xb * kBM);
+      }
+      int it = 0;
+      for (int kb = 0; kb < nkb && ok; ++kb) {
+        const int bb = kb & 1;
+        if (kb >= 2 && !wait_bar(&ctl.bias_empty[bb], ((kb >> 1) - 1) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t *bsm = smem + kOffB + bb * kBiasTileBytes;
+        mbar_arrive_expect_tx(&ctl.bias_full[bb], kBiasTileBytes);
+        tma_load_3d(bsm, &tm_b, &ctl.bias_full[bb], kb * kBN, xb * kBM, h);
+        tma_load_3d(bsm + kBiasTileBytes / 2, &tm_b, &ctl.bias_full[bb], kb * kBN + 64, xb * kBM, h);
+        armed_b[bb] = kb >> 1;
+        for (int rr = 0; rr < nrows; ++rr, ++it) {
+          const int st = it % kStages;
+          if (it >= kStages &&
+              !wait_bar(&ctl.kv_empty[st], ((it / kStages) - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&ctl.kv_full[st], 2 * kPairTileBytes);
+          uint8_t *kd = smem + kOffK + st * kPairTileBytes;
+          uint8_t *vd = smem + kOffV + st * kPairTileBytes;
+          if (a.x_inner) {
+            tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
+            tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
+          } else {
+            tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
+            tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
+          }
+          armed_kv[st] = it / kStages;
+        }
+      }
+      if (!ok) {
+        // Let every copy this thread started land before the CTA exits.
+        mbar_wait(&ctl.q_full, 0);
+        for (int s = 0; s < kStages; ++s)
+          if (armed_kv[s] >= 0) mbar_wait(&ctl.kv_full[s], armed_kv[s] & 1);
+        for (int b = 0; b < 2; ++b)
+          if (armed_b[b] >= 0) mbar_wait(&ctl.bias_full[b], armed_b[b] & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (elect_one()) {
+      const uint32_t id_s = make_idesc_bf16(kBM, kBN, false, false);
+      const uint32_t id_pv = make_idesc_bf16(kBM, kC, false, true);
+      bool ok = wait_bar(&ctl.q_full, 0, abort_flag, a.status);
+      tc_fence_after();
+      int it = 0;
+      auto issue_s = [&](int t) -> bool {
+        const int rr = t % nrows, st = t % kStages, sb = t & 1;
+        if (!wait_bar(&ctl.kv_full[st], (t / kStages) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(smem + kOffQ + rr * kPairTileBytes);
+        const uint32_t ka = smem_u32(smem + kOffK + st * kPairTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < kC / 16; ++ks) {
+          const uint64_t da = make_sdesc(qa + ks * 32, 16, 512, kSwizzle64B);
+          const uint64_t db = make_sdesc(ka + ks * 32, 16, 512, kSwizzle64B);
+          mma_ss(tmem + sb * kBN, da, db, id_s, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&ctl.s_full[sb]);
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int rr = t % nrows, kb = t / nrows, st = t % kStages, sb = t & 1;
+        if (!wait_bar(&ctl.p_full[sb], (t >> 1) & 1, abort_flag, a.status)) return false;
+        tc_fence_after();
+        const uint32_t va = smem_u32(smem + kOffV + st * kPairTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          const uint64_t db = make_sdesc(va + ks * 16 * 64, 512, 512, kSwizzle64B);
+          mma_ts(tmem + 2 * kBN + rr * kC, tmem + sb * kBN + ks * 8, db, id_pv,
+                 (kb > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&ctl.kv_empty[st]);
+        mma_commit(&ctl.o_done[rr]);
+        return true;
+      };
+      for (it = 0; ok && it < T; ++it) {
+        ok = issue_s(it);
+        if (ok && it >= 1) ok = issue_pv(it - 1);
+      }
+      if (ok && T > 0) ok = issue_pv(T - 1);
+      mma_commit(&ctl.o_final);
+      // No tensor-memory operation may be in flight when the CTA tears down.
+      mma_commit(&ctl.teardown);
+      mbar_wait(&ctl.teardown, 0);
+    }
+  } else {
+    // ------------------------------------------------ softmax and epilogue --
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;           // query within the tile = TMEM lane
+    const int x = xb * kBM + row;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const float c1 = a.scale * kLog2e;
+    float m_r[kRows], l_r[kRows];
+#pragma unroll
+    for (int rr = 0; rr < kRows; ++rr) {
+      m_r[rr] = -INFINITY;
+      l_r[rr] = 0.0f;
+    }
+    bool ok = true;
+    int it = 0;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int bb = kb & 1;
+      if (!wait_bar_warp(&ctl.bias_full[bb], (kb >> 1) & 1, abort_flag, a.status)) {
+        ok = false;
+        break;
+      }
+      const uint8_t *brow = smem + kOffB + bb * kBiasTileBytes + row * 128;
+#pragma unroll 1
+      for (int rr = 0; rr < kRows; ++rr) {
+        if (rr >= nrows) break;
+        const int sb = it & 1;
+        const int r = r0 + rr;
+        // key mask bits of this row and key tile (tail keys are zero bits)
+        const uint32_t *mb = a.mask_bits + (int64_t)r * a.mask_bits_stride + kb * 4;
+        const uint4 mw = *reinterpret_cast<const uint4 *>(mb);
+        const bool full_tile = (mw.x & mw.y & mw.z & mw.w) == 0xffffffffu;
+        if (!wait_bar_warp(&ctl.s_full[sb], (it >> 1) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float t[kBN];
+        {
+          uint32_t u[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_ld32(tl + sb * kBN + j * 32, u);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[j * 32 + e] = __uint_as_float(u[e]);
+          }
+        }
+        // logits in the log2 domain: s*c^-1/2*log2e + b*log2e, masked -> -inf
+        float mx = -INFINITY;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+          const int hh = ch >> 3, cc = ch & 7;
+          const uint4 bv = *reinterpret_cast<const uint4 *>(brow + hh * (kBiasTileBytes / 2) +
+                                                            ((cc ^ (row & 7)) << 4));
+          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = ch * 8 + e * 2;
+            t[j] = fmaf(t[j], c1, bf16lo(bw[e]) * kLog2e);
+            t[j + 1] = fmaf(t[j + 1], c1, bf16hi(bw[e]) * kLog2e);
+          }
+        }
+        if (!full_tile) {
+          const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
+#pragma unroll
+          for (int j = 0; j < kBN; ++j)
+            if (!((mws[j >> 5] >> (j & 31)) & 1u)) t[j] = -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < kBN; ++j) mx = fmaxf(mx, t[j]);
+        const float m_new = fmaxf(m_r[rr], mx);
+        const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
+        const float alpha = ex2_approx(m_r[rr] - m_use);
+        float sum = 0.0f;
+        uint32_t pk[kBN / 2];
+#pragma unroll
+        for (int j = 0; j < kBN; j += 2) {
+          const float p0 = ex2_approx(t[j] - m_use);
+          const float p1 = ex2_approx(t[j + 1] - m_use);
+          sum += p0 + p1;
+          pk[j / 2] = pack_bf16(p0, p1);
+        }
+        l_r[rr] = l_r[rr] * alpha + sum;
+        m_r[rr] = m_new;
+        {
+          uint32_t w0[32], w1[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            w0[e] = pk[e];
+            w1[e] = pk[32 + e];
+          }
+          tmem_st32(tl + sb * kBN, w0);
+          tmem_st32(tl + sb * kBN + 32, w1);
+        }
+        if (kb > 0) {
+          // rescale the running output once the previous PV of this row is done
+          if (!wait_bar_warp(&ctl.o_done[rr], (kb - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            uint32_t o[32];
+            const uint32_t oa = tl + 2 * kBN + rr * kC;
+            tmem_ld32(oa, o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(oa, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&ctl.p_full[sb]);
+        ++it;
+      }
+      if (ok) mbar_arrive(&ctl.bias_empty[bb]);
+    }
+    // epilogue: out = sigmoid(g) * O / l (bf16), lse = ln(sum exp s)
+    if (ok) ok = wait_bar_warp(&ctl.o_final, 0, abort_flag, a.status);
+    if (ok) tc_fence_after();
+    for (int rr = 0; rr < nrows; ++rr) {
+      const int r = r0 + rr;
+      uint32_t o[32];
+      if (ok) tmem_ld32(tl + 2 * kBN + rr * kC, o);
+      if (x >= N) continue;
+      float *lse_p = a.lse + ((int64_t)r * a.H + h) * N + x;
+      if (!ok) {
+        *lse_p = __int_as_float(0x7fc00000);  // NaN marks a tile the kernel gave up on
+        continue;
+      }
+      const float l = l_r[rr];
+      const float inv = l > 0.0f ? rcp_approx(l) : 0.0f;
+      const int64_t off = (int64_t)r * a.sR + (int64_t)x * a.sX + (int64_t)h * kC;
+      const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + off);
+      uint4 *op = reinterpret_cast<uint4 *>(a.out + off);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        const uint4 gv = gp[v4];
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int cc = v4 * 8 + e * 2;
+          const float g0 = bf16lo(gw[e]), g1 = bf16hi(gw[e]);
+          const float s0 = rcp_approx(1.0f + ex2_approx(-g0 * kLog2e));
+          const float s1 = rcp_approx(1.0f + ex2_approx(-g1 * kLog2e));
+          ow[e] = pack_bf16(s0 * __uint_as_float(o[cc]) * inv, s1 * __uint_as_float(o[cc + 1]) * inv);
+        }
+        op[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+      *lse_p = l > 0.0f ? (m_r[rr] + lg2_approx(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int fwd_bf16_rows_per_cta() { return kRows; }
+
+cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream) {
+  if (args.N == 0) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((args.N + kBM - 1) / kBM, args.H, (args.N + kRows - 1) / kRows);
+  fwd_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k, maps.v, maps.bias,
+                                                           args);
+  return cudaGetLastError();
+}
+
+}  // namespace tri

@@ -1,0 +1,135 @@
+// Preparation kernels of the bf16 path: key-mask bit packing, the transposed
+// bias of the ending-node variant, and the backward preprocess that turns
+// (dout, out, gate) into dU, D and dgate.
+#include <cmath>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "bf16.cuh"
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace tri {
+namespace {
+
+int blocks_for(int64_t n, int threads) {
+  int64_t b = (n + threads - 1) / threads;
+  if (b > 148 * 64) b = 148 * 64;
+  return (int)(b < 1 ? 1 : b);
+}
+
+// One word = 32 keys of one attention row; bit j set when key 32*w + j exists
+// and takes part. Also resets the call's status word.
+__global__ void mask_bits_kernel(Frame f, uint32_t *__restrict__ bits, int64_t rows,
+                                 int64_t words_per_row, int32_t *status) {
+  if (blockIdx.x == 0 && threadIdx.x == 0 && status) *status = kStatusOk;
+  const int64_t total = rows * words_per_row;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = w / words_per_row;
+    const int64_t y0 = (w % words_per_row) * 32;
+    uint32_t b = 0;
+    for (int j = 0; j < 32; ++j) {
+      const int64_t y = y0 + j;
+      if (y < f.N && (!f.mask || f.mask[r * f.mask_stride + y] != 0)) b |= 1u << j;
+    }
+    bits[w] = b;
+  }
+}
+
+__global__ void bias_transpose_kernel(const __nv_bfloat16 *__restrict__ in,
+                                      __nv_bfloat16 *__restrict__ out, int N) {
+  __shared__ __nv_bfloat16 t[32][33];
+  const int64_t hb = (int64_t)blockIdx.z * N * N;
+  const int bx = blockIdx.x * 32, by = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int row = by + i, col = bx + threadIdx.x;
+    if (row < N && col < N) t[i][threadIdx.x] = in[hb + (int64_t)row * N + col];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int row = bx + i, col = by + threadIdx.x;
+    if (row < N && col < N) out[hb + (int64_t)row * N + col] = t[threadIdx.x][i];
+  }
+}
+
+__device__ __forceinline__ float sigmoid_fast(float g) {
+  return rcp_approx(1.0f + ex2_approx(-g * 1.4426950408889634f));
+}
+
+// One thread per (storage row a, storage column b, head h): 32 channels.
+__global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ gate,
+                                    const __nv_bfloat16 *__restrict__ out,
+                                    const __nv_bfloat16 *__restrict__ dout,
+                                    __nv_bfloat16 *__restrict__ du, float *__restrict__ D,
+                                    __nv_bfloat16 *__restrict__ dgate, int ending) {
+  const int64_t total = (int64_t)f.N * f.N * f.H;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int h = (int)(w % f.H);
+    const int64_t b = (w / f.H) % f.N;
+    const int64_t aa = w / ((int64_t)f.H * f.N);
+    const int64_t r = ending ? b : aa;
+    const int64_t x = ending ? aa : b;
+    const int64_t so = w * 32;                                 // storage offset
+    const int64_t co = (((r * f.N + x) * f.H) + h) * 32;      // compact variant frame
+    const uint4 *gp = reinterpret_cast<const uint4 *>(gate + so);
+    const uint4 *op = reinterpret_cast<const uint4 *>(out + so);
+    const uint4 *dp = reinterpret_cast<const uint4 *>(dout + so);
+    uint4 *up = reinterpret_cast<uint4 *>(du + co);
+    uint4 *gq = reinterpret_cast<uint4 *>(dgate + so);
+    float d = 0.0f;
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint4 g4 = gp[v], o4 = op[v], d4 = dp[v];
+      const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+      const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+      const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+      uint32_t uw[4], rw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float s0 = sigmoid_fast(bf16lo(gw[e])), s1 = sigmoid_fast(bf16hi(gw[e]));
+        const float d0 = bf16lo(dw[e]), d1 = bf16hi(dw[e]);
+        const float o0 = bf16lo(ow[e]), o1 = bf16hi(ow[e]);
+        d = fmaf(d0, o0, d);
+        d = fmaf(d1, o1, d);
+        uw[e] = pack_bf16(d0 * s0, d1 * s1);
+        rw[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
+      }
+      up[v] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+      gq[v] = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+    }
+    D[(r * f.H + h) * f.N + x] = d;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_mask_bits(const Frame &f, uint32_t *bits, int64_t rows, int64_t words_per_row,
+                             int32_t *status, cudaStream_t stream) {
+  mask_bits_kernel<<<blocks_for(rows * words_per_row, 256), 256, 0, stream>>>(
+      f, bits, rows, words_per_row, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_transpose(const __nv_bfloat16 *bias, __nv_bfloat16 *biasT, int N, int H,
+                                  cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  dim3 grid((N + 31) / 32, (N + 31) / 32, H);
+  bias_transpose_kernel<<<grid, dim3(32, 8), 0, stream>>>(bias, biasT, N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
+                                const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
+                                __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
+                                cudaStream_t stream) {
+  const int64_t total = (int64_t)f.N * f.N * f.H;
+  if (total == 0) return cudaSuccess;
+  const int ending = f.variant == 1 ? 1 : 0;
+  bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, dout, du, D,
+                                                                  dgate, ending);
+  return cudaGetLastError();
+}
+
+}  // namespace tri
