@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Benchmark of gated triangle self-attention, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward and one backward call (every kernel of the path) over
+one batch of synthetic inputs: N=768 residues, H=4 heads, c=32, bf16, starting
+node, no mask, inputs drawn by tri_inputs (seeded). The metric counts
+4*N^3*H*c forward and 10*N^3*H*c backward FLOPs per step. Inputs (755 MB of
+pair tensors, 5.6 GB of workspace) are larger than the 126 MB L2, so no flush
+is needed between steps.
+
+With N > 1 GPUs (torchrun, one process per GPU) every rank runs its own
+independent problem (weak scaling); ranks share only a barrier and a max of
+the elapsed time. `--impl reference` times the fp64 CPU oracle on this host's
+cores instead (rank 0 only), on bounded samples of attention rows.
+
+Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import tri_inputs  # noqa: E402
+
+WORKLOAD = "n768_bf16"
+METRIC = "triangle-attention fwd+bwd TFLOP/s at N=768 bf16 (% of B200 BF16 peak)"
+UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0
+
+
+def flops(N: int, H: int, c: int) -> tuple:
+    n3 = float(N) ** 3 * H * c
+    return 4.0 * n3, 10.0 * n3
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def config_dict(w) -> dict:
+    return {"workload": w.name, "N": w.N, "H": w.H, "c": w.c, "dtype": w.dtype,
+            "variant": "starting", "mask": w.mask, "seed": w.seed,
+            "l2": "inputs larger than L2 (755 MB pair tensors + 5.6 GB workspace per step)",
+            "parallelism": "independent replica per GPU"}
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self, wait_s: float = 20.0):
+        """Start sampling and wait for the first sample, so that nvidia-smi's own
+        start-up (which can stall other driver clients) ends before timing."""
+        import threading
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        first = threading.Event()
+
+        def reader():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+                first.set()
+            first.set()
+
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        first.wait(wait_s)
+
+    def mark(self):
+        """Index of the first sample taken inside the timed region."""
+        self.begin = len(self.lines)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        end = len(self.lines)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        out = "".join(self.lines[getattr(self, "begin", 0):max(end, getattr(self, "begin", 0) + 1)])
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- distributed --
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+def oracle_threads() -> int:
+    env = os.environ.get("OMP_NUM_THREADS")
+    return int(env) if env and env.isdigit() else (os.cpu_count() or 1)
+
+
+def oracle_inputs(d) -> dict:
+    """The workload's tensors widened once to float32 numpy (exact for bf16), so
+    the oracle calls below time arithmetic, not conversion."""
+    out = {}
+    for k, v in d.items():
+        if torch.is_tensor(v):
+            v = v.to(torch.float32).numpy() if v.is_floating_point() else v.numpy()
+        out[k] = v
+    return out
+
+
+def oracle_rows_step(d, rows) -> float:
+    """fp64 oracle forward + backward of the listed attention rows; seconds."""
+    import oracle
+    args = (d["q"], d["k"], d["v"], d["bias"], d["gate"])
+    t0 = time.perf_counter()
+    oracle.fwd(*args, d["mask"], tri_inputs.STARTING, rows=rows)
+    oracle.bwd(*args, d["dout"], d["mask"], tri_inputs.STARTING, rows=rows)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(d, w, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands, on this host's cores, on a bounded sample of
+    attention rows of the same workload (whole rows: every head, query, key)."""
+    d = oracle_inputs(d)
+    cores = oracle_threads()
+    rows_per_call = max(2, 2 * ((cores + w.H - 1) // w.H))
+    rng = np.random.default_rng(1)
+    done, secs = 0, 0.0
+    while secs < budget_s and done < w.N:
+        rows = rng.choice(w.N, size=min(rows_per_call, w.N), replace=False)
+        secs += oracle_rows_step(d, rows)
+        done += len(rows)
+    f_fwd, f_bwd = flops(w.N, w.H, w.c)
+    unit_flops = (f_fwd + f_bwd) / w.N          # one attention row, all heads
+    return {"value": unit_flops * done / secs / 1e12, "unit": UNIT, "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} of {w.N} attention rows (all heads), fp64 forward+backward, "
+                      f"{secs:.1f} s"}
+
+
+def run_reference(args, rank, world, w):
+    """The oracle on host cores, each step a bounded sample of attention rows."""
+    if rank != 0:
+        return None
+    d = oracle_inputs(tri_inputs.workload_inputs(w.name))
+    cores = oracle_threads()
+    t_row = oracle_rows_step(d, [0]) + 1e-9     # calibration, also warms the library
+    budget_s = args.ref_budget_s
+    per_step = budget_s / max(1, args.steps + args.warmup)
+    rows_per_step = int(max(1, min(w.N, round(per_step / t_row))))
+    rng = np.random.default_rng(2)
+    for _ in range(args.warmup):
+        oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
+    secs = 0.0
+    for _ in range(args.steps):
+        secs += oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
+    f_fwd, f_bwd = flops(w.N, w.H, w.c)
+    unit_flops = (f_fwd + f_bwd) / w.N
+    value = unit_flops * rows_per_step * args.steps / secs / 1e12
+    sample = (f"{rows_per_step} of {w.N} attention rows (all heads) per step, fp64 "
+              f"forward+backward")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------- our arm --
+
+def traffic_record(kernel: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary, or None
+    if the kernel's source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = {"fwd_bf16_kernel": "fwd_bf16.cu", "bwd_bf16_kernel": "bwd_bf16.cu"}[kernel]
+    h = hashlib.sha256(open(os.path.join(ROOT, "triangle_attention_b200", "csrc", src),
+                            "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 3 and parts[0] == kernel and parts[1] == h:
+            return float(parts[2])
+    return None
+
+
+def run_ours(args, rank, world, local, w):
+    import triangle_attention_b200 as ta
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = tri_inputs.workload_inputs(w.name, seed=w.seed + rank)
+    g = {k: (v.to(dev).contiguous() if torch.is_tensor(v) else v) for k, v in d.items()}
+    q, k, v, bias, gate, dout, mask = (g[n] for n in ("q", "k", "v", "bias", "gate", "dout",
+                                                      "mask"))
+    prob = ta.problem(q, mask, ta.STARTING)
+    ws_f = ta.workspace(ta.fwd_workspace_size(prob), dev)
+    ws_b = ta.workspace(ta.bwd_workspace_size(prob), dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.N, w.H, w.N), dtype=torch.float32, device=dev)
+    grads = tuple(torch.empty_like(t) for t in (q, k, v, bias, gate))
+    stream = torch.cuda.current_stream()
+    launches_per_step = (ta.kernel_launches(prob, False, mask is not None) +
+                         ta.kernel_launches(prob, True, mask is not None))
+
+    def step(opts_f=None, opts_b=None):
+        ta.fwd(q, k, v, bias, gate, mask, ta.STARTING, out=out, lse=lse, ws=ws_f, opts=opts_f)
+        ta.bwd(q, k, v, bias, gate, mask, out, lse, dout, ta.STARTING, grads=grads, ws=ws_b,
+               opts=opts_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ta.read_status(ws_f) or ta.read_status(ws_b):
+        raise RuntimeError("device status reported a failure during warm-up")
+
+    # per-step events around the two main kernels
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    opts = [(ta.launch_opts(e[0], e[1]), ta.launch_opts(e[2], e[3])) for e in ev]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+
+    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
+    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(*opts[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    status = ta.read_status(ws_f) | ta.read_status(ws_b)
+    if status:
+        raise RuntimeError(f"device status {status} in the timed region")
+
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    f_fwd, f_bwd = flops(w.N, w.H, w.c)
+    value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+
+    # roofline of the dominant kernel: algorithmic FLOPs per launch / launch time
+    peaks = load_peaks()
+    if bwd_ms >= fwd_ms:
+        kname, kms, kflops = "bwd_bf16_kernel", bwd_ms, f_bwd
+    else:
+        kname, kms, kflops = "fwd_bf16_kernel", fwd_ms, f_fwd
+    achieved = kflops / (kms * 1e-3) / 1e12
+    traffic = traffic_record(kname)
+    roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
+                "peak": peaks["bf16_tflops"], "unit": UNIT,
+                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 matmul (burst)"}
+
+    # end to end through the public API with pinned host buffers
+    e2e_steps = max(3, min(args.steps, 10))
+    host_in = {n: d[n].pin_memory() for n in ("q", "k", "v", "bias", "gate", "dout")}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                for n, t in (("out", out), ("lse", lse), ("dq", grads[0]), ("dk", grads[1]),
+                             ("dv", grads[2]), ("dbias", grads[3]), ("dgate", grads[4]))}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    dev_in = {n: g[n] for n in host_in}
+
+    def e2e_step():
+        for n, t in host_in.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        ta.fwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["bias"], dev_in["gate"], mask,
+               ta.STARTING, out=out, lse=lse, ws=ws_f)
+        ta.bwd(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["bias"], dev_in["gate"], mask, out,
+               lse, dev_in["dout"], ta.STARTING, grads=grads, ws=ws_b)
+        for n, t in zip(("out", "lse", "dq", "dk", "dv", "dbias", "dgate"),
+                        (out, lse) + grads):
+            host_out[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * (f_fwd + f_bwd) / (e2e_ms * 1e-3) / 1e12
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) pair tensors, tri_inputs)",
+            "config": config_dict(w),
+            "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
+            "pct_of_measured_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+            "kernels": {"fwd_bf16_kernel_ms": fwd_ms, "bwd_bf16_kernel_ms": bwd_ms,
+                        "step_ms": ms_local},
+            "roofline": roofline,
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(d, w)
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=150.0,
+                    help="host seconds the reference arm spends over all its steps")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+    w = tri_inputs.WORKLOADS[args.workload]
+    if not w.backward:
+        ap.error("the benchmark step is forward + backward; pick a workload with a backward")
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, rank, world, w)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    rank, world, local = dist_setup()
+    try:
+        line = run_ours(args, rank, world, local, w)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

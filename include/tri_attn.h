@@ -143,6 +143,44 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
                              tri_attn_stream_t stream);
 
 /*
+ * Optional per-call settings of the _ex entry points. Zero-initialise, set
+ * struct_size = sizeof(tri_attn_launch_opts), then fill what is needed.
+ *   main_start / main_stop: cudaEvent_t handles (or NULL) that the call
+ *   records on its stream immediately before and after its main kernel (the
+ *   attention kernel itself, without the small preparation and reduction
+ *   kernels), so a caller can time that kernel alone with cudaEventElapsedTime.
+ */
+typedef struct {
+    uint32_t struct_size;
+    uint32_t flags;           /* reserved, must be 0 */
+    void *main_start;
+    void *main_stop;
+} tri_attn_launch_opts;
+
+/* tri_attn_fwd with options (opts may be NULL: same as tri_attn_fwd). */
+tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, void *out, float *lse, void *workspace,
+                                size_t workspace_bytes, tri_attn_stream_t stream,
+                                const tri_attn_launch_opts *opts);
+
+/* tri_attn_bwd with options (opts may be NULL: same as tri_attn_bwd). */
+tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, const void *out, const float *lse,
+                                const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                                void *dgate, void *workspace, size_t workspace_bytes,
+                                tri_attn_stream_t stream, const tri_attn_launch_opts *opts);
+
+/*
+ * Number of kernel launches one call of the forward (backward = 0) or the
+ * backward (backward = 1) enqueues for this problem and mask kind
+ * (has_mask != 0 for a non-NULL mask). Writes *launches; host-only.
+ */
+tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backward,
+                                         int has_mask, int32_t *launches);
+
+/*
  * Device status word of the last call that used this workspace: synchronises
  * the stream, copies the word to the host and stores a tri_attn_status in
  * *device_status. Returns TRI_ATTN_ERR_CUDA if the copy itself fails.

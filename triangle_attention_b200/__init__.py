@@ -41,6 +41,22 @@ class TriAttnError(RuntimeError):
         self.code = code
 
 
+class LaunchOpts(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
+                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p)]
+
+
+def launch_opts(main_start=None, main_stop=None) -> LaunchOpts:
+    """Options whose torch.cuda.Event objects are recorded around the main kernel."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if not ev.cuda_event:            # torch creates the event lazily
+            ev.record()
+        return ctypes.c_void_p(ev.cuda_event)
+    return LaunchOpts(ctypes.sizeof(LaunchOpts), 0, handle(main_start), handle(main_stop))
+
+
 class Problem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int32), ("c", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("variant", ctypes.c_int32),
@@ -63,11 +79,17 @@ def lib():
         L.tri_attn_status_string.restype = ctypes.c_char_p
         L.tri_attn_fwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
         L.tri_attn_bwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
+        PO = ctypes.POINTER(LaunchOpts)
         L.tri_attn_fwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, sz, P]
         L.tri_attn_bwd.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.tri_attn_fwd_ex.argtypes = [PP, P, P, P, P, P, P, P, P, P, sz, P, PO]
+        L.tri_attn_bwd_ex.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, PO]
+        L.tri_attn_kernel_launches.argtypes = [PP, ctypes.c_int, ctypes.c_int,
+                                               ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
-                  L.tri_attn_bwd, L.tri_attn_read_status):
+                  L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
+                  L.tri_attn_kernel_launches, L.tri_attn_read_status):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -124,6 +146,14 @@ def bwd_workspace_size(prob: Problem) -> int:
     return n.value
 
 
+def kernel_launches(prob: Problem, backward: bool, has_mask: bool) -> int:
+    """Kernel launches one forward (backward=False) or backward call enqueues."""
+    n = ctypes.c_int32(0)
+    _check(lib().tri_attn_kernel_launches(ctypes.byref(prob), int(backward), int(has_mask),
+                                          ctypes.byref(n)), "tri_attn_kernel_launches")
+    return n.value
+
+
 def workspace(nbytes: int, device) -> torch.Tensor:
     """A device buffer for the library's scratch (torch allocations are
     256-byte aligned)."""
@@ -137,7 +167,7 @@ def _contig(*ts):
 
 
 def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=None, ws=None,
-        stream=None):
+        stream=None, opts: Optional[LaunchOpts] = None):
     """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N]."""
     _contig(q, k, v, bias, gate, mask)
     prob = problem(q, mask, variant)
@@ -148,14 +178,15 @@ def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=N
         lse = torch.empty((N, H, N), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = workspace(fwd_workspace_size(prob), q.device)
-    _check(lib().tri_attn_fwd(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
-                              _p(mask), _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream)),
+    _check(lib().tri_attn_fwd_ex(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
+                                 _p(mask), _p(out), _p(lse), _p(ws), ws.numel(), _stream(stream),
+                                 None if opts is None else ctypes.byref(opts)),
            "tri_attn_fwd")
     return out, lse
 
 
 def bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, grads=None, ws=None,
-        stream=None):
+        stream=None, opts: Optional[LaunchOpts] = None):
     """Backward. Returns (dq, dk, dv, dbias, dgate) in the inputs' dtype."""
     _contig(q, k, v, bias, gate, mask, out, lse, dout)
     prob = problem(q, mask, variant)
@@ -165,9 +196,10 @@ def bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, grad
     dq, dk, dv, dbias, dgate = grads
     if ws is None:
         ws = workspace(bwd_workspace_size(prob), q.device)
-    _check(lib().tri_attn_bwd(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
-                              _p(mask), _p(out), _p(lse), _p(dout), _p(dq), _p(dk), _p(dv),
-                              _p(dbias), _p(dgate), _p(ws), ws.numel(), _stream(stream)),
+    _check(lib().tri_attn_bwd_ex(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
+                                 _p(mask), _p(out), _p(lse), _p(dout), _p(dq), _p(dk), _p(dv),
+                                 _p(dbias), _p(dgate), _p(ws), ws.numel(), _stream(stream),
+                                 None if opts is None else ctypes.byref(opts)),
            "tri_attn_bwd")
     return dq, dk, dv, dbias, dgate
 

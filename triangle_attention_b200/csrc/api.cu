@@ -193,6 +193,14 @@ tri_attn_status cuda_status(cudaError_t e) {
   return e == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
 }
 
+// Record the caller's timing event before (start) or after (stop) the main kernel.
+cudaError_t mark(const tri_attn_launch_opts *opts, bool start, cudaStream_t stream) {
+  if (!opts) return cudaSuccess;
+  void *ev = start ? opts->main_start : opts->main_stop;
+  if (!ev) return cudaSuccess;
+  return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev), stream);
+}
+
 #define TRI_CHECK_PTR(p)                                   \
   do {                                                     \
     if (!(p) || !aligned16(p)) return TRI_ATTN_ERR_INVALID_ARG; \
@@ -233,10 +241,13 @@ tri_attn_status tri_attn_bwd_workspace_size(const tri_attn_problem *prob, size_t
   return TRI_ATTN_OK;
 }
 
-tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
-                             const void *v, const void *bias, const void *gate,
-                             const uint8_t *mask, void *out, float *lse, void *workspace,
-                             size_t workspace_bytes, tri_attn_stream_t stream_) {
+tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, void *out, float *lse, void *workspace,
+                                size_t workspace_bytes, tri_attn_stream_t stream_,
+                                const tri_attn_launch_opts *opts) {
+  if (opts && (opts->struct_size < sizeof(tri_attn_launch_opts) || opts->flags != 0))
+    return TRI_ATTN_ERR_INVALID_ARG;
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -252,11 +263,13 @@ tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const 
 
   if (prob->dtype == TRI_ATTN_F32) {
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
+    if (e == cudaSuccess) e = mark(opts, true, stream);
     if (e == cudaSuccess)
       e = tri::launch_f32_fwd(f, static_cast<const float *>(q), static_cast<const float *>(k),
                               static_cast<const float *>(v), static_cast<const float *>(bias),
                               static_cast<const float *>(gate), static_cast<float *>(out), lse,
                               stream);
+    if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
 
@@ -287,16 +300,28 @@ tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const 
   if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
     e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.biasT, f.N, f.H,
                                    stream);
+  if (e == cudaSuccess) e = mark(opts, true, stream);
   if (e == cudaSuccess) e = tri::launch_fwd_bf16(maps, a, stream);
+  if (e == cudaSuccess) e = mark(opts, false, stream);
   return cuda_status(e);
 }
 
-tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const void *k,
+tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
                              const void *v, const void *bias, const void *gate,
-                             const uint8_t *mask, const void *out, const float *lse,
-                             const void *dout, void *dq, void *dk, void *dv, void *dbias,
-                             void *dgate, void *workspace, size_t workspace_bytes,
-                             tri_attn_stream_t stream_) {
+                             const uint8_t *mask, void *out, float *lse, void *workspace,
+                             size_t workspace_bytes, tri_attn_stream_t stream) {
+  return tri_attn_fwd_ex(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes,
+                         stream, nullptr);
+}
+
+tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, const void *out, const float *lse,
+                                const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                                void *dgate, void *workspace, size_t workspace_bytes,
+                                tri_attn_stream_t stream_, const tri_attn_launch_opts *opts) {
+  if (opts && (opts->struct_size < sizeof(tri_attn_launch_opts) || opts->flags != 0))
+    return TRI_ATTN_ERR_INVALID_ARG;
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
@@ -323,6 +348,7 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
     s.ntile = w.ntile;
     s.ngroups = w.ngroups;
     cudaError_t e = cudaMemsetAsync(w.fw.status, 0, sizeof(int32_t), stream);
+    if (e == cudaSuccess) e = mark(opts, true, stream);
     if (e == cudaSuccess)
       e = tri::launch_f32_bwd(
           f, static_cast<const float *>(q), static_cast<const float *>(k),
@@ -331,6 +357,7 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
           static_cast<const float *>(dout), static_cast<float *>(dq), static_cast<float *>(dk),
           static_cast<float *>(dv), static_cast<float *>(dbias), static_cast<float *>(dgate), s,
           stream);
+    if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
 
@@ -376,7 +403,9 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
                                  static_cast<const __nv_bfloat16 *>(dout),
                                  static_cast<__nv_bfloat16 *>(w.du), w.D,
                                  static_cast<__nv_bfloat16 *>(dgate), stream);
+  if (e == cudaSuccess) e = mark(opts, true, stream);
   if (e == cudaSuccess) e = tri::launch_bwd_bf16(maps, a, stream);
+  if (e == cudaSuccess) e = mark(opts, false, stream);
   const float scale = 1.0f / sqrtf((float)prob->c);
   if (e == cudaSuccess)
     e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dq, w.ntile, scale,
@@ -391,6 +420,47 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
     e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, w.ngroups,
                                                static_cast<__nv_bfloat16 *>(dbias), stream);
   return cuda_status(e);
+}
+
+tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const void *k,
+                             const void *v, const void *bias, const void *gate,
+                             const uint8_t *mask, const void *out, const float *lse,
+                             const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                             void *dgate, void *workspace, size_t workspace_bytes,
+                             tri_attn_stream_t stream) {
+  return tri_attn_bwd_ex(prob, q, k, v, bias, gate, mask, out, lse, dout, dq, dk, dv, dbias,
+                         dgate, workspace, workspace_bytes, stream, nullptr);
+}
+
+tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backward,
+                                         int has_mask, int32_t *launches) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!launches) return TRI_ATTN_ERR_INVALID_ARG;
+  (void)has_mask;
+  int32_t n = 0;
+  if (prob->N > 0) {
+    if (prob->dtype == TRI_ATTN_F32) {
+      if (!backward) {
+        n = 1;
+      } else {
+        BwdWs w;
+        carve_bwd(prob, nullptr, false, &w);
+        n = 5 + (w.ngroups > 1 ? 1 : 0);  // pre, main, three reductions, dbias reduction
+      }
+    } else {
+      const int ending = prob->variant == TRI_ATTN_ENDING ? 1 : 0;
+      if (!backward) {
+        n = 2 + ending;  // mask bits, [bias transpose], main
+      } else {
+        BwdWs w;
+        carve_bwd(prob, nullptr, false, &w);
+        n = 6 + ending + (w.ngroups > 1 ? 1 : 0);  // mask bits, pre, main, 3 reductions
+      }
+    }
+  }
+  *launches = n;
+  return TRI_ATTN_OK;
 }
 
 tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_status,
