@@ -180,6 +180,38 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
 tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backward,
                                          int has_mask, int32_t *launches);
 
+/* Size of the fixed scratch area behind tri_attn_fwd_noalloc, per GPU. */
+#define TRI_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * Forward that allocates nothing and takes no workspace. The pages describe no
+ * such entry point; it exists for callers that are not allowed to allocate
+ * device memory themselves: code inside a framework or inference engine whose
+ * allocator owns every device byte and hands out none for foreign scratch, and
+ * latency-critical loops that cannot afford the implicit device-wide
+ * synchronisation of cudaMalloc/cudaFree. Arguments, layout and results are
+ * those of tri_attn_fwd without the workspace.
+ *
+ * Scratch: a device array of TRI_ATTN_NOALLOC_SCRATCH_BYTES compiled into the
+ * library. Every GPU on which the library is used holds that array until the
+ * process exits. A problem whose tri_attn_fwd_workspace_size() exceeds it is
+ * rejected with TRI_ATTN_ERR_WORKSPACE before anything is enqueued (starting
+ * node: any size up to the N limit; ending node: H*N*N*2 bytes must also fit).
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture. The call
+ * itself never calls cudaMalloc, cudaFree or any allocating routine.
+ *
+ * All calls share the one array and leave their scratch in it; every call
+ * rewrites what it reads. Calls whose work overlaps on the GPU (other streams,
+ * other host threads) race on the array and corrupt each other's results:
+ * serialise them. A device-side failure shows as NaN in lse.
+ */
+tri_attn_status tri_attn_fwd_noalloc(const tri_attn_problem *prob, const void *q, const void *k,
+                                     const void *v, const void *bias, const void *gate,
+                                     const uint8_t *mask, void *out, float *lse,
+                                     tri_attn_stream_t stream);
+
 /*
  * Device status word of the last call that used this workspace: synchronises
  * the stream, copies the word to the host and stores a tri_attn_status in
