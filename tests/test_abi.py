@@ -70,8 +70,8 @@ def test_workspace_sizes(lib):
     rc, nb = ws_size(lib, P(N=768), "bwd")
     assert rc == 0
     pair = 768 * 768 * 4 * 32
-    # dU (bf16) + D + three sets of fp32 partials over 6 tiles
-    assert nb >= 2 * pair + 4 * 768 * 768 * 4 + 3 * 6 * 4 * pair
+    # dU (bf16) + D + three sets of bf16 tile-contribution slots over 6 tiles
+    assert nb >= 2 * pair + 4 * 768 * 768 * 4 + 3 * 6 * 2 * pair
     rc, nf = ws_size(lib, P(N=32, dtype=ta.F32), "bwd")
     assert rc == 0 and nf > 0
 

@@ -106,7 +106,11 @@ struct BwdWs {
   FwdWs fw;
   void *du;
   float *D;
-  float *part_dq, *part_dk, *part_dv, *part_db;
+  // fp32 path: partial sums per tile, reduced by a second kernel
+  float *part_dq, *part_dk, *part_dv;
+  // bf16 path: bf16 partials per tile
+  __nv_bfloat16 *bpart_q, *bpart_k, *bpart_v;
+  float *part_db;
   int ntile, ngroups;
 };
 
@@ -124,14 +128,18 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, BwdWs *
       w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
     tri::bwd_bf16_plan((int)p->N, p->H, &w.ntile, &w.ngroups);
     w.du = c.take(2 * pair);
+    w.D = static_cast<float *>(c.take(4 * nn * p->H));
+    w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+    w.bpart_k = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+    w.bpart_v = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
   } else {
     tri::f32_bwd_plan(make_frame(p, nullptr, nullptr), &w.ntile, &w.ngroups);
     w.du = c.take(4 * pair);
+    w.D = static_cast<float *>(c.take(4 * nn * p->H));
+    w.part_dq = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
+    w.part_dk = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
+    w.part_dv = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
   }
-  w.D = static_cast<float *>(c.take(4 * nn * p->H));
-  w.part_dq = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
-  w.part_dk = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
-  w.part_dv = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
   w.part_db = w.ngroups > 1 ? static_cast<float *>(c.take(4 * nn * p->H * (size_t)w.ngroups))
                             : nullptr;
   if (out) *out = w;
@@ -296,7 +304,8 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   a.mask_bits = w.mask_bits;
   a.mask_bits_stride = rows > 1 ? words : 0;
   a.status = w.status;
-  cudaError_t e = tri::launch_mask_bits(f, w.mask_bits, rows, words, w.status, stream);
+  cudaError_t e =
+      tri::launch_mask_bits(f, w.mask_bits, rows, words, w.status, nullptr, 0, stream);
   if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
     e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.biasT, f.N, f.H,
                                    stream);
@@ -377,14 +386,17 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   a.N = f.N;
   a.H = f.H;
   a.x_inner = x_inner ? 1 : 0;
+  a.nb = w.ntile;
   a.scale = 1.0f / sqrtf((float)prob->c);
+  a.sR = f.sR;
+  a.sX = f.sX;
   a.lse = lse;
   a.D = w.D;
   a.mask_bits = w.fw.mask_bits;
   a.mask_bits_stride = rows > 1 ? words : 0;
-  a.part_dq = w.part_dq;
-  a.part_dk = w.part_dk;
-  a.part_dv = w.part_dv;
+  a.part_q = w.bpart_q;
+  a.part_k = w.bpart_k;
+  a.part_v = w.bpart_v;
   a.part_db = w.part_db;
   a.dbias = static_cast<__nv_bfloat16 *>(dbias);
   a.bX = f.bX;
@@ -393,7 +405,8 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   a.rows_per_group = (f.N + w.ngroups - 1) / w.ngroups;
   a.status = w.fw.status;
 
-  cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, stream);
+  cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, nullptr,
+                                        0, stream);
   if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
     e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.fw.biasT, f.N,
                                    f.H, stream);
@@ -406,16 +419,11 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   if (e == cudaSuccess) e = mark(opts, true, stream);
   if (e == cudaSuccess) e = tri::launch_bwd_bf16(maps, a, stream);
   if (e == cudaSuccess) e = mark(opts, false, stream);
-  const float scale = 1.0f / sqrtf((float)prob->c);
   if (e == cudaSuccess)
-    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dq, w.ntile, scale,
-                                               static_cast<__nv_bfloat16 *>(dq), stream);
-  if (e == cudaSuccess)
-    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dk, w.ntile, scale,
-                                               static_cast<__nv_bfloat16 *>(dk), stream);
-  if (e == cudaSuccess)
-    e = tri::launch_pair_reduce<__nv_bfloat16>(f, w.part_dv, w.ntile, 1.0f,
-                                               static_cast<__nv_bfloat16 *>(dv), stream);
+    e = tri::launch_partial_reduce_bf16(f, w.bpart_q, w.bpart_k, w.bpart_v, w.ntile, a.scale,
+                                        static_cast<__nv_bfloat16 *>(dq),
+                                        static_cast<__nv_bfloat16 *>(dk),
+                                        static_cast<__nv_bfloat16 *>(dv), stream);
   if (e == cudaSuccess && w.ngroups > 1)
     e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, w.ngroups,
                                                static_cast<__nv_bfloat16 *>(dbias), stream);
@@ -455,7 +463,8 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
       } else {
         BwdWs w;
         carve_bwd(prob, nullptr, false, &w);
-        n = 6 + ending + (w.ngroups > 1 ? 1 : 0);  // mask bits, pre, main, 3 reductions
+        // mask bits, [transpose], pre, main, partial reduction, [dbias reduction]
+        n = 4 + ending + (w.ngroups > 1 ? 1 : 0);
       }
     }
   }

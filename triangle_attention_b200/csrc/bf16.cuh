@@ -49,14 +49,16 @@ struct BwdMaps {
 struct BwdArgs {
   int N, H;
   int x_inner;
+  int nb;                            // tiles per axis, ceil(N / 128)
   float scale;
+  int64_t sR, sX;                    // pair strides of the variant frame (outputs)
   const float *lse;                  // [N, H, N] natural log
   const float *D;                    // [N, H, N] sum_c dout * out
   const uint32_t *mask_bits;
   int64_t mask_bits_stride;
-  float *part_dq;                    // [nyb][N, N, H, 32] compact variant frame
-  float *part_dk;                    // [nxb][...]
-  float *part_dv;                    // [nxb][...]
+  // bf16 tile contributions [tile][N, N, H, 32] (compact variant frame):
+  // part_q over key tiles yb, part_k and part_v over query tiles xb
+  __nv_bfloat16 *part_q, *part_k, *part_v;
   float *part_db;                    // [ngroups][H, N, N] variant frame (ngroups > 1)
   __nv_bfloat16 *dbias;              // final dbias (ngroups == 1)
   int64_t bX, bY;                    // dbias strides of the variant frame
@@ -68,13 +70,20 @@ void bwd_bf16_plan(int N, int H, int *nxb, int *ngroups);
 cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream_t stream);
 
 // ------------------------------------------------------------ preparation --
-// Packs the key mask of every attention row into bits (0 beyond N) and resets
-// the status word. rows = N for a per-row mask, 1 for a shared one.
+// Packs the key mask of every attention row into bits (0 beyond N), resets the
+// status word and zeroes `nzero` int32 words at `zero` (counters; may be 0).
+// rows = N for a per-row mask, 1 for a shared one.
 cudaError_t launch_mask_bits(const Frame &f, uint32_t *bits, int64_t rows, int64_t words_per_row,
-                             int32_t *status, cudaStream_t stream);
+                             int32_t *status, int32_t *zero, int64_t nzero, cudaStream_t stream);
 // biasT[h][x][y] = bias[h][y][x] (bf16), for the ending-node variant.
 cudaError_t launch_bias_transpose(const __nv_bfloat16 *bias, __nv_bfloat16 *biasT, int N, int H,
                                   cudaStream_t stream);
+// dq, dk, dv (storage layout) = scale_q/k/v * sum over nb tiles of the bf16
+// partials [tile][N, N, H, 32] (compact variant frame), summed in tile order.
+cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part_q,
+                                       const __nv_bfloat16 *part_k, const __nv_bfloat16 *part_v,
+                                       int nb, float scale, __nv_bfloat16 *dq, __nv_bfloat16 *dk,
+                                       __nv_bfloat16 *dv, cudaStream_t stream);
 // du (compact variant frame, bf16) = dout * sigmoid(g); D = sum_c dout * out;
 // dgate (storage layout) = dout * out * (1 - sigmoid(g)).
 cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,

@@ -13,15 +13,19 @@
 // kernel ("HelixFold: An Efficient Implementation of AlphaFold2 using
 // PaddlePaddle", proposed methods: fused gated self-attention).
 //
-// Warp roles (192 threads):
+// Warp roles (320 threads):
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      tensor-memory allocator and MMA issuer (one elected lane)
-//   warps 2..5  softmax / epilogue warpgroup: thread = query row of the tile
-//               (tensor-memory lane), so row max and row sum are thread-local.
+//   warps 2..5  softmax / epilogue warpgroup 0: even rows of the CTA
+//   warps 6..9  softmax / epilogue warpgroup 1: odd rows
+// In a warpgroup, thread = query row of the tile (tensor-memory lane), so the
+// row max and row sum are thread-local. While one warpgroup turns its S tile
+// into probabilities, the tensor cores and the other warpgroup work on the
+// other row.
 //
-// Tensor memory (512 columns): S ping-pong buffers at columns 0 and 128 (the
-// bf16 probabilities overwrite the first 64 columns of their S buffer and feed
-// the PV MMA straight from tensor memory); O accumulators of the R rows at
+// Tensor memory (512 columns): one S buffer per warpgroup at columns 0 and 128
+// (the bf16 probabilities overwrite the first 64 columns of their S buffer and
+// feed the PV MMA straight from tensor memory); O accumulators of the 8 rows at
 // 256 + 32*rr.
 #include <cmath>
 #include <cstdint>
@@ -39,7 +43,7 @@ constexpr int kBN = 128;          // keys per tile
 constexpr int kC = 32;            // head dimension
 constexpr int kRows = 8;          // attention rows per CTA
 constexpr int kStages = 4;        // K/V pipeline depth
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kPairTileBytes = kBM * kC * 2;   // 8 KB
 constexpr uint32_t kBiasTileBytes = kBM * kBN * 2;  // 32 KB (two 16 KB halves)
@@ -65,7 +69,8 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kRows * kPairTileBytes;
 constexpr uint32_t kOffV = kOffK + kStages * kPairTileBytes;
 constexpr uint32_t kOffB = kOffV + kStages * kPairTileBytes;
-constexpr uint32_t kOffCtl = kOffB + 2 * kBiasTileBytes;
+constexpr uint32_t kOffMask = kOffB + 2 * kBiasTileBytes;   // 16 bytes of key bits per stage
+constexpr uint32_t kOffCtl = kOffMask + kStages * 16;
 constexpr uint32_t kSmemBytes = kOffCtl + sizeof(FwdSmem) + 1024;  // +1024 for alignment
 
 // Bounded wait on an mbarrier that also gives up once another role aborted.
@@ -90,6 +95,32 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity,
                                               volatile uint32_t *abort_flag, int32_t *status) {
   const bool ok = wait_bar(bar, parity, abort_flag, status);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Exponents (s*c^-1/2 + b)*log2e - m of 32 keys of this thread's query row:
+// S columns 32*c32.. from tensor memory, bias from the 128-byte-swizzled tile.
+__device__ __forceinline__ void logits32(uint32_t sbuf, const uint8_t *brow, int row, int c32,
+                                         uint64_t c1x2, uint64_t l2e2, uint64_t nm2,
+                                         float (&t)[32]) {
+  uint32_t u[32];
+  tmem_ld32(sbuf + c32 * 32, u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int ch = c32 * 4 + q;              // 16-byte chunk of 8 keys
+    const int hh = ch >> 3, cc = ch & 7;
+    const uint4 bv = *reinterpret_cast<const uint4 *>(brow + hh * (kBiasTileBytes / 2) +
+                                                      ((cc ^ (row & 7)) << 4));
+    const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int jj = q * 8 + e * 2;
+      const uint64_t bl = fma2(f2pack(bf16lo(bw[e]), bf16hi(bw[e])), l2e2, nm2);
+      const float2 v =
+          f2unpack(fma2(f2pack(__uint_as_float(u[jj]), __uint_as_float(u[jj + 1])), c1x2, bl));
+      t[jj] = v.x;
+      t[jj + 1] = v.y;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -119,9 +150,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl.bias_full[b], 1);
-      mbar_init(&ctl.bias_empty[b], 128);
+      mbar_init(&ctl.bias_empty[b], 256);
       mbar_init(&ctl.s_full[b], 1);
-      mbar_init(&ctl.p_full[b], 128);
+      mbar_init(&ctl.p_full[b], 128);   // buffer b belongs to warpgroup b
     }
     for (int rr = 0; rr < kRows; ++rr) mbar_init(&ctl.o_done[rr], 1);
     mbar_init(&ctl.o_final, 1);
@@ -176,7 +207,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctl.kv_full[st], 2 * kPairTileBytes);
+          mbar_arrive_expect_tx(&ctl.kv_full[st], 2 * kPairTileBytes + 16);
           uint8_t *kd = smem + kOffK + st * kPairTileBytes;
           uint8_t *vd = smem + kOffV + st * kPairTileBytes;
           if (a.x_inner) {
@@ -186,6 +217,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
             tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
           }
+          bulk_load(smem + kOffMask + st * 16,
+                    a.mask_bits + (int64_t)(r0 + rr) * a.mask_bits_stride + kb * 4, 16,
+                    &ctl.kv_full[st]);
           armed_kv[st] = it / kStages;
         }
       }
@@ -248,19 +282,28 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ------------------------------------------------ softmax and epilogue --
+    // Rows are handled in pairs: warpgroup wg owns the rows rr = 2j + wg and the
+    // S/P buffer wg (every CTA holds kRows = 8 rows, because N % 8 == 0).
+    const int wg = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;           // query within the tile = TMEM lane
     const int x = xb * kBM + row;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-    const float c1 = a.scale * kLog2e;
-    float m_r[kRows], l_r[kRows];
+    const uint32_t sbuf = tl + wg * kBN;
+    constexpr int kMine = kRows / 2;
+    const uint64_t c1x2 = f2pack(a.scale * kLog2e, a.scale * kLog2e);
+    const uint64_t l2e2 = f2pack(kLog2e, kLog2e);
+    float m_r[kMine], l_r[kMine];
 #pragma unroll
-    for (int rr = 0; rr < kRows; ++rr) {
-      m_r[rr] = -INFINITY;
-      l_r[rr] = 0.0f;
+    for (int j = 0; j < kMine; ++j) {
+      m_r[j] = -INFINITY;
+      l_r[j] = 0.0f;
     }
-    bool ok = true;
-    int it = 0;
+    bool ok = nrows == kRows;
+    if (!ok) {
+      *abort_flag = 1u;
+      report_status(a.status, kStatusBounds);
+    }
     for (int kb = 0; kb < nkb && ok; ++kb) {
       const int bb = kb & 1;
       if (!wait_bar_warp(&ctl.bias_full[bb], (kb >> 1) & 1, abort_flag, a.status)) {
@@ -268,77 +311,75 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       const uint8_t *brow = smem + kOffB + bb * kBiasTileBytes + row * 128;
+      // max of this query row's 128 bias values (shared by all rows of the CTA)
+      float bmax = -INFINITY;
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {
+        const uint4 bv = *reinterpret_cast<const uint4 *>(brow + (ch >> 3) * (kBiasTileBytes / 2) +
+                                                          (((ch & 7) ^ (row & 7)) << 4));
+        bmax = fmax3(bmax, fmax3(bf16lo(bv.x), bf16hi(bv.x), bf16lo(bv.y)),
+                     fmax3(bf16hi(bv.y), fmax3(bf16lo(bv.z), bf16hi(bv.z), bf16lo(bv.w)),
+                           bf16hi(bv.w)));
+      }
 #pragma unroll 1
-      for (int rr = 0; rr < kRows; ++rr) {
-        if (rr >= nrows) break;
-        const int sb = it & 1;
-        const int r = r0 + rr;
-        // key mask bits of this row and key tile (tail keys are zero bits)
-        const uint32_t *mb = a.mask_bits + (int64_t)r * a.mask_bits_stride + kb * 4;
-        const uint4 mw = *reinterpret_cast<const uint4 *>(mb);
-        const bool full_tile = (mw.x & mw.y & mw.z & mw.w) == 0xffffffffu;
-        if (!wait_bar_warp(&ctl.s_full[sb], (it >> 1) & 1, abort_flag, a.status)) {
+      for (int j = 0; j < kMine; ++j) {
+        const int rr = 2 * j + wg;
+        const int it = kb * kRows + rr;
+        const int st = it % kStages;
+        // key bits of this row and key tile arrive with the K/V stage
+        if (!wait_bar_warp(&ctl.kv_full[st], (it / kStages) & 1, abort_flag, a.status) ||
+            !wait_bar_warp(&ctl.s_full[wg], (it >> 1) & 1, abort_flag, a.status)) {
           ok = false;
           break;
         }
+        const uint4 mw = *reinterpret_cast<const uint4 *>(smem + kOffMask + st * 16);
+        const bool full_tile = (mw.x & mw.y & mw.z & mw.w) == 0xffffffffu;
         tc_fence_after();
-        float t[kBN];
-        {
+        // Pass 1: an upper bound of the row's logits, max(s) * c^-1/2 + max(b).
+        // Softmax is exact for any shift; a bound keeps every exponent <= 0.
+        float sm0 = -INFINITY, sm1 = -INFINITY;
+#pragma unroll 1
+        for (int c32 = 0; c32 < 4; ++c32) {
           uint32_t u[32];
+          tmem_ld32(sbuf + c32 * 32, u);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_ld32(tl + sb * kBN + j * 32, u);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) t[j * 32 + e] = __uint_as_float(u[e]);
+          for (int e = 0; e < 32; e += 4) {
+            sm0 = fmax3(sm0, __uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+            sm1 = fmax3(sm1, __uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
           }
         }
-        // logits in the log2 domain: s*c^-1/2*log2e + b*log2e, masked -> -inf
-        float mx = -INFINITY;
+        // log2-domain bound; the running max only moves when the bound grows by
+        // more than 8, so most tiles skip the rescale of O (p stays <= 2^8).
+        const float bound = (fmaxf(sm0, sm1) * a.scale + bmax) * kLog2e;
+        const float m_old = m_r[j];
+        const float m_new = bound > m_old + 8.0f ? bound : m_old;
+        const float alpha = ex2_approx(m_old - m_new);   // m_old = -inf gives 0
+        const uint64_t nm2 = f2pack(-m_new, -m_new);
+        uint64_t sum_a = 0, sum_b = 0;   // two packed running sums (bit pattern 0 = 0.0f)
+        uint32_t pk[16];
+#pragma unroll 1
+        for (int c32 = 0; c32 < 4; ++c32) {
+          float t[32];
+          logits32(sbuf, brow, row, c32, c1x2, l2e2, nm2, t);   // log2-domain exponents
+          const uint32_t mword = c32 == 0 ? mw.x : c32 == 1 ? mw.y : c32 == 2 ? mw.z : mw.w;
 #pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-          const int hh = ch >> 3, cc = ch & 7;
-          const uint4 bv = *reinterpret_cast<const uint4 *>(brow + hh * (kBiasTileBytes / 2) +
-                                                            ((cc ^ (row & 7)) << 4));
-          const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = ch * 8 + e * 2;
-            t[j] = fmaf(t[j], c1, bf16lo(bw[e]) * kLog2e);
-            t[j + 1] = fmaf(t[j + 1], c1, bf16hi(bw[e]) * kLog2e);
+          for (int e = 0; e < 32; e += 2) {
+            float p0 = ex2_approx(t[e]), p1 = ex2_approx(t[e + 1]);
+            if (!full_tile) {
+              if (!((mword >> e) & 1u)) p0 = 0.0f;
+              if (!((mword >> (e + 1)) & 1u)) p1 = 0.0f;
+            }
+            if (e & 2) sum_b = add2(sum_b, f2pack(p0, p1));
+            else sum_a = add2(sum_a, f2pack(p0, p1));
+            pk[e / 2] = pack_bf16(p0, p1);
           }
+          // P (bf16 pairs) of keys 32*c32.. goes to columns 16*c32..16*c32+15 of
+          // this S buffer, whose S values in those columns were already read.
+          tmem_st16(sbuf + c32 * 16, pk);
         }
-        if (!full_tile) {
-          const uint32_t mws[4] = {mw.x, mw.y, mw.z, mw.w};
-#pragma unroll
-          for (int j = 0; j < kBN; ++j)
-            if (!((mws[j >> 5] >> (j & 31)) & 1u)) t[j] = -INFINITY;
-        }
-#pragma unroll
-        for (int j = 0; j < kBN; ++j) mx = fmaxf(mx, t[j]);
-        const float m_new = fmaxf(m_r[rr], mx);
-        const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
-        const float alpha = ex2_approx(m_r[rr] - m_use);
-        float sum = 0.0f;
-        uint32_t pk[kBN / 2];
-#pragma unroll
-        for (int j = 0; j < kBN; j += 2) {
-          const float p0 = ex2_approx(t[j] - m_use);
-          const float p1 = ex2_approx(t[j + 1] - m_use);
-          sum += p0 + p1;
-          pk[j / 2] = pack_bf16(p0, p1);
-        }
-        l_r[rr] = l_r[rr] * alpha + sum;
-        m_r[rr] = m_new;
-        {
-          uint32_t w0[32], w1[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            w0[e] = pk[e];
-            w1[e] = pk[32 + e];
-          }
-          tmem_st32(tl + sb * kBN, w0);
-          tmem_st32(tl + sb * kBN + 32, w1);
-        }
+        const float2 sa = f2unpack(add2(sum_a, sum_b));
+        l_r[j] = l_r[j] * alpha + (sa.x + sa.y);
+        m_r[j] = m_new;
         if (kb > 0) {
           // rescale the running output once the previous PV of this row is done
           if (!wait_bar_warp(&ctl.o_done[rr], (kb - 1) & 1, abort_flag, a.status)) {
@@ -357,15 +398,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&ctl.p_full[sb]);
-        ++it;
+        mbar_arrive(&ctl.p_full[wg]);
       }
       if (ok) mbar_arrive(&ctl.bias_empty[bb]);
     }
     // epilogue: out = sigmoid(g) * O / l (bf16), lse = ln(sum exp s)
     if (ok) ok = wait_bar_warp(&ctl.o_final, 0, abort_flag, a.status);
     if (ok) tc_fence_after();
-    for (int rr = 0; rr < nrows; ++rr) {
+#pragma unroll 1
+    for (int j = 0; j < kMine; ++j) {
+      const int rr = 2 * j + wg;
+      if (rr >= nrows) break;
       const int r = r0 + rr;
       uint32_t o[32];
       if (ok) tmem_ld32(tl + 2 * kBN + rr * kC, o);
@@ -375,7 +418,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *lse_p = __int_as_float(0x7fc00000);  // NaN marks a tile the kernel gave up on
         continue;
       }
-      const float l = l_r[rr];
+      const float l = l_r[j];
       const float inv = l > 0.0f ? rcp_approx(l) : 0.0f;
       const int64_t off = (int64_t)r * a.sR + (int64_t)x * a.sX + (int64_t)h * kC;
       const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + off);
@@ -395,7 +438,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         op[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       }
-      *lse_p = l > 0.0f ? (m_r[rr] + lg2_approx(l)) * kLn2 : -INFINITY;
+      *lse_p = l > 0.0f ? (m_r[j] + lg2_approx(l)) * kLn2 : -INFINITY;
     }
   }
 

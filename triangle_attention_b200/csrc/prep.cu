@@ -21,8 +21,12 @@ int blocks_for(int64_t n, int threads) {
 // One word = 32 keys of one attention row; bit j set when key 32*w + j exists
 // and takes part. Also resets the call's status word.
 __global__ void mask_bits_kernel(Frame f, uint32_t *__restrict__ bits, int64_t rows,
-                                 int64_t words_per_row, int32_t *status) {
+                                 int64_t words_per_row, int32_t *status,
+                                 int32_t *__restrict__ zero, int64_t nzero) {
   if (blockIdx.x == 0 && threadIdx.x == 0 && status) *status = kStatusOk;
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < nzero;
+       w += (int64_t)gridDim.x * blockDim.x)
+    zero[w] = 0;
   const int64_t total = rows * words_per_row;
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
        w += (int64_t)gridDim.x * blockDim.x) {
@@ -103,12 +107,66 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
   }
 }
 
+// One thread per 8 channels of one output element of one of the three tensors:
+// the nb tile partials are summed in tile order in fp32, scaled, rounded once.
+__global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ pq,
+                                           const __nv_bfloat16 *__restrict__ pk,
+                                           const __nv_bfloat16 *__restrict__ pv, int nb,
+                                           float scale, __nv_bfloat16 *__restrict__ dq,
+                                           __nv_bfloat16 *__restrict__ dk,
+                                           __nv_bfloat16 *__restrict__ dv) {
+  const int64_t pair = (int64_t)f.N * f.N * f.H * 32;
+  const int64_t per = pair / 8;                 // 16-byte groups per tensor
+  for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < 3 * per;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int which = (int)(w / per);
+    const int64_t gidx = w - which * per;
+    const __nv_bfloat16 *src = which == 0 ? pq : which == 1 ? pk : pv;
+    const float sc = which == 2 ? 1.0f : scale;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    for (int t = 0; t < nb; ++t) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(src + t * pair) + gidx);
+      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += bf16lo(vw[e]);
+        acc[2 * e + 1] += bf16hi(vw[e]);
+      }
+    }
+    // compact index (r, x, h, c8) -> storage position through the frame
+    const int64_t cidx = gidx * 8;
+    const int h = (int)((cidx / 32) % f.H);
+    const int64_t x = (cidx / (32 * f.H)) % f.N;
+    const int64_t r = cidx / (32 * (int64_t)f.H * f.N);
+    const int c0 = (int)(cidx % 32);
+    __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + r * f.sR + x * f.sX +
+                         (int64_t)h * 32 + c0;
+    *reinterpret_cast<uint4 *>(dst) =
+        make_uint4(pack_bf16(acc[0] * sc, acc[1] * sc), pack_bf16(acc[2] * sc, acc[3] * sc),
+                   pack_bf16(acc[4] * sc, acc[5] * sc), pack_bf16(acc[6] * sc, acc[7] * sc));
+  }
+}
+
 }  // namespace
 
+cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part_q,
+                                       const __nv_bfloat16 *part_k, const __nv_bfloat16 *part_v,
+                                       int nb, float scale, __nv_bfloat16 *dq, __nv_bfloat16 *dk,
+                                       __nv_bfloat16 *dv, cudaStream_t stream) {
+  const int64_t work = 3 * ((int64_t)f.N * f.N * f.H * 32 / 8);
+  if (work == 0) return cudaSuccess;
+  partial_reduce_bf16_kernel<<<blocks_for(work, 256), 256, 0, stream>>>(f, part_q, part_k, part_v,
+                                                                         nb, scale, dq, dk, dv);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mask_bits(const Frame &f, uint32_t *bits, int64_t rows, int64_t words_per_row,
-                             int32_t *status, cudaStream_t stream) {
-  mask_bits_kernel<<<blocks_for(rows * words_per_row, 256), 256, 0, stream>>>(
-      f, bits, rows, words_per_row, status);
+                             int32_t *status, int32_t *zero, int64_t nzero, cudaStream_t stream) {
+  const int64_t work = rows * words_per_row > nzero ? rows * words_per_row : nzero;
+  mask_bits_kernel<<<blocks_for(work, 256), 256, 0, stream>>>(f, bits, rows, words_per_row,
+                                                              status, zero, nzero);
   return cudaGetLastError();
 }
 
