@@ -137,8 +137,8 @@ __device__ __forceinline__ void dsoftmax_chunk(const uint32_t (&s)[NC], const ui
     const float2 dbv = f2unpack(add2(f2pack(__uint_as_float(db[e]), __uint_as_float(db[e + 1])), d2));
     db[e] = __float_as_uint(dbv.x);
     db[e + 1] = __float_as_uint(dbv.y);
-    pw[e / 2] = pack_bf16(p0, p1);
-    dw[e / 2] = pack_bf16(dsv.x, dsv.y);
+    pw[e / 2] = pack_bf16_int(p0, p1);
+    dw[e / 2] = pack_bf16_int(dsv.x, dsv.y);
   }
 }
 
@@ -362,9 +362,7 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // 16 keys: kbase + 16*ch .. +15, i.e. 16-byte chunks 2*ch and 2*ch+1 of the half tile
         const uint32_t col = kbase + ch * 16;
         uint32_t s[16], dp[16], db[16], pw[8], dw[8], bw[8];
-        tmem_ld16(tl + kColS + col, s);
-        tmem_ld16(tl + kColDP + col, dp);
-        tmem_ld16(tl + kColDB + col, db);
+        tmem_ld16x3(tl + kColS + col, tl + kColDP + col, tl + kColDB + col, s, dp, db);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const uint4 bv =

@@ -97,13 +97,12 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
-// Exponents (s*c^-1/2 + b)*log2e - m of 32 keys of this thread's query row:
-// S columns 32*c32.. from tensor memory, bias from the 128-byte-swizzled tile.
-__device__ __forceinline__ void logits32(uint32_t sbuf, const uint8_t *brow, int row, int c32,
-                                         uint64_t c1x2, uint64_t l2e2, uint64_t nm2,
-                                         float (&t)[32]) {
-  uint32_t u[32];
-  tmem_ld32(sbuf + c32 * 32, u);
+// Exponents (s*c^-1/2 + b)*log2e - m of 32 keys (raw S bits in u, keys
+// 32*c32.. of the tile) of this thread's query row, in place; bias from the
+// 128-byte-swizzled tile in shared memory.
+__device__ __forceinline__ void exponents32(uint32_t (&u)[32], const uint8_t *brow, int row,
+                                            int c32, uint64_t c1x2, uint64_t l2e2,
+                                            uint64_t nm2) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int ch = c32 * 4 + q;              // 16-byte chunk of 8 keys
@@ -117,9 +116,26 @@ __device__ __forceinline__ void logits32(uint32_t sbuf, const uint8_t *brow, int
       const uint64_t bl = fma2(f2pack(bf16lo(bw[e]), bf16hi(bw[e])), l2e2, nm2);
       const float2 v =
           f2unpack(fma2(f2pack(__uint_as_float(u[jj]), __uint_as_float(u[jj + 1])), c1x2, bl));
-      t[jj] = v.x;
-      t[jj + 1] = v.y;
+      u[jj] = __float_as_uint(v.x);
+      u[jj + 1] = __float_as_uint(v.y);
     }
+  }
+}
+
+// Probabilities of 32 keys from their exponents: bf16 pairs into pk, running
+// sums into sa/sb; masked keys (zero bits of mword) give 0 when !full.
+__device__ __forceinline__ void probs32(const uint32_t (&u)[32], uint32_t mword, bool full,
+                                        uint64_t &sa, uint64_t &sb, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float p0 = ex2_approx(__uint_as_float(u[e])), p1 = ex2_approx(__uint_as_float(u[e + 1]));
+    if (!full) {
+      if (!((mword >> e) & 1u)) p0 = 0.0f;
+      if (!((mword >> (e + 1)) & 1u)) p1 = 0.0f;
+    }
+    if (e & 2) sb = add2(sb, f2pack(p0, p1));
+    else sa = add2(sa, f2pack(p0, p1));
+    pk[e / 2] = pack_bf16_int(p0, p1);
   }
 }
 
@@ -339,13 +355,13 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Softmax is exact for any shift; a bound keeps every exponent <= 0.
         float sm0 = -INFINITY, sm1 = -INFINITY;
 #pragma unroll 1
-        for (int c32 = 0; c32 < 4; ++c32) {
-          uint32_t u[32];
-          tmem_ld32(sbuf + c32 * 32, u);
+        for (int c64 = 0; c64 < 2; ++c64) {
+          uint32_t u[32], w[32];
+          tmem_ld32x2(sbuf + c64 * 64, sbuf + c64 * 64 + 32, u, w);
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
+          for (int e = 0; e < 32; e += 2) {
             sm0 = fmax3(sm0, __uint_as_float(u[e]), __uint_as_float(u[e + 1]));
-            sm1 = fmax3(sm1, __uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
+            sm1 = fmax3(sm1, __uint_as_float(w[e]), __uint_as_float(w[e + 1]));
           }
         }
         // log2-domain bound; the running max only moves when the bound grows by
@@ -358,24 +374,18 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         uint64_t sum_a = 0, sum_b = 0;   // two packed running sums (bit pattern 0 = 0.0f)
         uint32_t pk[16];
 #pragma unroll 1
-        for (int c32 = 0; c32 < 4; ++c32) {
-          float t[32];
-          logits32(sbuf, brow, row, c32, c1x2, l2e2, nm2, t);   // log2-domain exponents
-          const uint32_t mword = c32 == 0 ? mw.x : c32 == 1 ? mw.y : c32 == 2 ? mw.z : mw.w;
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float p0 = ex2_approx(t[e]), p1 = ex2_approx(t[e + 1]);
-            if (!full_tile) {
-              if (!((mword >> e) & 1u)) p0 = 0.0f;
-              if (!((mword >> (e + 1)) & 1u)) p1 = 0.0f;
-            }
-            if (e & 2) sum_b = add2(sum_b, f2pack(p0, p1));
-            else sum_a = add2(sum_a, f2pack(p0, p1));
-            pk[e / 2] = pack_bf16(p0, p1);
-          }
-          // P (bf16 pairs) of keys 32*c32.. goes to columns 16*c32..16*c32+15 of
-          // this S buffer, whose S values in those columns were already read.
-          tmem_st16(sbuf + c32 * 16, pk);
+        for (int c64 = 0; c64 < 2; ++c64) {
+          uint32_t u[32], w[32];
+          tmem_ld32x2(sbuf + c64 * 64, sbuf + c64 * 64 + 32, u, w);
+          const uint32_t mu = c64 == 0 ? mw.x : mw.z, mv = c64 == 0 ? mw.y : mw.w;
+          // P (bf16 pairs) of keys 64*c64.. goes to columns 32*c64..32*c64+31 of
+          // this S buffer, whose S values were already read into registers.
+          exponents32(u, brow, row, 2 * c64, c1x2, l2e2, nm2);
+          probs32(u, mu, full_tile, sum_a, sum_b, pk);
+          tmem_st16(sbuf + c64 * 32, pk);
+          exponents32(w, brow, row, 2 * c64 + 1, c1x2, l2e2, nm2);
+          probs32(w, mv, full_tile, sum_a, sum_b, pk);
+          tmem_st16(sbuf + c64 * 32 + 16, pk);
         }
         const float2 sa = f2unpack(add2(sum_a, sum_b));
         l_r[j] = l_r[j] * alpha + (sa.x + sa.y);

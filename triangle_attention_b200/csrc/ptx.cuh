@@ -226,6 +226,50 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "memory");
 }
 
+#define TRI_RA8(b) "=r"(a[b + 0]), "=r"(a[b + 1]), "=r"(a[b + 2]), "=r"(a[b + 3]), \
+    "=r"(a[b + 4]), "=r"(a[b + 5]), "=r"(a[b + 6]), "=r"(a[b + 7])
+#define TRI_RB8(b) "=r"(b_[b + 0]), "=r"(b_[b + 1]), "=r"(b_[b + 2]), "=r"(b_[b + 3]), \
+    "=r"(b_[b + 4]), "=r"(b_[b + 5]), "=r"(b_[b + 6]), "=r"(b_[b + 7])
+#define TRI_RC8(b) "=r"(c_[b + 0]), "=r"(c_[b + 1]), "=r"(c_[b + 2]), "=r"(c_[b + 3]), \
+    "=r"(c_[b + 4]), "=r"(c_[b + 5]), "=r"(c_[b + 6]), "=r"(c_[b + 7])
+
+// Three 16-column loads (e.g. S, dP and an accumulator of the same rows) with
+// a single wait, so their latencies overlap.
+__device__ __forceinline__ void tmem_ld16x3(uint32_t ta, uint32_t tb, uint32_t tc,
+                                            uint32_t (&a)[16], uint32_t (&b_)[16],
+                                            uint32_t (&c_)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%48];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,"
+      "%28,%29,%30,%31}, [%49];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,"
+      "%44,%45,%46,%47}, [%50];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : TRI_RA8(0), TRI_RA8(8), TRI_RB8(0), TRI_RB8(8), TRI_RC8(0), TRI_RC8(8)
+      : "r"(ta), "r"(tb), "r"(tc)
+      : "memory");
+}
+
+// Two 32-column loads with a single wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (&a)[32],
+                                            uint32_t (&b_)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,"
+      "%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : TRI_RA8(0), TRI_RA8(8), TRI_RA8(16), TRI_RA8(24), TRI_RB8(0), TRI_RB8(8), TRI_RB8(16),
+        TRI_RB8(24)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+#undef TRI_RA8
+#undef TRI_RB8
+#undef TRI_RC8
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
@@ -350,6 +394,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Two floats to bf16x2 on the integer pipes (low half = lo): round to nearest
+// with ties away from zero (add half an ulp of bf16 to the bit pattern, keep
+// the high halves). Differs from cvt.rn only on exact ties; infinities stay
+// infinite and finite values above the bf16 range round to infinity.
+__device__ __forceinline__ uint32_t pack_bf16_int(float lo, float hi) {
+  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
