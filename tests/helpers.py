@@ -63,10 +63,14 @@ def assert_close(name, got, ref, rel, max_abs=None):
     return err
 
 
-def compare_rows(res, ref_fwd, ref_bwd, rows, variant, dtype):
-    """Compare the CUDA results on the listed attention rows (variant frame)."""
+def compare_rows(res, ref_fwd, ref_bwd, rows, variant, dtype, out_abs_scale=None):
+    """Compare the CUDA results on the listed attention rows (variant frame).
+    out_abs_scale replaces the absolute max-error bound on out (2e-2, set for
+    N(0,1) inputs) by out_abs_scale * max|out_ref| for scaled-up inputs."""
     rel = F32_REL if dtype == "f32" else BF16_REL
     out_abs = None if dtype == "f32" else BF16_OUT_ABS
+    if out_abs is not None and out_abs_scale is not None:
+        out_abs = out_abs_scale * float(np.max(np.abs(ref_fwd[0])))
     errs = {}
     o_ref, l_ref = ref_fwd
     out = np64(variant_frame(res["out"], variant))[rows]

@@ -49,6 +49,8 @@ constexpr uint32_t kPairTileBytes = kBM * kC * 2;   // 8 KB
 constexpr uint32_t kBiasTileBytes = kBM * kBN * 2;  // 32 KB (two 16 KB halves)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// bf16 rounding of P: on the integer pipes (true) or with cvt.rn (false)
+constexpr bool kPackOnIntegerPipes = false;
 
 struct __align__(8) FwdSmem {
   uint64_t q_full;
@@ -123,19 +125,20 @@ __device__ __forceinline__ void exponents32(uint32_t (&u)[32], const uint8_t *br
 }
 
 // Probabilities of 32 keys from their exponents: bf16 pairs into pk, running
-// sums into sa/sb; masked keys (zero bits of mword) give 0 when !full.
-__device__ __forceinline__ void probs32(const uint32_t (&u)[32], uint32_t mword, bool full,
-                                        uint64_t &sa, uint64_t &sb, uint32_t (&pk)[16]) {
+// sums into sa/sb. MASKED: keys whose bit in mword is clear give 0.
+template <bool MASKED>
+__device__ __forceinline__ void probs32(const uint32_t (&u)[32], uint32_t mword, uint64_t &sa,
+                                        uint64_t &sb, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     float p0 = ex2_approx(__uint_as_float(u[e])), p1 = ex2_approx(__uint_as_float(u[e + 1]));
-    if (!full) {
+    if (MASKED) {
       if (!((mword >> e) & 1u)) p0 = 0.0f;
       if (!((mword >> (e + 1)) & 1u)) p1 = 0.0f;
     }
     if (e & 2) sb = add2(sb, f2pack(p0, p1));
     else sa = add2(sa, f2pack(p0, p1));
-    pk[e / 2] = pack_bf16_int(p0, p1);
+    pk[e / 2] = kPackOnIntegerPipes ? pack_bf16_int(p0, p1) : pack_bf16(p0, p1);
   }
 }
 
@@ -381,10 +384,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // P (bf16 pairs) of keys 64*c64.. goes to columns 32*c64..32*c64+31 of
           // this S buffer, whose S values were already read into registers.
           exponents32(u, brow, row, 2 * c64, c1x2, l2e2, nm2);
-          probs32(u, mu, full_tile, sum_a, sum_b, pk);
+          if (full_tile) probs32<false>(u, mu, sum_a, sum_b, pk);
+          else probs32<true>(u, mu, sum_a, sum_b, pk);
           tmem_st16(sbuf + c64 * 32, pk);
           exponents32(w, brow, row, 2 * c64 + 1, c1x2, l2e2, nm2);
-          probs32(w, mv, full_tile, sum_a, sum_b, pk);
+          if (full_tile) probs32<false>(w, mv, sum_a, sum_b, pk);
+          else probs32<true>(w, mv, sum_a, sum_b, pk);
           tmem_st16(sbuf + c64 * 32 + 16, pk);
         }
         const float2 sa = f2unpack(add2(sum_a, sum_b));

@@ -266,6 +266,18 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (
       : "memory");
 }
 
+// Two 8-column loads with a single wait.
+__device__ __forceinline__ void tmem_ld8x2(uint32_t ta, uint32_t tb, uint32_t (&a)[8],
+                                           uint32_t (&b_)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : TRI_RA8(0), TRI_RB8(0)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
 #undef TRI_RA8
 #undef TRI_RB8
 #undef TRI_RC8
