@@ -37,6 +37,7 @@
 // +128..255; after the row's gradient MMAs, dQ at +0, dK at +32, dV at +64.
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 
 #include "bf16.cuh"
@@ -50,7 +51,7 @@ constexpr int kBM = 128;
 constexpr int kBN = 128;
 constexpr int kC = 32;
 constexpr int kStages = 2;
-constexpr int kEltGroups = 2;                            // elementwise warpgroups
+constexpr int kEltGroups = 4;                            // elementwise warpgroups
 constexpr int kKeys = 128 / kEltGroups;                  // keys of the block per group
 constexpr int kThreads = 64 + kEltGroups * 128;
 constexpr int kEltThreads = kEltGroups * 128;
@@ -380,6 +381,10 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
     for (int e = 0; e < kKeys / 2; ++e) dbias2[e] = 0ull;
     const uint8_t *brow = smem + kOffBias + half * (kSqTileBytes / 2) + row * 128;
+    // 16-byte chunk chunk0 + ch of the swizzled row is at (cswz ^ ch) (chunk0 is a
+    // multiple of kKeys / 8, so adding ch never carries into its bits)
+    const uint32_t cswz = (uint32_t)(chunk0 ^ (row & 7));
+    static_assert((kKeys / 8 & (kKeys / 8 - 1)) == 0, "key groups must be powers of two");
 
     // Move the gradient partials of row t out of TMEM buffer t & 1 to the
     // per-tile partial tensors, in six 16-column pieces (dQ 0/16, dK 0/16,
@@ -420,14 +425,21 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint8_t *in = smem + kOffRow + st * kRowBytes;
       const float L = x < N ? reinterpret_cast<const float *>(in + kStLse)[row] : -INFINITY;
       const float Dx = x < N ? reinterpret_cast<const float *>(in + kStD)[row] : 0.0f;
-      // key bits of this warpgroup's keys (kKeys / 32 words from word kbase / 32)
+      // key bits of this warpgroup's keys: kKeys / 32 words from word kbase / 32
       const uint4 mw4 = *reinterpret_cast<const uint4 *>(in + kStMask);
-      const uint32_t mwords[4] = {mw4.x, mw4.y, mw4.z, mw4.w};
+      uint32_t kw[kKeys / 32];
       uint32_t mall = 0xffffffffu;
 #pragma unroll
-      for (int w = 0; w < kKeys / 32; ++w) mall &= mwords[(kbase / 32 + w) & 3];
+      for (int w = 0; w < kKeys / 32; ++w) {
+        const int i = (int)(kbase / 32) + w;
+        kw[w] = i == 0 ? mw4.x : i == 1 ? mw4.y : i == 2 ? mw4.z : mw4.w;
+        mall &= kw[w];
+      }
       const bool live = L > -INFINITY;
-      const bool full = live && mall == 0xffffffffu;
+      // The unmasked form runs only when every lane of the warp may take it: the
+      // per-row body holds warp-collective tensor-memory loads and waits, so the
+      // choice must be warp-uniform (lanes past N in a ragged tile are not live).
+      const bool full = __all_sync(0xffffffffu, live && mall == 0xffffffffu);
       const float lL = live ? L * kLog2e : 0.0f;
       const uint64_t nlx2 = f2pack(-lL, -lL);
       const uint64_t ndx2 = f2pack(-Dx, -Dx);
@@ -441,32 +453,36 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       uint8_t *dstile = ptile + kSqTileBytes;
       const uint32_t sb = tl + b * kBufCols + kColS + kbase;
       const uint32_t db = tl + b * kBufCols + kColDP + kbase;
+      // One row's kKeys keys, 8 at a time; the S/dP loads of the next 8 are in
+      // flight while these are processed. The masked form is chosen per row.
+      auto row_keys = [&](auto masked_tag) -> bool {
+        constexpr bool kMasked = decltype(masked_tag)::value;
+        uint32_t sv[2][8], dpv[2][8];
+        tmem_ld8x2_issue(sb, db, sv[0], dpv[0]);
+        tmem_wait_ld8x2(sv[0], dpv[0]);
 #pragma unroll
-      for (int ch = 0; ch < kKeys / 8; ++ch) {
-        if (ch == kKeys / 16 && it >= 1) {
-          // half-way through this row the previous row's gradients are done
-          if (!drain(it - 1)) {
-            ok = false;
-            break;
+        for (int ch = 0; ch < kKeys / 8; ++ch) {
+          const int cur = ch & 1, nxt = cur ^ 1;
+          if (ch == kKeys / 16 && it >= 1) {
+            // half-way through this row the previous row's gradients are done
+            if (!drain(it - 1)) return false;
           }
+          if (ch + 1 < kKeys / 8)
+            tmem_ld8x2_issue(sb + (ch + 1) * 8, db + (ch + 1) * 8, sv[nxt], dpv[nxt]);
+          const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((cswz ^ ch) << 4));
+          const uint32_t bias[4] = {bv.x, bv.y, bv.z, bv.w};
+          uint32_t mbits = 0u;
+          if (kMasked) mbits = live ? (kw[(8 * ch) / 32] >> ((8 * ch) % 32)) : 0u;
+          uint32_t pw[4], dw[4];
+          dsoftmax8<kMasked>(sv[cur], dpv[cur], bias, dbias2 + ch * 4, mbits, c1x2, l2e2, nlx2,
+                             ndx2, pw, dw);
+          st_tile_chunk(ptile, row, half, chunk0 + ch, pw[0], pw[1], pw[2], pw[3]);
+          st_tile_chunk(dstile, row, half, chunk0 + ch, dw[0], dw[1], dw[2], dw[3]);
+          if (ch + 1 < kKeys / 8) tmem_wait_ld8x2(sv[nxt], dpv[nxt]);
         }
-        uint32_t sv[8], dpv[8];
-        tmem_ld8x2(sb + ch * 8, db + ch * 8, sv, dpv);
-        const uint4 bv =
-            *reinterpret_cast<const uint4 *>(brow + (((chunk0 + ch) ^ (row & 7)) << 4));
-        const uint32_t bias[4] = {bv.x, bv.y, bv.z, bv.w};
-        uint32_t pw[4], dw[4];
-        if (full) {
-          dsoftmax8<false>(sv, dpv, bias, dbias2 + ch * 4, 0u, c1x2, l2e2, nlx2, ndx2, pw, dw);
-        } else {
-          // word (kbase + 8ch) / 32 of the row's key bits, shifted to this chunk
-          const uint32_t word = mwords[((kbase + 8 * ch) / 32) & 3];
-          const uint32_t mbits = live ? (word >> ((8 * ch + kbase) % 32)) : 0u;
-          dsoftmax8<true>(sv, dpv, bias, dbias2 + ch * 4, mbits, c1x2, l2e2, nlx2, ndx2, pw, dw);
-        }
-        st_tile_chunk(ptile, row, half, chunk0 + ch, pw[0], pw[1], pw[2], pw[3]);
-        st_tile_chunk(dstile, row, half, chunk0 + ch, dw[0], dw[1], dw[2], dw[3]);
-      }
+        return true;
+      };
+      ok = full ? row_keys(std::false_type{}) : row_keys(std::true_type{});
       if (!ok) break;
       tc_fence_before();
       fence_proxy_async_smem();

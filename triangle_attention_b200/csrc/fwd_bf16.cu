@@ -312,12 +312,25 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr int kMine = kRows / 2;
     const uint64_t c1x2 = f2pack(a.scale * kLog2e, a.scale * kLog2e);
     const uint64_t l2e2 = f2pack(kLog2e, kLog2e);
+    // running max and sum of this warpgroup's kMine rows; the loop over rows is
+    // not unrolled, so the registers rotate (row j's pair is always m_r[0],
+    // l_r[0]) instead of being indexed, which would put them in local memory
     float m_r[kMine], l_r[kMine];
 #pragma unroll
     for (int j = 0; j < kMine; ++j) {
       m_r[j] = -INFINITY;
       l_r[j] = 0.0f;
     }
+    auto rotate_rows = [&]() {
+      const float m0 = m_r[0], l0 = l_r[0];
+#pragma unroll
+      for (int j = 0; j + 1 < kMine; ++j) {
+        m_r[j] = m_r[j + 1];
+        l_r[j] = l_r[j + 1];
+      }
+      m_r[kMine - 1] = m0;
+      l_r[kMine - 1] = l0;
+    };
     bool ok = nrows == kRows;
     if (!ok) {
       *abort_flag = 1u;
@@ -370,7 +383,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // log2-domain bound; the running max only moves when the bound grows by
         // more than 8, so most tiles skip the rescale of O (p stays <= 2^8).
         const float bound = (fmaxf(sm0, sm1) * a.scale + bmax) * kLog2e;
-        const float m_old = m_r[j];
+        const float m_old = m_r[0];
         const float m_new = bound > m_old + 8.0f ? bound : m_old;
         const float alpha = ex2_approx(m_old - m_new);   // m_old = -inf gives 0
         const uint64_t nm2 = f2pack(-m_new, -m_new);
@@ -393,8 +406,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tmem_st16(sbuf + c64 * 32 + 16, pk);
         }
         const float2 sa = f2unpack(add2(sum_a, sum_b));
-        l_r[j] = l_r[j] * alpha + (sa.x + sa.y);
-        m_r[j] = m_new;
+        l_r[0] = l_r[0] * alpha + (sa.x + sa.y);
+        m_r[0] = m_new;
         if (kb > 0) {
           // rescale the running output once the previous PV of this row is done
           if (!wait_bar_warp(&ctl.o_done[rr], (kb - 1) & 1, abort_flag, a.status)) {
@@ -414,6 +427,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&ctl.p_full[wg]);
+        rotate_rows();
       }
       if (ok) mbar_arrive(&ctl.bias_empty[bb]);
     }
@@ -421,7 +435,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok) ok = wait_bar_warp(&ctl.o_final, 0, abort_flag, a.status);
     if (ok) tc_fence_after();
 #pragma unroll 1
-    for (int j = 0; j < kMine; ++j) {
+    for (int j = 0; j < kMine; ++j, rotate_rows()) {
       const int rr = 2 * j + wg;
       if (rr >= nrows) break;
       const int r = r0 + rr;
@@ -433,7 +447,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         *lse_p = __int_as_float(0x7fc00000);  // NaN marks a tile the kernel gave up on
         continue;
       }
-      const float l = l_r[j];
+      const float l = l_r[0];
       const float inv = l > 0.0f ? rcp_approx(l) : 0.0f;
       const int64_t off = (int64_t)r * a.sR + (int64_t)x * a.sX + (int64_t)h * kC;
       const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + off);
@@ -453,7 +467,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         op[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       }
-      *lse_p = l > 0.0f ? (m_r[j] + lg2_approx(l)) * kLn2 : -INFINITY;
+      *lse_p = l > 0.0f ? (m_r[0] + lg2_approx(l)) * kLn2 : -INFINITY;
     }
   }
 

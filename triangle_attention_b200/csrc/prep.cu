@@ -61,49 +61,51 @@ __device__ __forceinline__ float sigmoid_fast(float g) {
   return rcp_approx(1.0f + ex2_approx(-g * 1.4426950408889634f));
 }
 
-// One thread per (storage row a, storage column b, head h): 32 channels.
+// One thread per 8 channels (16 bytes) of one (storage row a, storage column b,
+// head h), so a warp reads 512 contiguous bytes of each tensor per load; the
+// four threads of one (a, b, h) sum their parts of D with two shuffles.
 __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ gate,
                                     const __nv_bfloat16 *__restrict__ out,
                                     const __nv_bfloat16 *__restrict__ dout,
                                     __nv_bfloat16 *__restrict__ du, float *__restrict__ D,
                                     __nv_bfloat16 *__restrict__ dgate, int ending) {
-  const int64_t total = (int64_t)f.N * f.N * f.H;
+  const int64_t total = (int64_t)f.N * f.N * f.H * 4;
+  const unsigned group = 0xfu << (threadIdx.x & 28);   // the 4 lanes of one (a, b, h)
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
        w += (int64_t)gridDim.x * blockDim.x) {
-    const int h = (int)(w % f.H);
-    const int64_t b = (w / f.H) % f.N;
-    const int64_t aa = w / ((int64_t)f.H * f.N);
+    const int q = (int)(w & 3);                                // channels 8q .. 8q+7
+    const int64_t e = w >> 2;                                  // (a, b, h)
+    const int h = (int)(e % f.H);
+    const int64_t b = (e / f.H) % f.N;
+    const int64_t aa = e / ((int64_t)f.H * f.N);
     const int64_t r = ending ? b : aa;
     const int64_t x = ending ? aa : b;
-    const int64_t so = w * 32;                                 // storage offset
-    const int64_t co = (((r * f.N + x) * f.H) + h) * 32;      // compact variant frame
-    const uint4 *gp = reinterpret_cast<const uint4 *>(gate + so);
-    const uint4 *op = reinterpret_cast<const uint4 *>(out + so);
-    const uint4 *dp = reinterpret_cast<const uint4 *>(dout + so);
-    uint4 *up = reinterpret_cast<uint4 *>(du + co);
-    uint4 *gq = reinterpret_cast<uint4 *>(dgate + so);
+    const int64_t so = w * 8;                                  // storage offset
+    const int64_t co = (((r * f.N + x) * f.H) + h) * 32 + q * 8;   // compact variant frame
+    const uint4 g4 = *reinterpret_cast<const uint4 *>(gate + so);
+    const uint4 o4 = *reinterpret_cast<const uint4 *>(out + so);
+    const uint4 d4 = *reinterpret_cast<const uint4 *>(dout + so);
+    const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
+    const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+    uint32_t uw[4], rw[4];
     float d = 0.0f;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const uint4 g4 = gp[v], o4 = op[v], d4 = dp[v];
-      const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
-      const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
-      const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
-      uint32_t uw[4], rw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float s0 = sigmoid_fast(bf16lo(gw[e])), s1 = sigmoid_fast(bf16hi(gw[e]));
-        const float d0 = bf16lo(dw[e]), d1 = bf16hi(dw[e]);
-        const float o0 = bf16lo(ow[e]), o1 = bf16hi(ow[e]);
-        d = fmaf(d0, o0, d);
-        d = fmaf(d1, o1, d);
-        uw[e] = pack_bf16(d0 * s0, d1 * s1);
-        rw[e] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
-      }
-      up[v] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
-      gq[v] = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+    for (int k = 0; k < 4; ++k) {
+      const float s0 = sigmoid_fast(bf16lo(gw[k])), s1 = sigmoid_fast(bf16hi(gw[k]));
+      const float d0 = bf16lo(dw[k]), d1 = bf16hi(dw[k]);
+      const float o0 = bf16lo(ow[k]), o1 = bf16hi(ow[k]);
+      d = fmaf(d0, o0, d);
+      d = fmaf(d1, o1, d);
+      uw[k] = pack_bf16(d0 * s0, d1 * s1);
+      rw[k] = pack_bf16(d0 * o0 * (1.0f - s0), d1 * o1 * (1.0f - s1));
     }
-    D[(r * f.H + h) * f.N + x] = d;
+    *reinterpret_cast<uint4 *>(du + co) = make_uint4(uw[0], uw[1], uw[2], uw[3]);
+    *reinterpret_cast<uint4 *>(dgate + so) = make_uint4(rw[0], rw[1], rw[2], rw[3]);
+    // fixed combination order: (q0 + q1) + (q2 + q3)
+    d += __shfl_xor_sync(group, d, 1);
+    d += __shfl_xor_sync(group, d, 2);
+    if (q == 0) D[(r * f.H + h) * f.N + x] = d;
   }
 }
 
@@ -126,13 +128,22 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-    for (int t = 0; t < nb; ++t) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(src + t * pair) + gidx);
-      const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+    // kBatch partials in flight per thread, then added in tile order
+    constexpr int kBatch = 8;
+    for (int t0 = 0; t0 < nb; t0 += kBatch) {
+      uint4 v[kBatch];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[2 * e] += bf16lo(vw[e]);
-        acc[2 * e + 1] += bf16hi(vw[e]);
+      for (int u = 0; u < kBatch; ++u)
+        if (t0 + u < nb) v[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (t0 + u) * pair) + gidx);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (t0 + u >= nb) break;
+        const uint32_t vw[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += bf16lo(vw[e]);
+          acc[2 * e + 1] += bf16hi(vw[e]);
+        }
       }
     }
     // compact index (r, x, h, c8) -> storage position through the frame
@@ -182,7 +193,7 @@ cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
                                 const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
                                 cudaStream_t stream) {
-  const int64_t total = (int64_t)f.N * f.N * f.H;
+  const int64_t total = (int64_t)f.N * f.N * f.H * 4;
   if (total == 0) return cudaSuccess;
   const int ending = f.variant == 1 ? 1 : 0;
   bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, dout, du, D,

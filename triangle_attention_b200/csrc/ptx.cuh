@@ -278,6 +278,31 @@ __device__ __forceinline__ void tmem_ld8x2(uint32_t ta, uint32_t tb, uint32_t (&
       : "memory");
 }
 
+// Two 8-column loads left in flight: the registers must not be read before
+// tmem_wait_ld8x2 on the same arrays, which ties them to the wait.
+__device__ __forceinline__ void tmem_ld8x2_issue(uint32_t ta, uint32_t tb, uint32_t (&a)[8],
+                                                 uint32_t (&b_)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%16];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%17];\n"
+      : TRI_RA8(0), TRI_RB8(0)
+      : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+#define TRI_UA8(b) "+r"(a[b + 0]), "+r"(a[b + 1]), "+r"(a[b + 2]), "+r"(a[b + 3]), \
+    "+r"(a[b + 4]), "+r"(a[b + 5]), "+r"(a[b + 6]), "+r"(a[b + 7])
+#define TRI_UB8(b) "+r"(b_[b + 0]), "+r"(b_[b + 1]), "+r"(b_[b + 2]), "+r"(b_[b + 3]), \
+    "+r"(b_[b + 4]), "+r"(b_[b + 5]), "+r"(b_[b + 6]), "+r"(b_[b + 7])
+
+// Waits for every tensor-memory load of this thread; the arrays of the loads
+// issued last are in-out operands, so no use of them moves above the wait.
+__device__ __forceinline__ void tmem_wait_ld8x2(uint32_t (&a)[8], uint32_t (&b_)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" : TRI_UA8(0), TRI_UB8(0) : : "memory");
+}
+
+#undef TRI_UA8
+#undef TRI_UB8
 #undef TRI_RA8
 #undef TRI_RB8
 #undef TRI_RC8
