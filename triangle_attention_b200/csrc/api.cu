@@ -108,7 +108,7 @@ struct BwdWs {
   float *D;
   // fp32 path: partial sums per tile, reduced by a second kernel
   float *part_dq, *part_dk, *part_dv;
-  // bf16 path: bf16 partials per tile
+  // bf16 path: bf16 contributions per tile, reduced by a second kernel
   __nv_bfloat16 *bpart_q, *bpart_k, *bpart_v;
   float *part_db;
   int ntile, ngroups;

@@ -374,7 +374,6 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int half = kbase / 64, chunk0 = (kbase % 64) / 8;   // place in the P/dS tiles
     const uint64_t c1x2 = f2pack(a.scale * kLog2e, a.scale * kLog2e);
     const uint64_t l2e2 = f2pack(kLog2e, kLog2e);
-    const int64_t pair = (int64_t)N * N * H * kC;
     bool ok = wait_bar_warp(&ctl.bias_full, 0, abort_flag, a.status);
     // this thread's kKeys dbias sums (fp32 pairs); its bias row stays in shared memory
     uint64_t dbias2[kKeys / 2];
@@ -386,29 +385,37 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t cswz = (uint32_t)(chunk0 ^ (row & 7));
     static_assert((kKeys / 8 & (kKeys / 8 - 1)) == 0, "key groups must be powers of two");
 
-    // Move the gradient partials of row t out of TMEM buffer t & 1 to the
-    // per-tile partial tensors, in six 16-column pieces (dQ 0/16, dK 0/16,
-    // dV 0/16) dealt round-robin to the warpgroups.
+    // Gradient pieces: piece j (0..5) is the 16 channels 16*(j&1).. of dQ (j < 2),
+    // dK (j < 4) or dV, for this warp's 32 lanes; warpgroup wg owns the pieces
+    // j = wg, wg + kEltGroups, ... A piece of row r is one tile's contribution:
+    // dQ of query tile xb (to be summed over key tiles), dK/dV of key tile yb (to
+    // be summed over query tiles). Contributions are stored piece-major,
+    // [t][r][h][j&1][i][16] (t the tile summed over, i the query or key), so one
+    // warp's piece fills eight whole 128-byte lines.
+    const int64_t pair = (int64_t)N * N * H * kC;
+    auto piece_base = [&](int j, int r) -> __nv_bfloat16 * {
+      __nv_bfloat16 *buf = j < 2 ? a.part_q : j < 4 ? a.part_k : a.part_v;
+      return buf + ((((int64_t)r * H + h) * 2 + (j & 1)) * N) * 16;
+    };
+
+    // Row t's pieces from TMEM buffer t & 1 to this tile's contribution slots.
     auto drain = [&](int t) -> bool {
       const int b = t & 1;
       if (!wait_bar_warp(&ctl.part_full[b], (t >> 1) & 1, abort_flag, a.status)) return false;
       tc_fence_after();
       const uint32_t tb = tl + b * kBufCols;
       const int r = r0 + t;
-      const int y = yb * kBN + row;             // key of this TMEM lane for dK/dV
-      const int64_t qoff = yb * pair + (((int64_t)r * N + x) * H + h) * kC;
-      const int64_t koff = xb * pair + (((int64_t)r * N + y) * H + h) * kC;
       for (int j = wg; j < 6; j += kEltGroups) {
         const uint32_t col = j < 2 ? kColDQ + 16 * j : j < 4 ? kColDK + 16 * (j - 2)
                                                              : kColDV + 16 * (j - 4);
-        uint32_t v[16];
-        tmem_ld16(tb + col, v);
-        if (j < 2) {
-          if (x < N) store_bf16<16>(a.part_q + qoff + 16 * j, v);
-        } else if (j < 4) {
-          if (y < N) store_bf16<16>(a.part_k + koff + 16 * (j - 2), v);
-        } else {
-          if (y < N) store_bf16<16>(a.part_v + koff + 16 * (j - 4), v);
+        const int i = (j < 2 ? xb : yb) * kBM + row;
+        const int tsum = j < 2 ? yb : xb;
+        __nv_bfloat16 *dst = piece_base(j, r) + tsum * pair + (int64_t)i * 16;
+#pragma unroll
+        for (int c8 = 0; c8 < 2; ++c8) {     // 8 columns at a time keeps registers low
+          uint32_t v[8];
+          tmem_ld8(tb + col + 8 * c8, v);
+          if (i < N) store_bf16<8>(dst + 8 * c8, v);
         }
       }
       tc_fence_before();

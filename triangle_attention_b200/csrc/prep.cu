@@ -109,8 +109,9 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
   }
 }
 
-// One thread per 8 channels of one output element of one of the three tensors:
-// the nb tile partials are summed in tile order in fp32, scaled, rounded once.
+// One thread per 8 channels of one contribution row: consecutive threads read
+// consecutive 16-byte groups of the [tile][row][H][2][N][16] contributions; the
+// nb tiles are summed in tile order in fp32, scaled and rounded once.
 __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ pq,
                                            const __nv_bfloat16 *__restrict__ pk,
                                            const __nv_bfloat16 *__restrict__ pv, int nb,
@@ -118,23 +119,23 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
                                            __nv_bfloat16 *__restrict__ dk,
                                            __nv_bfloat16 *__restrict__ dv) {
   const int64_t pair = (int64_t)f.N * f.N * f.H * 32;
-  const int64_t per = pair / 8;                 // 16-byte groups per tensor
+  const int64_t per = pair / 8;                 // 16-byte groups per tensor and tile
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < 3 * per;
        w += (int64_t)gridDim.x * blockDim.x) {
     const int which = (int)(w / per);
     const int64_t gidx = w - which * per;
-    const __nv_bfloat16 *src = which == 0 ? pq : which == 1 ? pk : pv;
+    const __nv_bfloat16 *src = (which == 0 ? pq : which == 1 ? pk : pv) + gidx * 8;
     const float sc = which == 2 ? 1.0f : scale;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-    // kBatch partials in flight per thread, then added in tile order
+    // kBatch contributions in flight per thread, then added in tile order
     constexpr int kBatch = 8;
     for (int t0 = 0; t0 < nb; t0 += kBatch) {
       uint4 v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u)
-        if (t0 + u < nb) v[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (t0 + u) * pair) + gidx);
+        if (t0 + u < nb) v[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (t0 + u) * pair));
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         if (t0 + u >= nb) break;
@@ -146,14 +147,14 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
         }
       }
     }
-    // compact index (r, x, h, c8) -> storage position through the frame
-    const int64_t cidx = gidx * 8;
-    const int h = (int)((cidx / 32) % f.H);
-    const int64_t x = (cidx / (32 * f.H)) % f.N;
-    const int64_t r = cidx / (32 * (int64_t)f.H * f.N);
-    const int c0 = (int)(cidx % 32);
-    __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + r * f.sR + x * f.sX +
-                         (int64_t)h * 32 + c0;
+    // gidx -> (r, h, half, i, c8) of the [r][H][2][N][16] layout
+    const int c8 = (int)(gidx & 1);
+    const int64_t i = (gidx >> 1) % f.N;
+    const int half = (int)((gidx >> 1) / f.N % 2);
+    const int h = (int)((gidx >> 1) / ((int64_t)f.N * 2) % f.H);
+    const int64_t r = (gidx >> 1) / ((int64_t)f.N * 2 * f.H);
+    __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + r * f.sR + i * f.sX +
+                         (int64_t)h * 32 + half * 16 + c8 * 8;
     *reinterpret_cast<uint4 *>(dst) =
         make_uint4(pack_bf16(acc[0] * sc, acc[1] * sc), pack_bf16(acc[2] * sc, acc[3] * sc),
                    pack_bf16(acc[4] * sc, acc[5] * sc), pack_bf16(acc[6] * sc, acc[7] * sc));

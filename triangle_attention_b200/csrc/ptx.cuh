@@ -130,7 +130,26 @@ __device__ __forceinline__ void discard_l2_line(const void *p) {
   asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
 }
 
-// 16-byte load that bypasses L1 (data written by other CTAs of this grid).
+// Device-scope fetch-and-add with acquire-release semantics: this thread's
+// earlier writes (and those ordered before them by a barrier) are visible to
+// whoever observes the new value; later reads see what the earlier arrivals
+// published.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t *p, int v) {
+  int old;
+  asm volatile("atom.add.acq_rel.gpu.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// 16-byte loads that bypass L1 (data written by other CTAs of this grid).
+__device__ __forceinline__ uint4 ld_cg_u4(const uint4 *p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ float4 ld_cg_f4(const float *p) {
   float4 v;
   asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -211,6 +230,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
       "tcgen05.wait::ld.sync.aligned;\n"
       : TRI_R8(0), TRI_R8(8), TRI_R8(16), TRI_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+
+// 8 consecutive columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : TRI_R8(0)
       : "r"(taddr)
       : "memory");
 }
