@@ -59,6 +59,9 @@ constexpr int kEltThreads = kEltGroups * 128;
 constexpr bool kPackOnIntegerPipes = false;
 // elementwise arithmetic on fp32 pairs (fma.rn.f32x2 and friends) or scalars
 constexpr bool kPairArithmetic = true;
+// the producer asks L2 for the input tiles of row it + kL2Ahead while it loads
+// row it (0: no prefetch)
+constexpr int kL2Ahead = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kBufCols = 256;
 constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 0, kColDK = 32, kColDV = 64;
@@ -285,6 +288,22 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_load(rd + kStMask, a.mask_bits + (int64_t)r * a.mask_bits_stride + yb * 4, 16,
                   &ctl.in_full[st]);
         armed[st] = it / kStages;
+        if (kL2Ahead > 0 && it + kL2Ahead < T) {
+          const int rp = r + kL2Ahead;
+          if (a.x_inner) {
+            tma_prefetch_l2_4d(&tm_q, 0, h, xb * kBM, rp);
+            tma_prefetch_l2_4d(&tm_k, 0, h, yb * kBN, rp);
+            tma_prefetch_l2_4d(&tm_v, 0, h, yb * kBN, rp);
+          } else {
+            tma_prefetch_l2_4d(&tm_q, 0, h, rp, xb * kBM);
+            tma_prefetch_l2_4d(&tm_k, 0, h, rp, yb * kBN);
+            tma_prefetch_l2_4d(&tm_v, 0, h, rp, yb * kBN);
+          }
+          tma_prefetch_l2_4d(&tm_du, 0, h, xb * kBM, rp);
+          const int64_t lp = ((int64_t)rp * H + h) * N + xb * kBM;
+          bulk_prefetch_l2(a.lse + lp, row_bytes);
+          bulk_prefetch_l2(a.D + lp, row_bytes);
+        }
       }
       if (!ok) {
         mbar_wait(&ctl.bias_full, 0);
@@ -389,13 +408,14 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // dK (j < 4) or dV, for this warp's 32 lanes; warpgroup wg owns the pieces
     // j = wg, wg + kEltGroups, ... A piece of row r is one tile's contribution:
     // dQ of query tile xb (to be summed over key tiles), dK/dV of key tile yb (to
-    // be summed over query tiles). Contributions are stored piece-major,
-    // [t][r][h][j&1][i][16] (t the tile summed over, i the query or key), so one
-    // warp's piece fills eight whole 128-byte lines.
+    // be summed over query tiles). Contributions are stored channel-group-major,
+    // [t][r][h][c/8][i][8] (t the tile summed over, i the query or key), so each
+    // warp store writes 512 contiguous bytes.
     const int64_t pair = (int64_t)N * N * H * kC;
-    auto piece_base = [&](int j, int r) -> __nv_bfloat16 * {
+    // channel group g (0..3) of row r of one tensor's contributions
+    auto group_base = [&](int j, int r, int g) -> __nv_bfloat16 * {
       __nv_bfloat16 *buf = j < 2 ? a.part_q : j < 4 ? a.part_k : a.part_v;
-      return buf + ((((int64_t)r * H + h) * 2 + (j & 1)) * N) * 16;
+      return buf + ((((int64_t)r * H + h) * 4 + g) * N) * 8;
     };
 
     // Row t's pieces from TMEM buffer t & 1 to this tile's contribution slots.
@@ -410,12 +430,12 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                              : kColDV + 16 * (j - 4);
         const int i = (j < 2 ? xb : yb) * kBM + row;
         const int tsum = j < 2 ? yb : xb;
-        __nv_bfloat16 *dst = piece_base(j, r) + tsum * pair + (int64_t)i * 16;
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {     // 8 columns at a time keeps registers low
           uint32_t v[8];
           tmem_ld8(tb + col + 8 * c8, v);
-          if (i < N) store_bf16<8>(dst + 8 * c8, v);
+          if (i < N)
+            store_bf16<8>(group_base(j, r, 2 * (j & 1) + c8) + tsum * pair + (int64_t)i * 8, v);
         }
       }
       tc_fence_before();
