@@ -59,6 +59,11 @@ constexpr int kEltThreads = kEltGroups * 128;
 constexpr bool kPackOnIntegerPipes = false;
 // elementwise arithmetic on fp32 pairs (fma.rn.f32x2 and friends) or scalars
 constexpr bool kPairArithmetic = true;
+// chunk (of kKeys / 8) at which warpgroup wg drains the previous row's
+// gradients: two warpgroups at a time (one with two pieces, one with one), the
+// later pair early enough to leave time for the next S/dP products
+__device__ constexpr int kDrainChunk[4] = {2, 3, 2, 3};
+static_assert(kEltGroups == 4, "drain schedule written for four warpgroups");
 // the producer asks L2 for the input tiles of row it + kL2Ahead while it loads
 // row it (0: no prefetch)
 constexpr int kL2Ahead = 4;
@@ -402,6 +407,9 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // 16-byte chunk chunk0 + ch of the swizzled row is at (cswz ^ ch) (chunk0 is a
     // multiple of kKeys / 8, so adding ch never carries into its bits)
     const uint32_t cswz = (uint32_t)(chunk0 ^ (row & 7));
+    // Each warpgroup drains the previous row's gradients at its own 8-key chunk,
+    // so the stores of the four warpgroups do not all leave the SM at once.
+    const int drain_chunk = kDrainChunk[wg];
     static_assert((kKeys / 8 & (kKeys / 8 - 1)) == 0, "key groups must be powers of two");
 
     // Gradient pieces: piece j (0..5) is the 16 channels 16*(j&1).. of dQ (j < 2),
@@ -490,8 +498,8 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
         for (int ch = 0; ch < kKeys / 8; ++ch) {
           const int cur = ch & 1, nxt = cur ^ 1;
-          if (ch == kKeys / 16 && it >= 1) {
-            // half-way through this row the previous row's gradients are done
+          if (ch == drain_chunk && it >= 1) {
+            // the previous row's gradients are done by now
             if (!drain(it - 1)) return false;
           }
           if (ch + 1 < kKeys / 8)
