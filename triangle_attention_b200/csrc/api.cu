@@ -169,13 +169,13 @@ EncodeTiledFn encode_fn() {
 // A pair tensor [.., .., H, 32] bf16 seen through the frame; dimensions by
 // increasing stride (c, h, then the smaller of x/r), box = one 128 x 32 tile.
 bool encode_pair(CUtensorMap *m, const void *base, int64_t N, int64_t H, int64_t sR, int64_t sX,
-                 bool x_inner) {
+                 bool x_inner, uint32_t box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[4] = {32, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)N};
   cuuint64_t strides[3] = {64, (cuuint64_t)((x_inner ? sX : sR) * 2),
                            (cuuint64_t)((x_inner ? sR : sX) * 2)};
-  cuuint32_t box[4] = {32, 1, x_inner ? 128u : 1u, x_inner ? 1u : 128u};
+  cuuint32_t box[4] = {32, 1, x_inner ? box_rows : 1u, x_inner ? 1u : box_rows};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -286,9 +286,10 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   const bool x_inner = prob->variant == TRI_ATTN_STARTING;
   tri::FwdMaps maps;
   const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.biasT : bias;
+  const uint32_t kv_rows = (uint32_t)tri::fwd_bf16_key_tile();
   if (!encode_pair(&maps.q, q, prob->N, prob->H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.k, k, prob->N, prob->H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.v, v, prob->N, prob->H, f.sR, f.sX, x_inner) ||
+      !encode_pair(&maps.k, k, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows) ||
+      !encode_pair(&maps.v, v, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows) ||
       !encode_bias(&maps.bias, bias_frame, prob->N, prob->H))
     return TRI_ATTN_ERR_CUDA;
   tri::FwdArgs a;

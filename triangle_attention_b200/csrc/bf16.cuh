@@ -37,6 +37,7 @@ struct FwdArgs {
 };
 
 int fwd_bf16_rows_per_cta();
+int fwd_bf16_key_tile();           // keys per K/V tile (rows of the K and V boxes)
 cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream);
 
 // ----------------------------------------------------------------- backward --

@@ -1,32 +1,31 @@
 // bf16 forward of gated triangle self-attention on sm_100a (tcgen05 + TMA).
 //
-// Work unit: one CTA owns (query tile of 128, head h, group of R attention
-// rows). The N^3*H logits never leave the chip: for each key tile the CTA
-// stages the 128x128 pair-bias tile once by TMA (shared by all R rows, since
-// the bias does not depend on the row) and then, row by row, computes
-// S = Q K^T on the tensor cores into tensor memory, turns it into
-// probabilities with an online softmax, and accumulates O += P V in tensor
-// memory. The probabilities never exist as a whole: each tile is produced and
-// consumed on chip ("MegaFold: Efficient Training of Next-Generation 3D
-// Attention Protein Models on Cross-Platform GPUs", tool 1, EvoFlash-3D). The
-// sigmoid gate, the key mask and the log-sum-exp save are fused into the same
-// kernel ("HelixFold: An Efficient Implementation of AlphaFold2 using
-// PaddlePaddle", proposed methods: fused gated self-attention).
+// Work unit: one CTA owns (query tile of 128, head h, group of 8 attention
+// rows). The N^3*H logits never leave the chip: for each key tile of 64 the CTA
+// stages the 128x64 pair-bias tile once by TMA (shared by all 8 rows, since the
+// bias does not depend on the row) and then, row by row, computes S = Q K^T on
+// the tensor cores into tensor memory, turns it into probabilities with an
+// online softmax, and accumulates O += P V in tensor memory. The probabilities
+// never exist as a whole: each tile is produced and consumed on chip
+// ("MegaFold: Efficient Training of Next-Generation 3D Attention Protein Models
+// on Cross-Platform GPUs", tool 1, EvoFlash-3D). The sigmoid gate, the key mask
+// and the log-sum-exp save are fused into the same kernel ("HelixFold: An
+// Efficient Implementation of AlphaFold2 using PaddlePaddle", proposed methods:
+// fused gated self-attention).
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer (one elected lane)
-//   warp 1      tensor-memory allocator and MMA issuer (one elected lane)
-//   warps 2..5  softmax / epilogue warpgroup 0: even rows of the CTA
-//   warps 6..9  softmax / epilogue warpgroup 1: odd rows
+// Warp roles (576 threads):
+//   warp 0       TMA producer (one elected lane)
+//   warp 1       tensor-memory allocator and MMA issuer (one elected lane)
+//   warps 2..17  four softmax / epilogue warpgroups; warpgroup w owns rows w and
+//                w + 4 of the CTA and the S buffer w
 // In a warpgroup, thread = query row of the tile (tensor-memory lane), so the
-// row max and row sum are thread-local. While one warpgroup turns its S tile
-// into probabilities, the tensor cores and the other warpgroup work on the
-// other row.
+// row max and row sum are thread-local. The four warpgroups cycle through their
+// rows independently: while one waits for the tensor cores (its P V product and
+// its next S), the other three turn their S tiles into probabilities.
 //
-// Tensor memory (512 columns): one S buffer per warpgroup at columns 0 and 128
-// (the bf16 probabilities overwrite the first 64 columns of their S buffer and
-// feed the PV MMA straight from tensor memory); O accumulators of the 8 rows at
-// 256 + 32*rr.
+// Tensor memory (512 columns): S buffer w (64 fp32 columns) at 64*w; the bf16
+// probabilities overwrite its first 32 columns and feed the PV product straight
+// from tensor memory. O accumulators of the 8 rows at 256 + 32*rr.
 #include <cmath>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -39,18 +38,22 @@ namespace tri {
 namespace {
 
 constexpr int kBM = 128;          // queries per tile
-constexpr int kBN = 128;          // keys per tile
+constexpr int kBN = 64;           // keys per tile
 constexpr int kC = 32;            // head dimension
 constexpr int kRows = 8;          // attention rows per CTA
-constexpr int kStages = 4;        // K/V pipeline depth
-constexpr int kThreads = 320;
+constexpr int kGroups = 4;        // softmax warpgroups; warpgroup w owns rows w, w + 4
+constexpr int kStages = 8;        // K/V pipeline depth (each stage 8 KB)
+constexpr int kThreads = 64 + 128 * kGroups;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kPairTileBytes = kBM * kC * 2;   // 8 KB
-constexpr uint32_t kBiasTileBytes = kBM * kBN * 2;  // 32 KB (two 16 KB halves)
+constexpr uint32_t kColO = kGroups * kBN;           // 256
+constexpr uint32_t kQTileBytes = kBM * kC * 2;      // 8 KB
+constexpr uint32_t kKVTileBytes = kBN * kC * 2;     // 4 KB
+constexpr uint32_t kBiasTileBytes = kBM * kBN * 2;  // 16 KB: 128 rows of 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // bf16 rounding of P: on the integer pipes (true) or with cvt.rn (false)
 constexpr bool kPackOnIntegerPipes = false;
+static_assert(kRows == 2 * kGroups, "each warpgroup owns two rows");
 
 struct __align__(8) FwdSmem {
   uint64_t q_full;
@@ -58,8 +61,8 @@ struct __align__(8) FwdSmem {
   uint64_t kv_empty[kStages];
   uint64_t bias_full[2];
   uint64_t bias_empty[2];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[kGroups];
+  uint64_t p_full[kGroups];
   uint64_t o_done[kRows];
   uint64_t o_final;
   uint64_t teardown;
@@ -68,12 +71,13 @@ struct __align__(8) FwdSmem {
 };
 
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kRows * kPairTileBytes;
-constexpr uint32_t kOffV = kOffK + kStages * kPairTileBytes;
-constexpr uint32_t kOffB = kOffV + kStages * kPairTileBytes;
+constexpr uint32_t kOffK = kOffQ + kRows * kQTileBytes;
+constexpr uint32_t kOffV = kOffK + kStages * kKVTileBytes;
+constexpr uint32_t kOffB = kOffV + kStages * kKVTileBytes;
 constexpr uint32_t kOffMask = kOffB + 2 * kBiasTileBytes;   // 16 bytes of key bits per stage
 constexpr uint32_t kOffCtl = kOffMask + kStages * 16;
 constexpr uint32_t kSmemBytes = kOffCtl + sizeof(FwdSmem) + 1024;  // +1024 for alignment
+static_assert(kOffB % 1024 == 0, "128-byte-swizzled bias tiles need 1 KB alignment");
 
 // Bounded wait on an mbarrier that also gives up once another role aborted.
 // Warp-uniform when every lane of the warp calls it.
@@ -101,16 +105,14 @@ __device__ __forceinline__ bool wait_bar_warp(uint64_t *bar, uint32_t parity,
 
 // Exponents (s*c^-1/2 + b)*log2e - m of 32 keys (raw S bits in u, keys
 // 32*c32.. of the tile) of this thread's query row, in place; bias from the
-// 128-byte-swizzled tile in shared memory.
+// 128-byte-swizzled tile row in shared memory.
 __device__ __forceinline__ void exponents32(uint32_t (&u)[32], const uint8_t *brow, int row,
                                             int c32, uint64_t c1x2, uint64_t l2e2,
                                             uint64_t nm2) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int ch = c32 * 4 + q;              // 16-byte chunk of 8 keys
-    const int hh = ch >> 3, cc = ch & 7;
-    const uint4 bv = *reinterpret_cast<const uint4 *>(brow + hh * (kBiasTileBytes / 2) +
-                                                      ((cc ^ (row & 7)) << 4));
+    const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((ch ^ (row & 7)) << 4));
     const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -159,7 +161,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int r0 = blockIdx.z * kRows;
   const int nrows = min(kRows, N - r0);
   const int nkb = (N + kBN - 1) / kBN;
-  const int T = nkb * nrows;
+  const int T = nkb * kRows;        // (key tile, row) steps, row fastest
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.q_full, 1);
@@ -169,9 +171,11 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl.bias_full[b], 1);
-      mbar_init(&ctl.bias_empty[b], 256);
-      mbar_init(&ctl.s_full[b], 1);
-      mbar_init(&ctl.p_full[b], 128);   // buffer b belongs to warpgroup b
+      mbar_init(&ctl.bias_empty[b], 128 * kGroups);
+    }
+    for (int w = 0; w < kGroups; ++w) {
+      mbar_init(&ctl.s_full[w], 1);
+      mbar_init(&ctl.p_full[w], 128);   // buffer w belongs to warpgroup w
     }
     for (int rr = 0; rr < kRows; ++rr) mbar_init(&ctl.o_done[rr], 1);
     mbar_init(&ctl.o_final, 1);
@@ -190,7 +194,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
-    if (elect_one()) {
+    if (elect_one() && nrows == kRows) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -199,9 +203,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int armed_b[2] = {-1, -1};
       for (int s = 0; s < kStages; ++s) armed_kv[s] = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(&ctl.q_full, nrows * kPairTileBytes);
-      for (int rr = 0; rr < nrows; ++rr) {
-        uint8_t *dst = smem + kOffQ + rr * kPairTileBytes;
+      mbar_arrive_expect_tx(&ctl.q_full, kRows * kQTileBytes);
+      for (int rr = 0; rr < kRows; ++rr) {
+        uint8_t *dst = smem + kOffQ + rr * kQTileBytes;
         if (a.x_inner)
           tma_load_4d(dst, &tm_q, &ctl.q_full, 0, h, xb * kBM, r0 + rr);
         else
@@ -214,21 +218,20 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           ok = false;
           break;
         }
-        uint8_t *bsm = smem + kOffB + bb * kBiasTileBytes;
         mbar_arrive_expect_tx(&ctl.bias_full[bb], kBiasTileBytes);
-        tma_load_3d(bsm, &tm_b, &ctl.bias_full[bb], kb * kBN, xb * kBM, h);
-        tma_load_3d(bsm + kBiasTileBytes / 2, &tm_b, &ctl.bias_full[bb], kb * kBN + 64, xb * kBM, h);
+        tma_load_3d(smem + kOffB + bb * kBiasTileBytes, &tm_b, &ctl.bias_full[bb], kb * kBN,
+                    xb * kBM, h);
         armed_b[bb] = kb >> 1;
-        for (int rr = 0; rr < nrows; ++rr, ++it) {
+        for (int rr = 0; rr < kRows; ++rr, ++it) {
           const int st = it % kStages;
           if (it >= kStages &&
               !wait_bar(&ctl.kv_empty[st], ((it / kStages) - 1) & 1, abort_flag, a.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&ctl.kv_full[st], 2 * kPairTileBytes + 16);
-          uint8_t *kd = smem + kOffK + st * kPairTileBytes;
-          uint8_t *vd = smem + kOffV + st * kPairTileBytes;
+          mbar_arrive_expect_tx(&ctl.kv_full[st], 2 * kKVTileBytes + 16);
+          uint8_t *kd = smem + kOffK + st * kKVTileBytes;
+          uint8_t *vd = smem + kOffV + st * kKVTileBytes;
           if (a.x_inner) {
             tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
             tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
@@ -236,8 +239,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
             tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
           }
+          // the 4 key-bit words of the 128 keys around this tile (16-byte aligned)
           bulk_load(smem + kOffMask + st * 16,
-                    a.mask_bits + (int64_t)(r0 + rr) * a.mask_bits_stride + kb * 4, 16,
+                    a.mask_bits + (int64_t)(r0 + rr) * a.mask_bits_stride + (kb >> 1) * 4, 16,
                     &ctl.kv_full[st]);
           armed_kv[st] = it / kStages;
         }
@@ -253,47 +257,50 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer --
-    if (elect_one()) {
+    if (elect_one() && nrows == kRows) {
       const uint32_t id_s = make_idesc_bf16(kBM, kBN, false, false);
       const uint32_t id_pv = make_idesc_bf16(kBM, kC, false, true);
       bool ok = wait_bar(&ctl.q_full, 0, abort_flag, a.status);
       tc_fence_after();
-      int it = 0;
+      // S of step t into the S buffer of its warpgroup
       auto issue_s = [&](int t) -> bool {
-        const int rr = t % nrows, st = t % kStages, sb = t & 1;
+        const int w = t % kGroups, rr = t % kRows, st = t % kStages;
         if (!wait_bar(&ctl.kv_full[st], (t / kStages) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
-        const uint32_t qa = smem_u32(smem + kOffQ + rr * kPairTileBytes);
-        const uint32_t ka = smem_u32(smem + kOffK + st * kPairTileBytes);
+        const uint32_t qa = smem_u32(smem + kOffQ + rr * kQTileBytes);
+        const uint32_t ka = smem_u32(smem + kOffK + st * kKVTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kC / 16; ++ks) {
           const uint64_t da = make_sdesc(qa + ks * 32, 16, 512, kSwizzle64B);
           const uint64_t db = make_sdesc(ka + ks * 32, 16, 512, kSwizzle64B);
-          mma_ss(tmem + sb * kBN, da, db, id_s, ks > 0 ? 1u : 0u);
+          mma_ss(tmem + w * kBN, da, db, id_s, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&ctl.s_full[sb]);
+        mma_commit(&ctl.s_full[w]);
         return true;
       };
+      // O[row] += P V of step t, P read from the warpgroup's S buffer
       auto issue_pv = [&](int t) -> bool {
-        const int rr = t % nrows, kb = t / nrows, st = t % kStages, sb = t & 1;
-        if (!wait_bar(&ctl.p_full[sb], (t >> 1) & 1, abort_flag, a.status)) return false;
+        const int w = t % kGroups, rr = t % kRows, kb = t / kRows, st = t % kStages;
+        if (!wait_bar(&ctl.p_full[w], (t / kGroups) & 1, abort_flag, a.status)) return false;
         tc_fence_after();
-        const uint32_t va = smem_u32(smem + kOffV + st * kPairTileBytes);
+        const uint32_t va = smem_u32(smem + kOffV + st * kKVTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
           const uint64_t db = make_sdesc(va + ks * 16 * 64, 512, 512, kSwizzle64B);
-          mma_ts(tmem + 2 * kBN + rr * kC, tmem + sb * kBN + ks * 8, db, id_pv,
+          mma_ts(tmem + kColO + rr * kC, tmem + w * kBN + ks * 8, db, id_pv,
                  (kb > 0 || ks > 0) ? 1u : 0u);
         }
         mma_commit(&ctl.kv_empty[st]);
         mma_commit(&ctl.o_done[rr]);
         return true;
       };
-      for (it = 0; ok && it < T; ++it) {
-        ok = issue_s(it);
-        if (ok && it >= 1) ok = issue_pv(it - 1);
+      // The PV product of step t - kGroups reads the S buffer that S of step t
+      // overwrites, so it is issued first (the tensor pipe runs them in order).
+      for (int t = 0; ok && t < T; ++t) {
+        if (t >= kGroups) ok = issue_pv(t - kGroups);
+        if (ok) ok = issue_s(t);
       }
-      if (ok && T > 0) ok = issue_pv(T - 1);
+      for (int t = max(0, T - kGroups); ok && t < T; ++t) ok = issue_pv(t);
       mma_commit(&ctl.o_final);
       // No tensor-memory operation may be in flight when the CTA tears down.
       mma_commit(&ctl.teardown);
@@ -301,35 +308,23 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
   } else {
     // ------------------------------------------------ softmax and epilogue --
-    // Rows are handled in pairs: warpgroup wg owns the rows rr = 2j + wg and the
-    // S/P buffer wg (every CTA holds kRows = 8 rows, because N % 8 == 0).
     const int wg = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;           // query within the tile = TMEM lane
     const int x = xb * kBM + row;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const uint32_t sbuf = tl + wg * kBN;
-    constexpr int kMine = kRows / 2;
     const uint64_t c1x2 = f2pack(a.scale * kLog2e, a.scale * kLog2e);
     const uint64_t l2e2 = f2pack(kLog2e, kLog2e);
-    // running max and sum of this warpgroup's kMine rows; the loop over rows is
-    // not unrolled, so the registers rotate (row j's pair is always m_r[0],
-    // l_r[0]) instead of being indexed, which would put them in local memory
-    float m_r[kMine], l_r[kMine];
-#pragma unroll
-    for (int j = 0; j < kMine; ++j) {
-      m_r[j] = -INFINITY;
-      l_r[j] = 0.0f;
-    }
-    auto rotate_rows = [&]() {
+    // running max and sum of this warpgroup's two rows (rows wg and wg + 4); the
+    // loop over them is not unrolled, so the pair swaps instead of being indexed
+    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f};
+    auto swap_rows = [&]() {
       const float m0 = m_r[0], l0 = l_r[0];
-#pragma unroll
-      for (int j = 0; j + 1 < kMine; ++j) {
-        m_r[j] = m_r[j + 1];
-        l_r[j] = l_r[j + 1];
-      }
-      m_r[kMine - 1] = m0;
-      l_r[kMine - 1] = l0;
+      m_r[0] = m_r[1];
+      l_r[0] = l_r[1];
+      m_r[1] = m0;
+      l_r[1] = l0;
     };
     bool ok = nrows == kRows;
     if (!ok) {
@@ -343,37 +338,36 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         break;
       }
       const uint8_t *brow = smem + kOffB + bb * kBiasTileBytes + row * 128;
-      // max of this query row's 128 bias values (shared by all rows of the CTA)
+      // max of this query row's 64 bias values (shared by all rows of the CTA)
       float bmax = -INFINITY;
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const uint4 bv = *reinterpret_cast<const uint4 *>(brow + (ch >> 3) * (kBiasTileBytes / 2) +
-                                                          (((ch & 7) ^ (row & 7)) << 4));
+      for (int ch = 0; ch < 8; ++ch) {
+        const uint4 bv = *reinterpret_cast<const uint4 *>(brow + ((ch ^ (row & 7)) << 4));
         bmax = fmax3(bmax, fmax3(bf16lo(bv.x), bf16hi(bv.x), bf16lo(bv.y)),
                      fmax3(bf16hi(bv.y), fmax3(bf16lo(bv.z), bf16hi(bv.z), bf16lo(bv.w)),
                            bf16hi(bv.w)));
       }
 #pragma unroll 1
-      for (int j = 0; j < kMine; ++j) {
-        const int rr = 2 * j + wg;
+      for (int j = 0; j < 2; ++j, swap_rows()) {
+        const int rr = wg + kGroups * j;
         const int it = kb * kRows + rr;
         const int st = it % kStages;
         // key bits of this row and key tile arrive with the K/V stage
         if (!wait_bar_warp(&ctl.kv_full[st], (it / kStages) & 1, abort_flag, a.status) ||
-            !wait_bar_warp(&ctl.s_full[wg], (it >> 1) & 1, abort_flag, a.status)) {
+            !wait_bar_warp(&ctl.s_full[wg], (it / kGroups) & 1, abort_flag, a.status)) {
           ok = false;
           break;
         }
         const uint4 mw = *reinterpret_cast<const uint4 *>(smem + kOffMask + st * 16);
-        const bool full_tile = (mw.x & mw.y & mw.z & mw.w) == 0xffffffffu;
+        const uint32_t mk0 = (kb & 1) ? mw.z : mw.x, mk1 = (kb & 1) ? mw.w : mw.y;
+        const bool full_tile = (mk0 & mk1) == 0xffffffffu;
         tc_fence_after();
         // Pass 1: an upper bound of the row's logits, max(s) * c^-1/2 + max(b).
         // Softmax is exact for any shift; a bound keeps every exponent <= 0.
         float sm0 = -INFINITY, sm1 = -INFINITY;
-#pragma unroll 1
-        for (int c64 = 0; c64 < 2; ++c64) {
+        {
           uint32_t u[32], w[32];
-          tmem_ld32x2(sbuf + c64 * 64, sbuf + c64 * 64 + 32, u, w);
+          tmem_ld32x2(sbuf, sbuf + 32, u, w);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             sm0 = fmax3(sm0, __uint_as_float(u[e]), __uint_as_float(u[e + 1]));
@@ -388,22 +382,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float alpha = ex2_approx(m_old - m_new);   // m_old = -inf gives 0
         const uint64_t nm2 = f2pack(-m_new, -m_new);
         uint64_t sum_a = 0, sum_b = 0;   // two packed running sums (bit pattern 0 = 0.0f)
-        uint32_t pk[16];
 #pragma unroll 1
-        for (int c64 = 0; c64 < 2; ++c64) {
-          uint32_t u[32], w[32];
-          tmem_ld32x2(sbuf + c64 * 64, sbuf + c64 * 64 + 32, u, w);
-          const uint32_t mu = c64 == 0 ? mw.x : mw.z, mv = c64 == 0 ? mw.y : mw.w;
-          // P (bf16 pairs) of keys 64*c64.. goes to columns 32*c64..32*c64+31 of
-          // this S buffer, whose S values were already read into registers.
-          exponents32(u, brow, row, 2 * c64, c1x2, l2e2, nm2);
-          if (full_tile) probs32<false>(u, mu, sum_a, sum_b, pk);
-          else probs32<true>(u, mu, sum_a, sum_b, pk);
-          tmem_st16(sbuf + c64 * 32, pk);
-          exponents32(w, brow, row, 2 * c64 + 1, c1x2, l2e2, nm2);
-          if (full_tile) probs32<false>(w, mv, sum_a, sum_b, pk);
-          else probs32<true>(w, mv, sum_a, sum_b, pk);
-          tmem_st16(sbuf + c64 * 32 + 16, pk);
+        for (int c32 = 0; c32 < 2; ++c32) {
+          uint32_t u[32];
+          uint32_t pk[16];
+          tmem_ld32(sbuf + 32 * c32, u);
+          // P (bf16 pairs) of keys 32*c32.. goes to columns 16*c32.. of this S
+          // buffer, whose S values were already read into registers.
+          exponents32(u, brow, row, c32, c1x2, l2e2, nm2);
+          if (full_tile) probs32<false>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
+          else probs32<true>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
+          tmem_st16(sbuf + 16 * c32, pk);
         }
         const float2 sa = f2unpack(add2(sum_a, sum_b));
         l_r[0] = l_r[0] * alpha + (sa.x + sa.y);
@@ -417,7 +406,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
             uint32_t o[32];
-            const uint32_t oa = tl + 2 * kBN + rr * kC;
+            const uint32_t oa = tl + kColO + rr * kC;
             tmem_ld32(oa, o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
@@ -427,7 +416,6 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&ctl.p_full[wg]);
-        rotate_rows();
       }
       if (ok) mbar_arrive(&ctl.bias_empty[bb]);
     }
@@ -435,13 +423,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok) ok = wait_bar_warp(&ctl.o_final, 0, abort_flag, a.status);
     if (ok) tc_fence_after();
 #pragma unroll 1
-    for (int j = 0; j < kMine; ++j, rotate_rows()) {
-      const int rr = 2 * j + wg;
-      if (rr >= nrows) break;
+    for (int j = 0; j < 2; ++j, swap_rows()) {
+      const int rr = wg + kGroups * j;
       const int r = r0 + rr;
       uint32_t o[32];
-      if (ok) tmem_ld32(tl + 2 * kBN + rr * kC, o);
-      if (x >= N) continue;
+      if (ok) tmem_ld32(tl + kColO + rr * kC, o);
+      if (x >= N || rr >= nrows) continue;
       float *lse_p = a.lse + ((int64_t)r * a.H + h) * N + x;
       if (!ok) {
         *lse_p = __int_as_float(0x7fc00000);  // NaN marks a tile the kernel gave up on
@@ -483,6 +470,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }  // namespace
 
 int fwd_bf16_rows_per_cta() { return kRows; }
+int fwd_bf16_key_tile() { return kBN; }
 
 cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream) {
   if (args.N == 0) return cudaSuccess;
