@@ -140,16 +140,21 @@ class ClockSampler:
 
 # ------------------------------------------------------------- distributed --
 
-def dist_setup():
+def dist_setup(backend=None):
+    """One process per GPU (torchrun's RANK/LOCAL_RANK/WORLD_SIZE): NCCL over the
+    GPUs, or gloo when asked for (the CPU tests of the multi-process path)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return rank, world, local
 
 
@@ -160,12 +165,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Slowest rank's time: every rank contributes, every rank gets the maximum."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_replica_step: float, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas, each doing one step's FLOPs,
+    timed by the slowest rank (weak scaling)."""
+    return world * flops_per_replica_step / (ms_max * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------- CPU oracle --
@@ -322,7 +335,7 @@ def run_ours(args, rank, world, local, w):
     ms_local = t0.elapsed_time(t1) / args.steps
     ms = max_over_ranks(ms_local, world)
     f_fwd, f_bwd = flops(w.N, w.H, w.c)
-    value = world * (f_fwd + f_bwd) / (ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, f_fwd + f_bwd, ms)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
 

@@ -60,7 +60,6 @@ Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status
   return f;
 }
 
-size_t elem_size(const tri_attn_problem *p) { return p->dtype == TRI_ATTN_BF16 ? 2 : 4; }
 
 // ------------------------------------------------------- workspace layout --
 
