@@ -220,6 +220,20 @@ tri_attn_status tri_attn_fwd_noalloc(const tri_attn_problem *prob, const void *q
 tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_status,
                                      tri_attn_stream_t stream);
 
+/*
+ * Diagnostic of the failure path (no counterpart on the pages): enqueues one
+ * small kernel whose warp waits on a barrier that nothing ever completes,
+ * using the same bounded wait (about 2 s) as the forward and backward kernels.
+ * The wait gives up and the kernel writes TRI_ATTN_ERR_TIMEOUT to the status
+ * word at the start of `workspace` (which it first resets); it never traps or
+ * faults, so the stream and context stay usable. Read the result with
+ * tri_attn_read_status(). workspace: device, 16-byte aligned, at least 256
+ * bytes, caller-owned. Returns TRI_ATTN_ERR_WORKSPACE for a missing, misaligned
+ * or short workspace, TRI_ATTN_ERR_CUDA if the launch fails.
+ */
+tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
+                                            tri_attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -87,9 +87,11 @@ def lib():
         L.tri_attn_kernel_launches.argtypes = [PP, ctypes.c_int, ctypes.c_int,
                                                ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
+        L.tri_attn_check_wait_timeout.argtypes = [P, sz, P]
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
-                  L.tri_attn_kernel_launches, L.tri_attn_read_status):
+                  L.tri_attn_kernel_launches, L.tri_attn_read_status,
+                  L.tri_attn_check_wait_timeout):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -211,6 +213,14 @@ def read_status(ws: torch.Tensor, stream=None) -> int:
     _check(lib().tri_attn_read_status(_p(ws), ctypes.byref(v), _stream(stream)),
            "tri_attn_read_status")
     return v.value
+
+
+def check_wait_timeout(ws: torch.Tensor, stream=None) -> int:
+    """Runs the diagnostic kernel whose bounded wait nothing satisfies and
+    returns the status word it leaves (TIMEOUT when the wait gave up)."""
+    _check(lib().tri_attn_check_wait_timeout(_p(ws), ws.numel(), _stream(stream)),
+           "tri_attn_check_wait_timeout")
+    return read_status(ws, stream)
 
 
 class TriangleAttention(torch.autograd.Function):

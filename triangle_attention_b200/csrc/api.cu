@@ -484,4 +484,12 @@ tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_stat
   return TRI_ATTN_OK;
 }
 
+tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
+                                            tri_attn_stream_t stream) {
+  if (!workspace || !aligned16(workspace) || workspace_bytes < 256)
+    return TRI_ATTN_ERR_WORKSPACE;
+  return cuda_status(tri::launch_unsatisfied_wait(static_cast<int32_t *>(workspace),
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -31,6 +31,9 @@ __device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Diagnostic kernel: a bounded wait that nothing satisfies (see selftest.cu).
+cudaError_t launch_unsatisfied_wait(int32_t *status, cudaStream_t stream);
+
 __host__ __device__ inline int64_t pair_elems(const Frame &f) {
   return (int64_t)f.N * f.N * f.H * f.c;
 }
