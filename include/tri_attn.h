@@ -144,18 +144,34 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
 
 /*
  * Optional per-call settings of the _ex entry points. Zero-initialise, set
- * struct_size = sizeof(tri_attn_launch_opts), then fill what is needed.
+ * struct_size = sizeof(tri_attn_launch_opts), then fill what is needed. A
+ * struct_size of TRI_ATTN_LAUNCH_OPTS_V1_SIZE (the first four fields) is also
+ * accepted; fields past struct_size count as zero.
  *   main_start / main_stop: cudaEvent_t handles (or NULL) that the call
  *   records on its stream immediately before and after its main kernel (the
  *   attention kernel itself, without the small preparation and reduction
  *   kernels), so a caller can time that kernel alone with cudaEventElapsedTime.
+ *   out_residual: bf16 path only (NULL on the fp32 path, else
+ *   TRI_ATTN_ERR_UNSUPPORTED). Device, caller-owned, 16-byte aligned, shape and
+ *   layout of `out` (bf16). The forward writes there the part of each output
+ *   element that rounding to bf16 removed, itself rounded to bf16
+ *   (bf16(o - bf16(o)) for the fp32 value o); `out` is bit-identical with or
+ *   without it. The backward, given the same tensor, forms D = sum_c dout * out
+ *   and dgate from out + out_residual instead of the rounded out: the rounding
+ *   residual compensation of "TurboPairFormer accelera fino a 1,73x
+ *   l'addestramento di OpenFold3 nei test" (section "Accuratezza e
+ *   riproducibilita"), which lowers the error of dq, dk and dbias; dv does not
+ *   depend on D and is unchanged. NULL: no residual.
  */
 typedef struct {
     uint32_t struct_size;
     uint32_t flags;           /* reserved, must be 0 */
     void *main_start;
     void *main_stop;
+    void *out_residual;
 } tri_attn_launch_opts;
+
+#define TRI_ATTN_LAUNCH_OPTS_V1_SIZE ((uint32_t)(2 * sizeof(uint32_t) + 2 * sizeof(void *)))
 
 /* tri_attn_fwd with options (opts may be NULL: same as tri_attn_fwd). */
 tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,

@@ -43,18 +43,31 @@ class TriAttnError(RuntimeError):
 
 class LaunchOpts(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("flags", ctypes.c_uint32),
-                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p)]
+                ("main_start", ctypes.c_void_p), ("main_stop", ctypes.c_void_p),
+                ("out_residual", ctypes.c_void_p)]
 
 
-def launch_opts(main_start=None, main_stop=None) -> LaunchOpts:
-    """Options whose torch.cuda.Event objects are recorded around the main kernel."""
+def launch_opts(main_start=None, main_stop=None, residual=None) -> LaunchOpts:
+    """Options: torch.cuda.Event objects recorded around the main kernel, and
+    the bf16 rounding residual of `out` (a tensor shaped like out) that the
+    forward writes and the backward uses for D and dgate."""
     def handle(ev):
         if ev is None:
             return None
         if not ev.cuda_event:            # torch creates the event lazily
             ev.record()
         return ctypes.c_void_p(ev.cuda_event)
-    return LaunchOpts(ctypes.sizeof(LaunchOpts), 0, handle(main_start), handle(main_stop))
+    return LaunchOpts(ctypes.sizeof(LaunchOpts), 0, handle(main_start), handle(main_stop),
+                      None if residual is None else ctypes.c_void_p(residual.data_ptr()))
+
+
+def _with_residual(opts, residual):
+    if residual is None:
+        return opts
+    if opts is None:
+        return launch_opts(residual=residual)
+    opts.out_residual = ctypes.c_void_p(residual.data_ptr())
+    return opts
 
 
 class Problem(ctypes.Structure):
@@ -169,9 +182,12 @@ def _contig(*ts):
 
 
 def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=None, ws=None,
-        stream=None, opts: Optional[LaunchOpts] = None):
-    """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N]."""
-    _contig(q, k, v, bias, gate, mask)
+        stream=None, opts: Optional[LaunchOpts] = None, residual=None):
+    """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N].
+    residual (bf16 path): a tensor shaped like out that receives out's rounding
+    residual, for the compensated backward."""
+    _contig(q, k, v, bias, gate, mask, residual)
+    opts = _with_residual(opts, residual)
     prob = problem(q, mask, variant)
     N, _, H, _ = q.shape
     if out is None:
@@ -188,9 +204,12 @@ def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=N
 
 
 def bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, grads=None, ws=None,
-        stream=None, opts: Optional[LaunchOpts] = None):
-    """Backward. Returns (dq, dk, dv, dbias, dgate) in the inputs' dtype."""
-    _contig(q, k, v, bias, gate, mask, out, lse, dout)
+        stream=None, opts: Optional[LaunchOpts] = None, residual=None):
+    """Backward. Returns (dq, dk, dv, dbias, dgate) in the inputs' dtype.
+    residual: the tensor the forward filled, to form D and dgate from out plus
+    its rounding residual."""
+    _contig(q, k, v, bias, gate, mask, out, lse, dout, residual)
+    opts = _with_residual(opts, residual)
     prob = problem(q, mask, variant)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),

@@ -2,6 +2,7 @@
 // workspace carving, TMA tensor-map encoding and dispatch to the kernels.
 // Nothing here allocates device memory or keeps state between calls.
 #include <cmath>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <cuda.h>
@@ -201,6 +202,25 @@ tri_attn_status cuda_status(cudaError_t e) {
 }
 
 // Record the caller's timing event before (start) or after (stop) the main kernel.
+// The residual tensor of the options (NULL when absent or past struct_size).
+void *opt_residual(const tri_attn_launch_opts *opts) {
+  if (!opts || opts->struct_size < offsetof(tri_attn_launch_opts, out_residual) + sizeof(void *))
+    return nullptr;
+  return opts->out_residual;
+}
+
+// Options are well formed: a known size, no flags, an aligned residual that
+// only the bf16 path takes.
+tri_attn_status check_opts(const tri_attn_problem *prob, const tri_attn_launch_opts *opts) {
+  if (!opts) return TRI_ATTN_OK;
+  if (opts->struct_size < TRI_ATTN_LAUNCH_OPTS_V1_SIZE || opts->flags != 0)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  const void *res = opt_residual(opts);
+  if (res && !aligned16(res)) return TRI_ATTN_ERR_INVALID_ARG;
+  if (res && prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
 cudaError_t mark(const tri_attn_launch_opts *opts, bool start, cudaStream_t stream) {
   if (!opts) return cudaSuccess;
   void *ev = start ? opts->main_start : opts->main_stop;
@@ -253,9 +273,9 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
                                 const uint8_t *mask, void *out, float *lse, void *workspace,
                                 size_t workspace_bytes, tri_attn_stream_t stream_,
                                 const tri_attn_launch_opts *opts) {
-  if (opts && (opts->struct_size < sizeof(tri_attn_launch_opts) || opts->flags != 0))
-    return TRI_ATTN_ERR_INVALID_ARG;
   tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  st = check_opts(prob, opts);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
@@ -300,6 +320,7 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   a.sX = f.sX;
   a.gate = static_cast<const __nv_bfloat16 *>(gate);
   a.out = static_cast<__nv_bfloat16 *>(out);
+  a.out_res = static_cast<__nv_bfloat16 *>(opt_residual(opts));
   a.lse = lse;
   a.mask_bits = w.mask_bits;
   a.mask_bits_stride = rows > 1 ? words : 0;
@@ -329,9 +350,9 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                 const void *dout, void *dq, void *dk, void *dv, void *dbias,
                                 void *dgate, void *workspace, size_t workspace_bytes,
                                 tri_attn_stream_t stream_, const tri_attn_launch_opts *opts) {
-  if (opts && (opts->struct_size < sizeof(tri_attn_launch_opts) || opts->flags != 0))
-    return TRI_ATTN_ERR_INVALID_ARG;
   tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  st = check_opts(prob, opts);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
@@ -413,6 +434,7 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   if (e == cudaSuccess)
     e = tri::launch_bwd_pre_bf16(f, static_cast<const __nv_bfloat16 *>(gate),
                                  static_cast<const __nv_bfloat16 *>(out),
+                                 static_cast<const __nv_bfloat16 *>(opt_residual(opts)),
                                  static_cast<const __nv_bfloat16 *>(dout),
                                  static_cast<__nv_bfloat16 *>(w.du), w.D,
                                  static_cast<__nv_bfloat16 *>(dgate), stream);

@@ -30,6 +30,7 @@ struct FwdArgs {
   int64_t sR, sX;                    // pair strides of the variant frame (elements)
   const __nv_bfloat16 *gate;
   __nv_bfloat16 *out;
+  __nv_bfloat16 *out_res;            // rounding residual of out (bf16) or null
   float *lse;
   const uint32_t *mask_bits;         // [rows][ceil(N/128)*4] key bits, 0 beyond N
   int64_t mask_bits_stride;          // words per attention row (0: shared by all rows)
@@ -86,9 +87,11 @@ cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part
                                        int nb, float scale, __nv_bfloat16 *dq, __nv_bfloat16 *dk,
                                        __nv_bfloat16 *dv, cudaStream_t stream);
 // du (compact variant frame, bf16) = dout * sigmoid(g); D = sum_c dout * out;
-// dgate (storage layout) = dout * out * (1 - sigmoid(g)).
+// dgate (storage layout) = dout * out * (1 - sigmoid(g)); out + out_res in
+// place of out when out_res (the forward's rounding residual) is given.
 cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
-                                const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
+                                const __nv_bfloat16 *out, const __nv_bfloat16 *out_res,
+                                const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
                                 cudaStream_t stream);
 

@@ -439,20 +439,26 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int64_t off = (int64_t)r * a.sR + (int64_t)x * a.sX + (int64_t)h * kC;
       const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + off);
       uint4 *op = reinterpret_cast<uint4 *>(a.out + off);
+      uint4 *rp = a.out_res ? reinterpret_cast<uint4 *>(a.out_res + off) : nullptr;
 #pragma unroll
       for (int v4 = 0; v4 < 4; ++v4) {
         const uint4 gv = gp[v4];
         const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        uint32_t ow[4];
+        uint32_t ow[4], rw[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int cc = v4 * 8 + e * 2;
           const float g0 = bf16lo(gw[e]), g1 = bf16hi(gw[e]);
           const float s0 = rcp_approx(1.0f + ex2_approx(-g0 * kLog2e));
           const float s1 = rcp_approx(1.0f + ex2_approx(-g1 * kLog2e));
-          ow[e] = pack_bf16(s0 * __uint_as_float(o[cc]) * inv, s1 * __uint_as_float(o[cc + 1]) * inv);
+          const float y0 = s0 * __uint_as_float(o[cc]) * inv;
+          const float y1 = s1 * __uint_as_float(o[cc + 1]) * inv;
+          ow[e] = pack_bf16(y0, y1);
+          // what the bf16 output lost, itself kept to bf16 precision
+          rw[e] = pack_bf16(y0 - bf16lo(ow[e]), y1 - bf16hi(ow[e]));
         }
         op[v4] = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        if (rp) rp[v4] = make_uint4(rw[0], rw[1], rw[2], rw[3]);
       }
       *lse_p = l > 0.0f ? (m_r[0] + lg2_approx(l)) * kLn2 : -INFINITY;
     }

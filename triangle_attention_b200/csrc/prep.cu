@@ -66,6 +66,7 @@ __device__ __forceinline__ float sigmoid_fast(float g) {
 // four threads of one (a, b, h) sum their parts of D with two shuffles.
 __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ gate,
                                     const __nv_bfloat16 *__restrict__ out,
+                                    const __nv_bfloat16 *__restrict__ out_res,
                                     const __nv_bfloat16 *__restrict__ dout,
                                     __nv_bfloat16 *__restrict__ du, float *__restrict__ D,
                                     __nv_bfloat16 *__restrict__ dgate, int ending) {
@@ -85,16 +86,20 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
     const uint4 g4 = *reinterpret_cast<const uint4 *>(gate + so);
     const uint4 o4 = *reinterpret_cast<const uint4 *>(out + so);
     const uint4 d4 = *reinterpret_cast<const uint4 *>(dout + so);
+    const uint4 r4 = out_res ? *reinterpret_cast<const uint4 *>(out_res + so)
+                             : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
     const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w};
     const uint32_t dw[4] = {d4.x, d4.y, d4.z, d4.w};
+    const uint32_t rs[4] = {r4.x, r4.y, r4.z, r4.w};
     uint32_t uw[4], rw[4];
     float d = 0.0f;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float s0 = sigmoid_fast(bf16lo(gw[k])), s1 = sigmoid_fast(bf16hi(gw[k]));
       const float d0 = bf16lo(dw[k]), d1 = bf16hi(dw[k]);
-      const float o0 = bf16lo(ow[k]), o1 = bf16hi(ow[k]);
+      // the forward's fp32 output, as far as out and its residual carry it
+      const float o0 = bf16lo(ow[k]) + bf16lo(rs[k]), o1 = bf16hi(ow[k]) + bf16hi(rs[k]);
       d = fmaf(d0, o0, d);
       d = fmaf(d1, o1, d);
       uw[k] = pack_bf16(d0 * s0, d1 * s1);
@@ -190,14 +195,15 @@ cudaError_t launch_bias_transpose(const __nv_bfloat16 *bias, __nv_bfloat16 *bias
 }
 
 cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
-                                const __nv_bfloat16 *out, const __nv_bfloat16 *dout,
+                                const __nv_bfloat16 *out, const __nv_bfloat16 *out_res,
+                                const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
                                 cudaStream_t stream) {
   const int64_t total = (int64_t)f.N * f.N * f.H * 4;
   if (total == 0) return cudaSuccess;
   const int ending = f.variant == 1 ? 1 : 0;
-  bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, dout, du, D,
-                                                                  dgate, ending);
+  bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, out_res, dout,
+                                                                  du, D, dgate, ending);
   return cudaGetLastError();
 }
 
