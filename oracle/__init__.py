@@ -178,6 +178,68 @@ def dbias_entries(q, k, v, bias, gate, dout, entries, mask=None, variant: int = 
     return out
 
 
+# ------------------------------------------------ triangle multiplication --
+
+OUTGOING = 0
+INCOMING = 1
+_MUL_SRC = os.path.join(_HERE, "tri_mul_oracle.c")
+_MUL_LIB = os.path.join(_HERE, "libtri_mul_oracle.so")
+_mul_lib = None
+
+
+def load_mul_library(path: str):
+    """Open a triangle-multiplication oracle library and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lib.tri_mul_oracle_fwd.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P]
+    lib.tri_mul_oracle_bwd.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                       P]
+    lib.tri_mul_oracle_fwd.restype = ctypes.c_int
+    lib.tri_mul_oracle_bwd.restype = ctypes.c_int
+    return lib
+
+
+def build_mul(force: bool = False) -> str:
+    return build(force, _MUL_SRC, _MUL_LIB)
+
+
+def _load_mul():
+    global _mul_lib
+    if _mul_lib is None:
+        _mul_lib = load_mul_library(build_mul())
+    return _mul_lib
+
+
+def _mul_dims(a) -> tuple:
+    C, N, N2 = a.shape
+    assert N == N2
+    return N, C
+
+
+def mul_fwd(a, b, direction: int = OUTGOING, lib=None) -> np.ndarray:
+    """t[c, i, j] of the triangle multiplicative update, channel-major."""
+    a, b = map(_f32, (a, b))
+    N, C = _mul_dims(a)
+    t = np.zeros((C, N, N), dtype=np.float64)
+    rc = (lib or _load_mul()).tri_mul_oracle_fwd(N, C, direction, _ptr(a), _ptr(b), _ptr(t))
+    if rc != 0:
+        raise RuntimeError(f"tri_mul_oracle_fwd failed with {rc}")
+    return t
+
+
+def mul_bwd(a, b, dt, direction: int = OUTGOING, lib=None) -> tuple:
+    """(da, db) of L = sum(dt * t), channel-major."""
+    a, b, dt = map(_f32, (a, b, dt))
+    N, C = _mul_dims(a)
+    da = np.zeros((C, N, N), dtype=np.float64)
+    db = np.zeros((C, N, N), dtype=np.float64)
+    rc = (lib or _load_mul()).tri_mul_oracle_bwd(N, C, direction, _ptr(a), _ptr(b), _ptr(dt),
+                                                 _ptr(da), _ptr(db))
+    if rc != 0:
+        raise RuntimeError(f"tri_mul_oracle_bwd failed with {rc}")
+    return da, db
+
+
 def to_storage(x_rows: np.ndarray, variant: int) -> np.ndarray:
     """Map a full-row result [N(row), N(query), H, C] from the variant frame to
     the storage layout of the pair tensors (a transpose for the ending node)."""
