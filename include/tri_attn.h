@@ -250,6 +250,46 @@ tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_stat
 tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
                                             tri_attn_stream_t stream);
 
+/* ------------------------------------------------ triangle multiplication --
+ *
+ * The contraction at the core of the triangle multiplicative update, the other
+ * pair operation the pages' kernels accelerate ("TurboPairFormer accelera fino
+ * a 1,73x l'addestramento di OpenFold3 nei test", section "Dove si impiega il
+ * tempo"; the pages print no formula, this is the standard AlphaFold-family
+ * one). Per channel c, on channel-major bf16 stacks x[c][r][s] at
+ * (c*N + r)*N + s:
+ *   TRI_MUL_OUTGOING: t[c][i][j] = sum_k a[c][i][k] * b[c][j][k]
+ *   TRI_MUL_INCOMING: t[c][i][j] = sum_k a[c][k][i] * b[c][k][j]
+ * fp32 accumulation on the tensor cores, bf16 results. The backward of
+ * L = sum(dt * t) gives da and db in the layout of a and b:
+ *   outgoing: da[c][i][k] = sum_j dt[c][i][j] b[c][j][k],
+ *             db[c][j][k] = sum_i dt[c][i][j] a[c][i][k]
+ *   incoming: da[c][k][i] = sum_j dt[c][i][j] b[c][k][j],
+ *             db[c][k][j] = sum_i dt[c][i][j] a[c][k][i]
+ * Pointers: device, caller-owned, 16-byte aligned, contiguous [C][N][N] bf16.
+ * N must be a multiple of 8 (TRI_ATTN_ERR_UNSUPPORTED otherwise); N = 0
+ * returns TRI_ATTN_OK after the argument checks and enqueues nothing. The workspace (device, 16-byte aligned, tri_mul_workspace_size bytes)
+ * holds the status word that tri_attn_read_status() reads. Calls are
+ * asynchronous on the stream, allocate nothing and are deterministic (each
+ * output element is one fixed-order tensor-core accumulation).
+ */
+typedef enum { TRI_MUL_OUTGOING = 0, TRI_MUL_INCOMING = 1 } tri_mul_direction;
+
+typedef struct {
+    int64_t N;          /* residues */
+    int32_t C;          /* channels (independent N x N products) */
+    int32_t direction;  /* tri_mul_direction */
+} tri_mul_problem;
+
+tri_attn_status tri_mul_workspace_size(const tri_mul_problem *prob, size_t *bytes);
+
+tri_attn_status tri_mul_fwd(const tri_mul_problem *prob, const void *a, const void *b, void *t,
+                            void *workspace, size_t workspace_bytes, tri_attn_stream_t stream);
+
+tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const void *b,
+                            const void *dt, void *da, void *db, void *workspace,
+                            size_t workspace_bytes, tri_attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -70,6 +70,13 @@ def _with_residual(opts, residual):
     return opts
 
 
+OUTGOING, INCOMING = 0, 1
+
+
+class MulProblem(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("C", ctypes.c_int32), ("direction", ctypes.c_int32)]
+
+
 class Problem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int32), ("c", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("variant", ctypes.c_int32),
@@ -101,10 +108,15 @@ def lib():
                                                ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.tri_attn_check_wait_timeout.argtypes = [P, sz, P]
+        MP = ctypes.POINTER(MulProblem)
+        L.tri_mul_workspace_size.argtypes = [MP, ctypes.POINTER(sz)]
+        L.tri_mul_fwd.argtypes = [MP, P, P, P, P, sz, P]
+        L.tri_mul_bwd.argtypes = [MP, P, P, P, P, P, P, sz, P]
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
                   L.tri_attn_kernel_launches, L.tri_attn_read_status,
-                  L.tri_attn_check_wait_timeout):
+                  L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
+                  L.tri_mul_bwd):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -240,6 +252,39 @@ def check_wait_timeout(ws: torch.Tensor, stream=None) -> int:
     _check(lib().tri_attn_check_wait_timeout(_p(ws), ws.numel(), _stream(stream)),
            "tri_attn_check_wait_timeout")
     return read_status(ws, stream)
+
+
+def _mul_problem(a: torch.Tensor, direction: int) -> MulProblem:
+    C, N, N2 = a.shape
+    if N != N2 or a.dtype != torch.bfloat16:
+        raise ValueError("triangle multiplication takes bf16 [C, N, N] stacks")
+    return MulProblem(N, C, direction)
+
+
+def mul_fwd(a, b, direction: int = OUTGOING, t=None, ws=None, stream=None) -> torch.Tensor:
+    """Triangle multiplicative update contraction, channel-major bf16 [C, N, N]:
+    outgoing t[c,i,j] = sum_k a[c,i,k] b[c,j,k]; incoming sum_k a[c,k,i] b[c,k,j]."""
+    _contig(a, b, t)
+    prob = _mul_problem(a, direction)
+    if t is None:
+        t = torch.empty_like(a)
+    if ws is None:
+        ws = workspace(256, a.device)
+    _check(lib().tri_mul_fwd(ctypes.byref(prob), _p(a), _p(b), _p(t), _p(ws), ws.numel(),
+                             _stream(stream)), "tri_mul_fwd")
+    return t
+
+
+def mul_bwd(a, b, dt, direction: int = OUTGOING, grads=None, ws=None, stream=None) -> tuple:
+    """(da, db) of L = sum(dt * t) for mul_fwd(a, b, direction)."""
+    _contig(a, b, dt)
+    prob = _mul_problem(a, direction)
+    da, db = grads if grads is not None else (torch.empty_like(a), torch.empty_like(b))
+    if ws is None:
+        ws = workspace(256, a.device)
+    _check(lib().tri_mul_bwd(ctypes.byref(prob), _p(a), _p(b), _p(dt), _p(da), _p(db), _p(ws),
+                             ws.numel(), _stream(stream)), "tri_mul_bwd")
+    return da, db
 
 
 class TriangleAttention(torch.autograd.Function):

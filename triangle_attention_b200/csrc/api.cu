@@ -12,6 +12,7 @@
 #include "../../include/tri_attn.h"
 #include "bf16.cuh"
 #include "common.cuh"
+#include "trimul.cuh"
 
 namespace {
 
@@ -195,6 +196,47 @@ bool encode_bias(CUtensorMap *m, const void *base, int64_t N, int64_t H) {
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+
+tri_attn_status cuda_status(cudaError_t e);
+
+// One operand of a triangle-multiplication product: a channel-major bf16
+// stack [C][N][N]. K-major operands are read as 64 (k) x 128 boxes of the
+// stored rows, MN-major ones as 64 (m or n) x 64 (k) boxes.
+bool encode_mul_operand(CUtensorMap *m, const void *base, int64_t N, int64_t C, bool mn) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)C};
+  cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(N * N * 2)};
+  cuuint32_t box[3] = {64, mn ? 64u : 128u, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+tri_attn_status check_mul(const tri_mul_problem *p) {
+  if (!p) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->N < 0 || p->N > kMaxN || p->C < 1 || p->C > 65535) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->direction != TRI_MUL_OUTGOING && p->direction != TRI_MUL_INCOMING)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->N % 8 != 0) return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
+// One product D = X Y^T of the contraction (see trimul.cu) into `out`.
+tri_attn_status mul_product(const tri_mul_problem *p, const void *x, bool x_mn, const void *y,
+                            bool y_mn, void *out, int32_t *status, cudaStream_t stream) {
+  CUtensorMap mx, my;
+  if (!encode_mul_operand(&mx, x, p->N, p->C, x_mn) || !encode_mul_operand(&my, y, p->N, p->C, y_mn))
+    return TRI_ATTN_ERR_CUDA;
+  tri::MulArgs args;
+  args.N = (int)p->N;
+  args.C = p->C;
+  args.out = static_cast<__nv_bfloat16 *>(out);
+  args.status = status;
+  return cuda_status(tri::launch_trimul_gemm(x_mn, y_mn, mx, my, args, stream));
 }
 
 tri_attn_status cuda_status(cudaError_t e) {
@@ -512,6 +554,58 @@ tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_by
     return TRI_ATTN_ERR_WORKSPACE;
   return cuda_status(tri::launch_unsatisfied_wait(static_cast<int32_t *>(workspace),
                                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+tri_attn_status tri_mul_workspace_size(const tri_mul_problem *prob, size_t *bytes) {
+  tri_attn_status st = check_mul(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!bytes) return TRI_ATTN_ERR_INVALID_ARG;
+  *bytes = 256;
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status tri_mul_fwd(const tri_mul_problem *prob, const void *a, const void *b, void *t,
+                            void *workspace, size_t workspace_bytes, tri_attn_stream_t stream_) {
+  tri_attn_status st = check_mul(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < 256) return TRI_ATTN_ERR_WORKSPACE;
+  TRI_CHECK_PTR(a);
+  TRI_CHECK_PTR(b);
+  TRI_CHECK_PTR(t);
+  if (prob->N == 0) return TRI_ATTN_OK;      // nothing to do, nothing enqueued
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int32_t *status = static_cast<int32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), stream) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  // outgoing: t = A B^T (both K-major); incoming: t = A^T B (both MN-major)
+  const bool mn = prob->direction == TRI_MUL_INCOMING;
+  return mul_product(prob, a, mn, b, mn, t, status, stream);
+}
+
+tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const void *b,
+                            const void *dt, void *da, void *db, void *workspace,
+                            size_t workspace_bytes, tri_attn_stream_t stream_) {
+  tri_attn_status st = check_mul(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < 256) return TRI_ATTN_ERR_WORKSPACE;
+  TRI_CHECK_PTR(a);
+  TRI_CHECK_PTR(b);
+  TRI_CHECK_PTR(dt);
+  TRI_CHECK_PTR(da);
+  TRI_CHECK_PTR(db);
+  if (prob->N == 0) return TRI_ATTN_OK;      // nothing to do, nothing enqueued
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int32_t *status = static_cast<int32_t *>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(int32_t), stream) != cudaSuccess) return TRI_ATTN_ERR_CUDA;
+  if (prob->direction == TRI_MUL_OUTGOING) {
+    // da[i][k] = sum_j dt[i][j] b[j][k];  db[j][k] = sum_i dt[i][j] a[i][k]
+    st = mul_product(prob, dt, false, b, true, da, status, stream);
+    if (st == TRI_ATTN_OK) st = mul_product(prob, dt, true, a, true, db, status, stream);
+  } else {
+    // da[k][i] = sum_j b[k][j] dt[i][j];  db[k][j] = sum_i a[k][i] dt[i][j]
+    st = mul_product(prob, b, false, dt, false, da, status, stream);
+    if (st == TRI_ATTN_OK) st = mul_product(prob, a, false, dt, true, db, status, stream);
+  }
+  return st;
 }
 
 }  // extern "C"

@@ -1,0 +1,240 @@
+// Triangle multiplicative update on sm_100a: the contraction at its core,
+//   outgoing edges: t[c][i][j] = sum_k a[c][i][k] b[c][j][k]
+//   incoming edges: t[c][i][j] = sum_k a[c][k][i] b[c][k][j]
+// and its backward, for channel-major bf16 stacks x[c][r][s] (one N x N matrix
+// per channel). The pages name triangle multiplication beside triangle
+// attention as the other pair operation their kernels accelerate
+// ("TurboPairFormer accelera fino a 1,73x l'addestramento di OpenFold3 nei
+// test", section "Dove si impiega il tempo"); the contraction is the standard
+// AlphaFold-family one.
+//
+// Per channel each of the six products (forward and the two gradients, two
+// directions) is one GEMM D[m][n] = sum_k X[m][k] Y[n][k] in which each operand
+// is read straight from its stored matrix, either K-major (the stored rows are
+// m or n, k contiguous) or MN-major (the stored rows are k, m or n contiguous):
+// tcgen05 takes both, so no operand is ever transposed in memory.
+//
+// One CTA computes one 128x128 tile of one channel (fp32 in tensor memory):
+//   warp 0      TMA producer: 64-wide K slices of X and Y, 3-stage ring
+//   warp 1      tensor-memory allocator and MMA issuer
+//   warps 2..5  epilogue: tensor memory -> bf16 -> the output rows
+// 96 KB of shared memory and 128 tensor-memory columns, so two CTAs share an
+// SM and one's epilogue overlaps the other's main loop.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "trimul.cuh"
+
+namespace tri {
+namespace {
+
+constexpr int kTM = 128, kTN = 128, kTK = 64;
+constexpr int kStages = 3;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kOpBytes = kTM * kTK * 2;          // 16 KB per operand slice
+constexpr uint32_t kStageBytes = 2 * kOpBytes;
+constexpr uint32_t kOffCtl = kStages * kStageBytes;
+
+struct __align__(8) MulSmem {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full;
+  uint64_t teardown;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+constexpr uint32_t kSmemBytes = kOffCtl + sizeof(MulSmem) + 1024;   // +1024 for alignment
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
+                                         volatile uint32_t *abort_flag, int32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t polls = 1; polls < kWaitMaxPolls; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+    }
+  }
+  *abort_flag = 1u;
+  report_status(status, kStatusTimeout);
+  return false;
+}
+
+// A 128 x 64 operand slice into shared memory. K-major: one 64 (k) x 128 box of
+// the stored matrix (rows m, k contiguous). MN-major: two 64 (m) x 64 (k)
+// boxes of the stored matrix (rows k, m contiguous), one per half of m.
+template <bool MN>
+__device__ __forceinline__ void load_slice(uint8_t *dst, const CUtensorMap *map, uint64_t *bar,
+                                           int mn0, int k0, int c) {
+  if (MN) {
+    tma_load_3d(dst, map, bar, mn0, k0, c);
+    tma_load_3d(dst + kOpBytes / 2, map, bar, mn0 + 64, k0, c);
+  } else {
+    tma_load_3d(dst, map, bar, k0, mn0, c);
+  }
+}
+
+// Descriptor of the 16-wide K step ks of a slice (128-byte swizzle). K-major:
+// rows of 128 bytes, 8-row groups 1 KB apart, the K step 32 bytes along a row.
+// MN-major: two 64-wide MN halves 8 KB apart, 8 k-rows per 1 KB group, the K
+// step 16 rows (2 KB).
+template <bool MN>
+__device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
+  return MN ? make_sdesc(base + ks * 2048, kOpBytes / 2, 1024, kSwizzle128B)
+            : make_sdesc(base + ks * 32, 16, 1024, kSwizzle128B);
+}
+
+template <bool XMN, bool YMN>
+__global__ void __launch_bounds__(kThreads, 2)
+trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_y, const MulArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  MulSmem &ctl = *reinterpret_cast<MulSmem *>(smem + kOffCtl);
+  volatile uint32_t *abort_flag = &ctl.abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.N;
+  const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * kTN, c = blockIdx.z;
+  const int nk = (N + kTK - 1) / kTK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl.full[s], 1);
+      mbar_init(&ctl.empty[s], 1);
+    }
+    mbar_init(&ctl.acc_full, 1);
+    mbar_init(&ctl.teardown, 1);
+    ctl.abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&ctl.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_y);
+      int armed[kStages];
+      for (int s = 0; s < kStages; ++s) armed[s] = -1;
+      bool ok = true;
+      for (int kt = 0; kt < nk; ++kt) {
+        const int st = kt % kStages;
+        if (kt >= kStages &&
+            !wait_bar(&ctl.empty[st], ((kt / kStages) - 1) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        uint8_t *dst = smem + st * kStageBytes;
+        mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
+        load_slice<XMN>(dst, &tm_x, &ctl.full[st], m0, kt * kTK, c);
+        load_slice<YMN>(dst + kOpBytes, &tm_y, &ctl.full[st], n0, kt * kTK, c);
+        armed[st] = kt / kStages;
+      }
+      if (!ok)
+        for (int s = 0; s < kStages; ++s)
+          if (armed[s] >= 0) mbar_wait(&ctl.full[s], armed[s] & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer --
+    if (elect_one()) {
+      const uint32_t idesc = make_idesc_bf16(kTM, kTN, XMN, YMN);
+      bool ok = true;
+      for (int kt = 0; kt < nk && ok; ++kt) {
+        const int st = kt % kStages;
+        if (!wait_bar(&ctl.full[st], (kt / kStages) & 1, abort_flag, a.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + st * kStageBytes);
+        const uint32_t ya = xa + kOpBytes;
+#pragma unroll
+        for (int ks = 0; ks < kTK / 16; ++ks)
+          mma_ss(tmem, slice_desc<XMN>(xa, ks), slice_desc<YMN>(ya, ks), idesc,
+                 (kt > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&ctl.empty[st]);
+      }
+      mma_commit(&ctl.acc_full);
+      // No tensor-memory operation may be in flight when the CTA tears down.
+      mma_commit(&ctl.teardown);
+      mbar_wait(&ctl.teardown, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue --
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;           // output row of the tile = TMEM lane
+    const int m = m0 + row;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    bool ok = true;
+    if (!mbar_try_wait(&ctl.acc_full, 0)) ok = wait_bar(&ctl.acc_full, 0, abort_flag, a.status);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16 *orow = a.out + ((int64_t)c * N + m) * N + n0;
+#pragma unroll 1
+      for (int cb = 0; cb < kTN / 32; ++cb) {
+        uint32_t v[32];
+        tmem_ld32(tl + cb * 32, v);
+        if (m < N) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int n = n0 + cb * 32 + q * 8;
+            if (n < N) {
+              const uint4 w = make_uint4(
+                  pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                  pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                  pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                  pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+              *reinterpret_cast<uint4 *>(orow + cb * 32 + q * 8) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <bool XMN, bool YMN>
+cudaError_t launch(const CUtensorMap &x, const CUtensorMap &y, const MulArgs &args,
+                   cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(trimul_gemm_kernel<XMN, YMN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((args.N + kTM - 1) / kTM, (args.N + kTN - 1) / kTN, args.C);
+  trimul_gemm_kernel<XMN, YMN><<<grid, kThreads, kSmemBytes, stream>>>(x, y, args);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_trimul_gemm(bool x_mn, bool y_mn, const CUtensorMap &x, const CUtensorMap &y,
+                               const MulArgs &args, cudaStream_t stream) {
+  if (args.N == 0 || args.C == 0) return cudaSuccess;
+  if (!x_mn && !y_mn) return launch<false, false>(x, y, args, stream);
+  if (!x_mn && y_mn) return launch<false, true>(x, y, args, stream);
+  if (x_mn && y_mn) return launch<true, true>(x, y, args, stream);
+  return cudaErrorInvalidValue;       // X MN-major with Y K-major: no product needs it
+}
+
+}  // namespace tri
