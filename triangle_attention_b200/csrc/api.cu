@@ -203,17 +203,24 @@ tri_attn_status cuda_status(cudaError_t e);
 // One operand of a triangle-multiplication product: a channel-major bf16
 // stack [C][N][N]. K-major operands are read as 64 (k) x 128 boxes of the
 // stored rows, MN-major ones as 64 (m or n) x 64 (k) boxes.
-bool encode_mul_operand(CUtensorMap *m, const void *base, int64_t N, int64_t C, bool mn) {
+bool encode_mul_stack(CUtensorMap *m, const void *base, int64_t N, int64_t C, uint32_t rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)C};
   cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(N * N * 2)};
-  cuuint32_t box[3] = {64, mn ? 64u : 128u, 1};
+  cuuint32_t box[3] = {64, rows, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
+}
+bool encode_mul_operand(CUtensorMap *m, const void *base, int64_t N, int64_t C, bool mn) {
+  return encode_mul_stack(m, base, N, C, mn ? 64u : 128u);
+}
+// The product's output: the epilogue stores 64-column boxes of 32 rows.
+bool encode_mul_output(CUtensorMap *m, void *base, int64_t N, int64_t C) {
+  return encode_mul_stack(m, base, N, C, 32u);
 }
 
 tri_attn_status check_mul(const tri_mul_problem *p) {
@@ -228,15 +235,16 @@ tri_attn_status check_mul(const tri_mul_problem *p) {
 // One product D = X Y^T of the contraction (see trimul.cu) into `out`.
 tri_attn_status mul_product(const tri_mul_problem *p, const void *x, bool x_mn, const void *y,
                             bool y_mn, void *out, int32_t *status, cudaStream_t stream) {
-  CUtensorMap mx, my;
-  if (!encode_mul_operand(&mx, x, p->N, p->C, x_mn) || !encode_mul_operand(&my, y, p->N, p->C, y_mn))
+  CUtensorMap mx, my, md;
+  if (!encode_mul_operand(&mx, x, p->N, p->C, x_mn) ||
+      !encode_mul_operand(&my, y, p->N, p->C, y_mn) || !encode_mul_output(&md, out, p->N, p->C))
     return TRI_ATTN_ERR_CUDA;
   tri::MulArgs args;
   args.N = (int)p->N;
   args.C = p->C;
   args.out = static_cast<__nv_bfloat16 *>(out);
   args.status = status;
-  return cuda_status(tri::launch_trimul_gemm(x_mn, y_mn, mx, my, args, stream));
+  return cuda_status(tri::launch_trimul_gemm(x_mn, y_mn, mx, my, md, args, stream));
 }
 
 tri_attn_status cuda_status(cudaError_t e) {

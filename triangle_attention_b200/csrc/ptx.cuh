@@ -113,6 +113,23 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const void *map, uint64_t
       : "memory");
 }
 
+// Shared -> global store of a 3-D tensor-map tile (bulk group completion).
+// Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const void *map, const void *src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Prefetch of a 4-D tensor-map tile into L2 (no shared memory, no barrier).
 __device__ __forceinline__ void tma_prefetch_l2_4d(const void *map, int c0, int c1, int c2,
                                                    int c3) {

@@ -14,11 +14,12 @@
 // m or n, k contiguous) or MN-major (the stored rows are k, m or n contiguous):
 // tcgen05 takes both, so no operand is ever transposed in memory.
 //
-// One CTA computes one 128x128 tile of one channel (fp32 in tensor memory):
-//   warp 0      TMA producer: 64-wide K slices of X and Y, 3-stage ring
-//   warp 1      tensor-memory allocator and MMA issuer
-//   warps 2..5  epilogue: tensor memory -> bf16 -> the output rows
-// 96 KB of shared memory and 128 tensor-memory columns, so two CTAs share an
+// One CTA computes one 128x256 tile of one channel (fp32 in tensor memory):
+//   warp 0      TMA producer: 64-wide K slices of X and Y (48 KB), 2-stage ring
+//   warp 1      tensor-memory allocator and MMA issuer (N = 256 products)
+//   warps 2..5  epilogue: tensor memory -> bf16 -> the idle stage buffers ->
+//               TMA stores of 64-column boxes
+// 96 KB of shared memory and 256 tensor-memory columns, so two CTAs share an
 // SM and one's epilogue overlaps the other's main loop.
 #include <cstdint>
 #include <cuda.h>
@@ -31,13 +32,17 @@
 namespace tri {
 namespace {
 
-constexpr int kTM = 128, kTN = 128, kTK = 64;
-constexpr int kStages = 3;
+constexpr int kTM = 128, kTK = 64;
+constexpr int kTN = 256;                               // output tile 128 x kTN
+constexpr int kStages = 2;
+constexpr int kMinBlocks = 2;                          // CTAs per SM the budget is sized for
 constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = 128;
-constexpr uint32_t kOpBytes = kTM * kTK * 2;          // 16 KB per operand slice
-constexpr uint32_t kStageBytes = 2 * kOpBytes;
+constexpr uint32_t kTmemCols = kTN;
+constexpr uint32_t kXBytes = kTM * kTK * 2;            // 16 KB X slice
+constexpr uint32_t kYBytes = kTN * kTK * 2;            // Y slice
+constexpr uint32_t kStageBytes = kXBytes + kYBytes;
 constexpr uint32_t kOffCtl = kStages * kStageBytes;
+constexpr uint32_t kAtomBytes = 64 * kTK * 2;          // one 64-wide MN atom column: 8 KB
 
 struct __align__(8) MulSmem {
   uint64_t full[kStages];
@@ -65,34 +70,38 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
   return false;
 }
 
-// A 128 x 64 operand slice into shared memory. K-major: one 64 (k) x 128 box of
-// the stored matrix (rows m, k contiguous). MN-major: two 64 (m) x 64 (k)
-// boxes of the stored matrix (rows k, m contiguous), one per half of m.
-template <bool MN>
+// A ROWS x 64 operand slice into shared memory. K-major: ROWS/128 boxes of
+// 64 (k) x 128 rows of the stored matrix (rows m or n, k contiguous), stacked.
+// MN-major: ROWS/64 boxes of 64 (m or n) x 64 (k) of the stored matrix (rows k,
+// m or n contiguous), one 8 KB atom column each.
+template <bool MN, int ROWS>
 __device__ __forceinline__ void load_slice(uint8_t *dst, const CUtensorMap *map, uint64_t *bar,
                                            int mn0, int k0, int c) {
   if (MN) {
-    tma_load_3d(dst, map, bar, mn0, k0, c);
-    tma_load_3d(dst + kOpBytes / 2, map, bar, mn0 + 64, k0, c);
+#pragma unroll
+    for (int h = 0; h < ROWS / 64; ++h) tma_load_3d(dst + h * kAtomBytes, map, bar, mn0 + 64 * h, k0, c);
   } else {
-    tma_load_3d(dst, map, bar, k0, mn0, c);
+#pragma unroll
+    for (int h = 0; h < ROWS / 128; ++h)
+      tma_load_3d(dst + h * (128 * kTK * 2), map, bar, k0, mn0 + 128 * h, c);
   }
 }
 
 // Descriptor of the 16-wide K step ks of a slice (128-byte swizzle). K-major:
 // rows of 128 bytes, 8-row groups 1 KB apart, the K step 32 bytes along a row.
-// MN-major: two 64-wide MN halves 8 KB apart, 8 k-rows per 1 KB group, the K
+// MN-major: 64-wide MN atom columns 8 KB apart, 8 k-rows per 1 KB group, the K
 // step 16 rows (2 KB).
 template <bool MN>
 __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
-  return MN ? make_sdesc(base + ks * 2048, kOpBytes / 2, 1024, kSwizzle128B)
+  return MN ? make_sdesc(base + ks * 2048, kAtomBytes, 1024, kSwizzle128B)
             : make_sdesc(base + ks * 32, 16, 1024, kSwizzle128B);
 }
 
 template <bool XMN, bool YMN>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
 trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_y, const MulArgs a) {
+                   const __grid_constant__ CUtensorMap tm_y,
+                   const __grid_constant__ CUtensorMap tm_d, const MulArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -139,8 +148,8 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         }
         uint8_t *dst = smem + st * kStageBytes;
         mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
-        load_slice<XMN>(dst, &tm_x, &ctl.full[st], m0, kt * kTK, c);
-        load_slice<YMN>(dst + kOpBytes, &tm_y, &ctl.full[st], n0, kt * kTK, c);
+        load_slice<XMN, kTM>(dst, &tm_x, &ctl.full[st], m0, kt * kTK, c);
+        load_slice<YMN, kTN>(dst + kXBytes, &tm_y, &ctl.full[st], n0, kt * kTK, c);
         armed[st] = kt / kStages;
       }
       if (!ok)
@@ -160,7 +169,7 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         }
         tc_fence_after();
         const uint32_t xa = smem_u32(smem + st * kStageBytes);
-        const uint32_t ya = xa + kOpBytes;
+        const uint32_t ya = xa + kXBytes;
 #pragma unroll
         for (int ks = 0; ks < kTK / 16; ++ks)
           mma_ss(tmem, slice_desc<XMN>(xa, ks), slice_desc<YMN>(ya, ks), idesc,
@@ -175,34 +184,41 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
   } else {
     // ------------------------------------------------------------ epilogue --
     const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;           // output row of the tile = TMEM lane
-    const int m = m0 + row;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     bool ok = true;
     if (!mbar_try_wait(&ctl.acc_full, 0)) ok = wait_bar(&ctl.acc_full, 0, abort_flag, a.status);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16 *orow = a.out + ((int64_t)c * N + m) * N + n0;
+      // The operand stages are idle once the accumulator is complete: each warp
+      // stages its 32 rows there (64-column boxes of 32 rows x 128 bytes, 128-byte
+      // swizzle) and stores them with TMA, which clips rows and columns past N.
+      uint8_t *stage = smem + q4 * (32 * kTN * 2);
 #pragma unroll 1
       for (int cb = 0; cb < kTN / 32; ++cb) {
         uint32_t v[32];
         tmem_ld32(tl + cb * 32, v);
-        if (m < N) {
+        uint8_t *box = stage + (cb >> 1) * (32 * 128);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int n = n0 + cb * 32 + q * 8;
-            if (n < N) {
-              const uint4 w = make_uint4(
-                  pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                  pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                  pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                  pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-              *reinterpret_cast<uint4 *>(orow + cb * 32 + q * 8) = w;
-            }
+        for (int q = 0; q < 4; ++q) {
+          const int chunk = (cb & 1) * 4 + q;         // 16-byte chunk of the 128-byte row
+          *reinterpret_cast<uint4 *>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+              make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                         pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                         pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                         pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+        }
+        if (cb & 1) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tm_d, box, n0 + (cb >> 1) * 64, m0 + q4 * 32, c);
+            bulk_commit_group();
           }
         }
       }
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
     }
   }
 
@@ -216,24 +232,24 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
 }
 
 template <bool XMN, bool YMN>
-cudaError_t launch(const CUtensorMap &x, const CUtensorMap &y, const MulArgs &args,
-                   cudaStream_t stream) {
+cudaError_t launch(const CUtensorMap &x, const CUtensorMap &y, const CUtensorMap &d,
+                   const MulArgs &args, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(trimul_gemm_kernel<XMN, YMN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((args.N + kTM - 1) / kTM, (args.N + kTN - 1) / kTN, args.C);
-  trimul_gemm_kernel<XMN, YMN><<<grid, kThreads, kSmemBytes, stream>>>(x, y, args);
+  trimul_gemm_kernel<XMN, YMN><<<grid, kThreads, kSmemBytes, stream>>>(x, y, d, args);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_trimul_gemm(bool x_mn, bool y_mn, const CUtensorMap &x, const CUtensorMap &y,
-                               const MulArgs &args, cudaStream_t stream) {
+                               const CUtensorMap &d, const MulArgs &args, cudaStream_t stream) {
   if (args.N == 0 || args.C == 0) return cudaSuccess;
-  if (!x_mn && !y_mn) return launch<false, false>(x, y, args, stream);
-  if (!x_mn && y_mn) return launch<false, true>(x, y, args, stream);
-  if (x_mn && y_mn) return launch<true, true>(x, y, args, stream);
+  if (!x_mn && !y_mn) return launch<false, false>(x, y, d, args, stream);
+  if (!x_mn && y_mn) return launch<false, true>(x, y, d, args, stream);
+  if (x_mn && y_mn) return launch<true, true>(x, y, d, args, stream);
   return cudaErrorInvalidValue;       // X MN-major with Y K-major: no product needs it
 }
 
