@@ -41,6 +41,8 @@ WORKLOAD = "n768_bf16"
 METRIC = "triangle-attention fwd+bwd TFLOP/s at N=768 bf16 (% of B200 BF16 peak)"
 UNIT = "TFLOP/s"
 SPEC_BF16_TFLOPS = 2250.0
+SMS = 148
+EXP2_PER_CLK_PER_SM = 16     # measured ex2.approx issue rate of one SM
 
 
 def flops(N: int, H: int, c: int) -> tuple:
@@ -57,6 +59,16 @@ def load_peaks() -> dict:
                 "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def tensor_peak(peaks: dict, clk: dict) -> tuple:
+    """The bf16 matmul peak that matches how the kernel ran: the sustained figure
+    when the sampled SM clock sat below 90% of its maximum under load (the
+    power cap of a long run), else the burst figure."""
+    mhz, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if mhz and mx and peaks.get("bf16_tflops_sustained") and mhz < 0.9 * mx:
+        return peaks["bf16_tflops_sustained"], f"{peaks['source']} bf16 matmul (sustained)"
+    return peaks["bf16_tflops"], f"{peaks['source']} bf16 matmul (burst)"
 
 
 def config_dict(w) -> dict:
@@ -338,6 +350,8 @@ def run_ours(args, rank, world, local, w):
     value = whole_job_tflops(world, f_fwd + f_bwd, ms)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    fwd_med = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_med = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
 
     # roofline of the dominant kernel: algorithmic FLOPs per launch / launch time
     peaks = load_peaks()
@@ -347,10 +361,27 @@ def run_ours(args, rank, world, local, w):
         kname, kms, kflops = "fwd_bf16_kernel", fwd_ms, f_fwd
     achieved = kflops / (kms * 1e-3) / 1e12
     traffic = traffic_record(kname)
+    tpeak, tsrc = tensor_peak(peaks, clk)
     roofline = {"bound": "tensor", "kernel": kname, "achieved": achieved,
-                "peak": peaks["bf16_tflops"], "unit": UNIT,
-                "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                "peak_source": f"{peaks['source']} bf16 matmul (burst)"}
+                "peak": tpeak, "unit": UNIT, "frac": achieved / tpeak, "traffic": traffic,
+                "peak_source": tsrc}
+    # the same kernel against the other two ceilings: HBM (its measured DRAM
+    # bytes, when recorded for this source) and the exp2 unit (one exp2 per
+    # logit; 16 per clock per SM, at the SM clock sampled during the run)
+    sm_mhz = clk.get("sm_mhz") or 1965.0
+    exp_peak = EXP2_PER_CLK_PER_SM * SMS * sm_mhz * 1e6
+    exps = float(w.N) ** 3 * w.H
+    rooflines = {
+        "kernel": kname,
+        "tensor": {"achieved_tflops": achieved, "peak_tflops": tpeak, "frac": achieved / tpeak},
+        "hbm": ({"achieved_gbs": traffic / (kms * 1e-3) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                 "frac": traffic / (kms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+                if traffic else None),
+        "exp2": {"achieved_per_s": exps / (kms * 1e-3), "peak_per_s": exp_peak,
+                 "frac": exps / (kms * 1e-3) / exp_peak,
+                 "peak_source": "16 ex2 per clock per SM (microbenchmark) x 148 SMs x sampled clock"},
+        "step_exp2_frac": 2 * exps / (ms_local * 1e-3) / exp_peak,
+    }
 
     # End to end through the public API with pinned host buffers. Every step
     # uploads its inputs, runs forward + backward and downloads all its
@@ -424,8 +455,10 @@ def run_ours(args, rank, world, local, w):
             "pct_of_spec_bf16_peak": 100.0 * value / world / SPEC_BF16_TFLOPS,
             "pct_of_measured_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
             "kernels": {"fwd_bf16_kernel_ms": fwd_ms, "bwd_bf16_kernel_ms": bwd_ms,
-                        "step_ms": ms_local},
+                        "fwd_bf16_kernel_median_ms": fwd_med,
+                        "bwd_bf16_kernel_median_ms": bwd_med, "step_ms": ms_local},
             "roofline": roofline,
+            "rooflines": rooflines,
             "clocks": clk,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -437,12 +470,94 @@ def run_ours(args, rank, world, local, w):
     return line
 
 
+# ---------------------------------------------- triangle multiplication --
+
+TRIMUL_METRIC = "triangle-multiplication fwd+bwd TFLOP/s at N=768, C=128 bf16 (both directions)"
+
+
+def run_trimul(args, rank, world, local):
+    """One step: forward and backward of the outgoing and the incoming
+    contraction on channel-major bf16 stacks, N=768 residues, C=128 channels."""
+    import triangle_attention_b200 as ta
+    N, C = 768, 128
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    gen = np.random.default_rng(11 + rank)
+    host = [torch.from_numpy(gen.standard_normal((C, N, N)).astype(np.float32))
+            .to(torch.bfloat16) for _ in range(3)]
+    a, b, dt = (x.to(dev) for x in host)
+    t = torch.empty_like(a)
+    da, db = torch.empty_like(a), torch.empty_like(a)
+    ws = ta.workspace(256, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for d in (ta.OUTGOING, ta.INCOMING):
+            ta.mul_fwd(a, b, d, t=t, ws=ws)
+            ta.mul_bwd(a, b, dt, d, grads=(da, db), ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
+    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if ta.read_status(ws):
+        raise RuntimeError("device status set in the timed region")
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    flops_step = 2 * 6.0 * N ** 3 * C          # per direction: fwd 2N^3C, bwd 4N^3C
+    value = whole_job_tflops(world, flops_step, ms)
+    peaks = load_peaks()
+    per_gemm_ms = ms_local / 6                 # six GEMMs of 2N^3C each per step
+    achieved = 2.0 * N ** 3 * C / (per_gemm_ms * 1e-3) / 1e12
+    line = {"metric": TRIMUL_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) channel-major stacks)",
+            "config": {"workload": "trimul_n768_c128", "N": N, "C": C,
+                       "directions": ["outgoing", "incoming"],
+                       "l2": "inputs larger than L2 (3 x 151 MB stacks)",
+                       "parallelism": "independent replica per GPU"},
+            "roofline": {"bound": "tensor", "kernel": "trimul_gemm_kernel",
+                         "achieved": achieved, "peak": tensor_peak(peaks, clk)[0], "unit": UNIT,
+                         "frac": achieved / tensor_peak(peaks, clk)[0], "traffic": None,
+                         "peak_source": tensor_peak(peaks, clk)[1]},
+            "clocks": clk,
+            "gpu_launches": 6 * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        t_start = time.perf_counter()
+        oracle.mul_fwd(host[0][:1], host[1][:1], oracle.OUTGOING)
+        oracle.mul_bwd(host[0][:1], host[1][:1], host[2][:1], oracle.OUTGOING)
+        secs = time.perf_counter() - t_start
+        line["cpu_baseline"] = {"value": 6.0 * N ** 3 / secs / 1e12, "unit": UNIT,
+                                "cores": oracle_threads(), "kind": "oracle",
+                                "sample": f"1 of {C} channels, outgoing fwd+bwd, fp64, "
+                                          f"{secs:.1f} s"}
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["attention", "trimul"], default="attention",
+                    help="attention (the default line) or the triangle multiplication")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget-s", type=float, default=150.0,
@@ -464,7 +579,8 @@ def main():
 
     rank, world, local = dist_setup()
     try:
-        line = run_ours(args, rank, world, local, w)
+        line = (run_trimul(args, rank, world, local) if args.op == "trimul"
+                else run_ours(args, rank, world, local, w))
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:
