@@ -288,19 +288,78 @@ def mul_bwd(a, b, dt, direction: int = OUTGOING, grads=None, ws=None, stream=Non
 
 
 class TriangleAttention(torch.autograd.Function):
-    """out = TriangleAttention.apply(q, k, v, bias, gate, mask, variant)."""
+    """out = TriangleAttention.apply(q, k, v, bias, gate, mask, variant).
+
+    Unbatched: q, k, v, gate [N, N, H, c], bias [H, N, N], mask None, [N] or
+    [N, N]. Batched: a leading batch dimension on every tensor (q [B, N, N, H,
+    c], bias [B, H, N, N], mask None, [B, N] or [B, N, N]); each batch element
+    is an independent problem, run in turn on the current stream."""
 
     @staticmethod
     def forward(ctx, q, k, v, bias, gate, mask=None, variant=STARTING):
-        out, lse = fwd(q, k, v, bias, gate, mask, variant)
-        ctx.save_for_backward(q, k, v, bias, gate, out, lse)
+        batched = q.dim() == 5
+        ctx.batched = batched
         ctx.mask = mask
         ctx.variant = variant
+        if not batched:
+            out, lse = fwd(q, k, v, bias, gate, mask, variant)
+        else:
+            out = torch.empty_like(q)
+            B, N, _, H, _ = q.shape
+            lse = torch.empty((B, N, H, N), dtype=torch.float32, device=q.device)
+            for i in range(B):
+                fwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i],
+                    variant, out=out[i], lse=lse[i])
+        ctx.save_for_backward(q, k, v, bias, gate, out, lse)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, bias, gate, out, lse = ctx.saved_tensors
-        dq, dk, dv, dbias, dgate = bwd(q, k, v, bias, gate, ctx.mask, out, lse,
-                                       dout.contiguous(), ctx.variant)
+        dout = dout.contiguous()
+        mask = ctx.mask
+        if not ctx.batched:
+            dq, dk, dv, dbias, dgate = bwd(q, k, v, bias, gate, mask, out, lse, dout,
+                                           ctx.variant)
+        else:
+            dq, dk, dv, dgate = (torch.empty_like(t) for t in (q, k, v, gate))
+            dbias = torch.empty_like(bias)
+            for i in range(q.shape[0]):
+                bwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i],
+                    out[i], lse[i], dout[i], ctx.variant,
+                    grads=(dq[i], dk[i], dv[i], dbias[i], dgate[i]))
         return dq, dk, dv, dbias, dgate, None, None
+
+
+def triangle_attention(q, k, v, bias, gate, mask=None, variant: int = STARTING) -> torch.Tensor:
+    """Gated triangle self-attention with pair bias (differentiable), unbatched or
+    with a leading batch dimension; see TriangleAttention."""
+    return TriangleAttention.apply(q, k, v, bias, gate, mask, variant)
+
+
+class TriangleMultiplication(torch.autograd.Function):
+    """t = TriangleMultiplication.apply(a, b, direction) on channel-major bf16
+    stacks [C, N, N] (or [B, C, N, N], each batch element in turn)."""
+
+    @staticmethod
+    def forward(ctx, a, b, direction=OUTGOING):
+        ctx.direction = direction
+        ctx.save_for_backward(a, b)
+        if a.dim() == 3:
+            return mul_fwd(a, b, direction)
+        t = torch.empty_like(a)
+        for i in range(a.shape[0]):
+            mul_fwd(a[i], b[i], direction, t=t[i])
+        return t
+
+    @staticmethod
+    def backward(ctx, dt):
+        a, b = ctx.saved_tensors
+        dt = dt.contiguous()
+        if a.dim() == 3:
+            da, db = mul_bwd(a, b, dt, ctx.direction)
+        else:
+            da, db = torch.empty_like(a), torch.empty_like(b)
+            for i in range(a.shape[0]):
+                mul_bwd(a[i], b[i], dt[i], ctx.direction, grads=(da[i], db[i]))
+        return da, db, None
