@@ -132,3 +132,12 @@ def test_bf16_wide_logit_range(variant):
     d = make_inputs(264, H=2, c=32, dtype="bf16", seed=21, bias_std=6.0, std=2.0,
                     mask="random:20")
     full_check(d, variant, "bf16", out_abs_scale=1e-2)
+
+
+@pytest.mark.parametrize("variant", [STARTING, ENDING])
+def test_bf16_n1536_backward_sampled(variant):
+    """bf16 backward at N=1536 (12 tiles per axis, 576 backward CTAs over several
+    waves, 12 tile contributions per gradient): sampled rows of every pair
+    gradient and 32 dbias entries, each summed over all 1536 rows."""
+    d = make_inputs(1536, H=4, c=32, dtype="bf16", seed=15, mask="trailing:77")
+    sampled_check(d, variant, rows=[0, 901, 1535], n_entries=32, seed=3)
