@@ -58,7 +58,7 @@ struct BwdArgs {
   const float *D;                    // [N, H, N] sum_c dout * out
   const uint32_t *mask_bits;
   int64_t mask_bits_stride;
-  // bf16 tile contributions, [tile][row][H][4][N][8] (8-channel groups):
+  // bf16 tile contributions, [tile][row][H][2][N][16] (16-channel halves):
   // part_q over key tiles yb, part_k and part_v over query tiles xb
   __nv_bfloat16 *part_q, *part_k, *part_v;
   float *part_db;                    // [ngroups][H, N, N] variant frame (ngroups > 1)
@@ -81,7 +81,7 @@ cudaError_t launch_mask_bits(const Frame &f, uint32_t *bits, int64_t rows, int64
 cudaError_t launch_bias_transpose(const __nv_bfloat16 *bias, __nv_bfloat16 *biasT, int N, int H,
                                   cudaStream_t stream);
 // dq, dk, dv (variant frame strides) = scale_q/k/v * the sum over nb tiles of
-// the bf16 contributions [tile][row][H][4][N][8], added in tile order.
+// the bf16 contributions [tile][row][H][2][N][16], added in tile order.
 cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part_q,
                                        const __nv_bfloat16 *part_k, const __nv_bfloat16 *part_v,
                                        int nb, float scale, __nv_bfloat16 *dq, __nv_bfloat16 *dk,

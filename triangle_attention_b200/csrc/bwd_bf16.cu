@@ -416,14 +416,14 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // dK (j < 4) or dV, for this warp's 32 lanes; warpgroup wg owns the pieces
     // j = wg, wg + kEltGroups, ... A piece of row r is one tile's contribution:
     // dQ of query tile xb (to be summed over key tiles), dK/dV of key tile yb (to
-    // be summed over query tiles). Contributions are stored channel-group-major,
-    // [t][r][h][c/8][i][8] (t the tile summed over, i the query or key), so each
-    // warp store writes 512 contiguous bytes.
+    // be summed over query tiles). Contributions are stored piece-major,
+    // [t][r][h][j&1][i][16] (t the tile summed over, i the query or key): a lane
+    // writes its 16 channels with one 32-byte store and a warp store covers 1 KB.
     const int64_t pair = (int64_t)N * N * H * kC;
-    // channel group g (0..3) of row r of one tensor's contributions
-    auto group_base = [&](int j, int r, int g) -> __nv_bfloat16 * {
+    // piece j's 16-channel plane of row r in one tensor's contributions
+    auto piece_base = [&](int j, int r) -> __nv_bfloat16 * {
       __nv_bfloat16 *buf = j < 2 ? a.part_q : j < 4 ? a.part_k : a.part_v;
-      return buf + ((((int64_t)r * H + h) * 4 + g) * N) * 8;
+      return buf + ((((int64_t)r * H + h) * 2 + (j & 1)) * N) * 16;
     };
 
     // Row t's pieces from TMEM buffer t & 1 to this tile's contribution slots.
@@ -438,13 +438,16 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                                              : kColDV + 16 * (j - 4);
         const int i = (j < 2 ? xb : yb) * kBM + row;
         const int tsum = j < 2 ? yb : xb;
+        uint32_t w[8];
 #pragma unroll
         for (int c8 = 0; c8 < 2; ++c8) {     // 8 columns at a time keeps registers low
           uint32_t v[8];
           tmem_ld8(tb + col + 8 * c8, v);
-          if (i < N)
-            store_bf16<8>(group_base(j, r, 2 * (j & 1) + c8) + tsum * pair + (int64_t)i * 8, v);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[4 * c8 + e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
         }
+        if (i < N) st_global_cs_v8(piece_base(j, r) + tsum * pair + (int64_t)i * 16, w);
       }
       tc_fence_before();
       mbar_arrive(&ctl.part_free[b]);

@@ -115,7 +115,7 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
 }
 
 // One thread per 8 channels of one contribution row: consecutive threads read
-// consecutive 16-byte groups of the [tile][row][H][4][N][8] contributions; the
+// consecutive 16-byte groups of the [tile][row][H][2][N][16] contributions; the
 // nb tiles are summed in tile order in fp32, scaled and rounded once.
 __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ pq,
                                            const __nv_bfloat16 *__restrict__ pk,
@@ -152,13 +152,14 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
         }
       }
     }
-    // gidx -> (r, h, channel group g, i) of the [r][H][4][N][8] layout
-    const int64_t i = gidx % f.N;
-    const int g = (int)(gidx / f.N % 4);
-    const int h = (int)(gidx / ((int64_t)f.N * 4) % f.H);
-    const int64_t r = gidx / ((int64_t)f.N * 4 * f.H);
+    // gidx -> (r, h, half, i, c8) of the [r][H][2][N][16] layout
+    const int c8 = (int)(gidx & 1);
+    const int64_t i = (gidx >> 1) % f.N;
+    const int half = (int)((gidx >> 1) / f.N % 2);
+    const int h = (int)((gidx >> 1) / ((int64_t)f.N * 2) % f.H);
+    const int64_t r = (gidx >> 1) / ((int64_t)f.N * 2 * f.H);
     __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + r * f.sR + i * f.sX +
-                         (int64_t)h * 32 + g * 8;
+                         (int64_t)h * 32 + half * 16 + c8 * 8;
     *reinterpret_cast<uint4 *>(dst) =
         make_uint4(pack_bf16(acc[0] * sc, acc[1] * sc), pack_bf16(acc[2] * sc, acc[3] * sc),
                    pack_bf16(acc[4] * sc, acc[5] * sc), pack_bf16(acc[6] * sc, acc[7] * sc));

@@ -170,6 +170,14 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t *p, int v) {
   return old;
 }
 
+// 32-byte streaming store (eight 32-bit words, 32-byte aligned address).
+__device__ __forceinline__ void st_global_cs_v8(void *p, const uint32_t (&v)[8]) {
+  asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+               "r"(v[7])
+               : "memory");
+}
+
 // 16-byte loads that bypass L1 (data written by other CTAs of this grid).
 __device__ __forceinline__ uint4 ld_cg_u4(const uint4 *p) {
   uint4 v;
