@@ -531,7 +531,7 @@ def run_trimul(args, rank, world, local):
                        "directions": ["outgoing", "incoming"],
                        "l2": "inputs larger than L2 (3 x 151 MB stacks)",
                        "parallelism": "independent replica per GPU"},
-            "roofline": {"bound": "tensor", "kernel": "trimul_gemm_kernel",
+            "roofline": {"bound": "tensor", "kernel": "gemm_tc_kernel",
                          "achieved": achieved, "peak": tensor_peak(peaks, clk)[0], "unit": UNIT,
                          "frac": achieved / tensor_peak(peaks, clk)[0], "traffic": None,
                          "peak_source": tensor_peak(peaks, clk)[1]},

@@ -12,7 +12,7 @@
 #include "../../include/tri_attn.h"
 #include "bf16.cuh"
 #include "common.cuh"
-#include "trimul.cuh"
+#include "gemm.cuh"
 
 namespace {
 
@@ -200,27 +200,53 @@ bool encode_bias(CUtensorMap *m, const void *base, int64_t N, int64_t H) {
 
 tri_attn_status cuda_status(cudaError_t e);
 
-// One operand of a triangle-multiplication product: a channel-major bf16
-// stack [C][N][N]. K-major operands are read as 64 (k) x 128 boxes of the
-// stored rows, MN-major ones as 64 (m or n) x 64 (k) boxes.
-bool encode_mul_stack(CUtensorMap *m, const void *base, int64_t N, int64_t C, uint32_t rows) {
+// A dense stack [batch][rows][cols] (cols contiguous) as a 3-D tensor map with
+// boxes of box_cols x box_rows and the 128-byte swizzle.
+bool encode_stack(CUtensorMap *m, const void *base, bool f32, int64_t cols, int64_t rows,
+                  int64_t batch, uint32_t box_cols, uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)C};
-  cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(N * N * 2)};
-  cuuint32_t box[3] = {64, rows, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  const int64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)(cols * es), (cuuint64_t)(rows * cols * es)};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-bool encode_mul_operand(CUtensorMap *m, const void *base, int64_t N, int64_t C, bool mn) {
-  return encode_mul_stack(m, base, N, C, mn ? 64u : 128u);
+
+// A GEMM operand whose product dimension has `mn` entries and whose summed
+// dimension has `k`: K-major when stored [mn][k], MN-major when stored [k][mn].
+bool encode_operand(CUtensorMap *m, const void *base, bool mn_major, int64_t mn, int64_t k,
+                    int64_t batch) {
+  return mn_major ? encode_stack(m, base, false, mn, k, batch, 64, 64)
+                  : encode_stack(m, base, false, k, mn, batch, 64, 128);
 }
-// The product's output: the epilogue stores 64-column boxes of 32 rows.
-bool encode_mul_output(CUtensorMap *m, void *base, int64_t N, int64_t C) {
-  return encode_mul_stack(m, base, N, C, 32u);
+
+// D = X Y^T per batch into one bf16 output [batch][M][Nn].
+tri_attn_status gemm_bf16(const void *x, bool x_mn, const void *y, bool y_mn, void *out,
+                          int64_t M, int64_t Nn, int64_t K, int64_t batch, int32_t *status,
+                          cudaStream_t stream) {
+  CUtensorMap my;
+  tri::GemmXs xs;
+  tri::GemmOuts outs;
+  if (!encode_operand(&xs.map[0], x, x_mn, M, K, batch) ||
+      !encode_operand(&my, y, y_mn, Nn, K, batch) ||
+      !encode_stack(&outs.map[0], out, false, Nn, M, batch, 64, 32))
+    return TRI_ATTN_ERR_CUDA;
+  tri::GemmArgs args;
+  args.M = (int)M;
+  args.Nn = (int)Nn;
+  args.K = (int)K;
+  args.batch = (int)batch;
+  args.nouts = 1;
+  args.cols_per_out = (int)Nn;
+  args.k_per_x = 1 << 30;           // one X tensor: every K slice comes from map 0
+  args.col_bias = nullptr;
+  args.status = status;
+  return cuda_status(tri::launch_gemm_tc(x_mn, y_mn, false, xs, my, outs, args, stream));
 }
 
 tri_attn_status check_mul(const tri_mul_problem *p) {
@@ -232,19 +258,10 @@ tri_attn_status check_mul(const tri_mul_problem *p) {
   return TRI_ATTN_OK;
 }
 
-// One product D = X Y^T of the contraction (see trimul.cu) into `out`.
+// One product D = X Y^T of the contraction (channel-major N x N per channel).
 tri_attn_status mul_product(const tri_mul_problem *p, const void *x, bool x_mn, const void *y,
                             bool y_mn, void *out, int32_t *status, cudaStream_t stream) {
-  CUtensorMap mx, my, md;
-  if (!encode_mul_operand(&mx, x, p->N, p->C, x_mn) ||
-      !encode_mul_operand(&my, y, p->N, p->C, y_mn) || !encode_mul_output(&md, out, p->N, p->C))
-    return TRI_ATTN_ERR_CUDA;
-  tri::MulArgs args;
-  args.N = (int)p->N;
-  args.C = p->C;
-  args.out = static_cast<__nv_bfloat16 *>(out);
-  args.status = status;
-  return cuda_status(tri::launch_trimul_gemm(x_mn, y_mn, mx, my, md, args, stream));
+  return gemm_bf16(x, x_mn, y, y_mn, out, p->N, p->N, p->N, p->C, status, stream);
 }
 
 tri_attn_status cuda_status(cudaError_t e) {

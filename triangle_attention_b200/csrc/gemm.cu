@@ -1,24 +1,21 @@
-// Triangle multiplicative update on sm_100a: the contraction at its core,
-//   outgoing edges: t[c][i][j] = sum_k a[c][i][k] b[c][j][k]
-//   incoming edges: t[c][i][j] = sum_k a[c][k][i] b[c][k][j]
-// and its backward, for channel-major bf16 stacks x[c][r][s] (one N x N matrix
-// per channel). The pages name triangle multiplication beside triangle
-// attention as the other pair operation their kernels accelerate
-// ("TurboPairFormer accelera fino a 1,73x l'addestramento di OpenFold3 nei
-// test", section "Dove si impiega il tempo"); the contraction is the standard
-// AlphaFold-family one.
-//
-// Per channel each of the six products (forward and the two gradients, two
-// directions) is one GEMM D[m][n] = sum_k X[m][k] Y[n][k] in which each operand
-// is read straight from its stored matrix, either K-major (the stored rows are
-// m or n, k contiguous) or MN-major (the stored rows are k, m or n contiguous):
+// Batched bf16 GEMM on the sm_100a tensor cores, D[b][m][n] = sum_k X[b](m, k)
+// Y[b](n, k) with fp32 accumulation in tensor memory. Each operand is read
+// straight from its stored matrix, either K-major (the stored rows are m or n,
+// k contiguous) or MN-major (the stored rows are k, m or n contiguous):
 // tcgen05 takes both, so no operand is ever transposed in memory.
 //
-// One CTA computes one 128x256 tile of one channel (fp32 in tensor memory):
+// It carries the triangle multiplicative update (each of its six products is
+// one batch of per-channel N x N GEMMs) and the projections around the
+// attention (LayerNorm output times the projection weights, and their
+// gradients, the weight gradients as split-K batches of fp32 partial sums).
+//
+// One CTA computes one 128x256 tile of one batch (fp32 in tensor memory):
 //   warp 0      TMA producer: 64-wide K slices of X and Y (48 KB), 2-stage ring
 //   warp 1      tensor-memory allocator and MMA issuer (N = 256 products)
-//   warps 2..5  epilogue: tensor memory -> bf16 -> the idle stage buffers ->
-//               TMA stores of 64-column boxes
+//   warps 2..5  epilogue: tensor memory -> bf16 or fp32 -> the idle stage
+//               buffers -> TMA stores (bf16: 64-column boxes, each routed to one
+//               of up to four output tensors by its column; fp32: 32-column
+//               boxes)
 // 96 KB of shared memory and 256 tensor-memory columns, so two CTAs share an
 // SM and one's epilogue overlaps the other's main loop.
 #include <cstdint>
@@ -27,7 +24,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
-#include "trimul.cuh"
+#include "gemm.cuh"
 
 namespace tri {
 namespace {
@@ -43,6 +40,9 @@ constexpr uint32_t kYBytes = kTN * kTK * 2;            // Y slice
 constexpr uint32_t kStageBytes = kXBytes + kYBytes;
 constexpr uint32_t kOffCtl = kStages * kStageBytes;
 constexpr uint32_t kAtomBytes = 64 * kTK * 2;          // one 64-wide MN atom column: 8 KB
+constexpr uint32_t kWarpStage = 16 * 1024;             // epilogue staging per warp
+static_assert(32 * kTN * 2 <= kWarpStage, "a warp's bf16 rows must fit its staging");
+static_assert(4 * kWarpStage <= kStages * kStageBytes, "staging reuses the operand stages");
 
 struct __align__(8) MulSmem {
   uint64_t full[kStages];
@@ -97,20 +97,18 @@ __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
             : make_sdesc(base + ks * 32, 16, 1024, kSwizzle128B);
 }
 
-template <bool XMN, bool YMN>
+template <bool XMN, bool YMN, bool F32>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
-trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_y,
-                   const __grid_constant__ CUtensorMap tm_d, const MulArgs a) {
+gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtensorMap tm_y,
+               const __grid_constant__ GemmOuts outs, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   MulSmem &ctl = *reinterpret_cast<MulSmem *>(smem + kOffCtl);
   volatile uint32_t *abort_flag = &ctl.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int N = a.N;
   const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * kTN, c = blockIdx.z;
-  const int nk = (N + kTK - 1) / kTK;
+  const int nk = (a.K + kTK - 1) / kTK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -134,7 +132,7 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (elect_one()) {
-      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&xs.map[0]);
       tma_prefetch_desc(&tm_y);
       int armed[kStages];
       for (int s = 0; s < kStages; ++s) armed[s] = -1;
@@ -148,7 +146,8 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
         }
         uint8_t *dst = smem + st * kStageBytes;
         mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
-        load_slice<XMN, kTM>(dst, &tm_x, &ctl.full[st], m0, kt * kTK, c);
+        const int xi = (kt * kTK) / a.k_per_x;       // the X tensor holding this K slice
+        load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], m0, kt * kTK - xi * a.k_per_x, c);
         load_slice<YMN, kTN>(dst + kXBytes, &tm_y, &ctl.full[st], n0, kt * kTK, c);
         armed[st] = kt / kStages;
       }
@@ -191,29 +190,59 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
     if (ok) {
       tc_fence_after();
       // The operand stages are idle once the accumulator is complete: each warp
-      // stages its 32 rows there (64-column boxes of 32 rows x 128 bytes, 128-byte
-      // swizzle) and stores them with TMA, which clips rows and columns past N.
-      uint8_t *stage = smem + q4 * (32 * kTN * 2);
+      // stages its 32 rows there (boxes of 32 rows x 128 bytes, 128-byte
+      // swizzle) and stores them with TMA, which clips rows and columns past the
+      // output's extent.
+      // 16 KB per warp: the four 64-column bf16 boxes of its rows, or a ring of
+      // four 32-column fp32 boxes whose slot is reused once its store has read it
+      uint8_t *stage = smem + q4 * kWarpStage;
 #pragma unroll 1
       for (int cb = 0; cb < kTN / 32; ++cb) {
         uint32_t v[32];
         tmem_ld32(tl + cb * 32, v);
-        uint8_t *box = stage + (cb >> 1) * (32 * 128);
+        if (F32) {
+          // 32 fp32 columns = one 128-byte row of a box
+          uint8_t *box = stage + (cb & 3) * (32 * 128);
+          if (cb >= 4) {
+            if (lane == 0) bulk_wait_read<3>();
+            __syncwarp();
+          }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int chunk = (cb & 1) * 4 + q;         // 16-byte chunk of the 128-byte row
-          *reinterpret_cast<uint4 *>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-              make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                         pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                         pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                         pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-        }
-        if (cb & 1) {
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tm_d, box, n0 + (cb >> 1) * 64, m0 + q4 * 32, c);
+            tma_store_3d(&outs.map[0], box, n0 + cb * 32, m0 + q4 * 32, c);
             bulk_commit_group();
+          }
+        } else {
+          uint8_t *box = stage + (cb >> 1) * (32 * 128);
+          if (a.col_bias) {
+            const float *cbias = a.col_bias + n0 + cb * 32;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (n0 + cb * 32 + e < a.Nn) v[e] = __float_as_uint(__uint_as_float(v[e]) + cbias[e]);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int chunk = (cb & 1) * 4 + q;       // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                           pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                           pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                           pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+          }
+          if (cb & 1) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int n = n0 + (cb >> 1) * 64;        // first column of the box
+            const int o = n / a.cols_per_out;          // the output tensor it belongs to
+            if (lane == 0 && o < a.nouts) {
+              tma_store_3d(&outs.map[o], box, n - o * a.cols_per_out, m0 + q4 * 32, c);
+              bulk_commit_group();
+            }
           }
         }
       }
@@ -231,25 +260,32 @@ trimul_gemm_kernel(const __grid_constant__ CUtensorMap tm_x,
   }
 }
 
-template <bool XMN, bool YMN>
-cudaError_t launch(const CUtensorMap &x, const CUtensorMap &y, const CUtensorMap &d,
-                   const MulArgs &args, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(trimul_gemm_kernel<XMN, YMN>,
+template <bool XMN, bool YMN, bool F32>
+cudaError_t launch(const GemmXs &x, const CUtensorMap &y, const GemmOuts &d,
+                   const GemmArgs &args, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((args.N + kTM - 1) / kTM, (args.N + kTN - 1) / kTN, args.C);
-  trimul_gemm_kernel<XMN, YMN><<<grid, kThreads, kSmemBytes, stream>>>(x, y, d, args);
+  dim3 grid((args.M + kTM - 1) / kTM, (args.Nn + kTN - 1) / kTN, args.batch);
+  gemm_tc_kernel<XMN, YMN, F32><<<grid, kThreads, kSmemBytes, stream>>>(x, y, d, args);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_trimul_gemm(bool x_mn, bool y_mn, const CUtensorMap &x, const CUtensorMap &y,
-                               const CUtensorMap &d, const MulArgs &args, cudaStream_t stream) {
-  if (args.N == 0 || args.C == 0) return cudaSuccess;
-  if (!x_mn && !y_mn) return launch<false, false>(x, y, d, args, stream);
-  if (!x_mn && y_mn) return launch<false, true>(x, y, d, args, stream);
-  if (x_mn && y_mn) return launch<true, true>(x, y, d, args, stream);
+cudaError_t launch_gemm_tc(bool x_mn, bool y_mn, bool f32_out, const GemmXs &x,
+                           const CUtensorMap &y, const GemmOuts &d, const GemmArgs &args,
+                           cudaStream_t stream) {
+  if (args.M == 0 || args.Nn == 0 || args.batch == 0) return cudaSuccess;
+  if (f32_out) {
+    if (!x_mn && !y_mn) return launch<false, false, true>(x, y, d, args, stream);
+    if (!x_mn && y_mn) return launch<false, true, true>(x, y, d, args, stream);
+    if (x_mn && y_mn) return launch<true, true, true>(x, y, d, args, stream);
+  } else {
+    if (!x_mn && !y_mn) return launch<false, false, false>(x, y, d, args, stream);
+    if (!x_mn && y_mn) return launch<false, true, false>(x, y, d, args, stream);
+    if (x_mn && y_mn) return launch<true, true, false>(x, y, d, args, stream);
+  }
   return cudaErrorInvalidValue;       // X MN-major with Y K-major: no product needs it
 }
 
