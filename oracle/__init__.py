@@ -244,3 +244,7 @@ def to_storage(x_rows: np.ndarray, variant: int) -> np.ndarray:
     """Map a full-row result [N(row), N(query), H, C] from the variant frame to
     the storage layout of the pair tensors (a transpose for the ending node)."""
     return x_rows if variant == STARTING else np.ascontiguousarray(x_rows.transpose(1, 0, 2, 3))
+
+
+from .proj_oracle import (layer_norm, layer_norm_bwd, proj_in_bwd, proj_in_fwd,  # noqa: E402
+                          proj_out_bwd, proj_out_fwd)
