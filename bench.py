@@ -550,14 +550,142 @@ def run_trimul(args, rank, world, local):
     return line
 
 
+BLOCK_METRIC = ("triangle-attention block fwd+bwd TFLOP/s at N=768, cz=128, H=4, c=32 bf16 "
+                "(LayerNorm, projections, attention, output projection)")
+
+
+def block_flops(N: int, cz: int, H: int, c: int) -> dict:
+    """Matmul FLOPs of each stage of the block (2 per multiply-add)."""
+    R, hc = N * N, H * c
+    f_fwd, f_bwd = flops(N, H, c)
+    return {"proj_in_fwd": 2.0 * R * cz * (4 * hc + H),
+            "attention_fwd": f_fwd, "proj_out_fwd": 2.0 * R * hc * cz,
+            "proj_out_bwd": 4.0 * R * hc * cz, "attention_bwd": f_bwd,
+            "proj_in_bwd": 4.0 * R * cz * (4 * hc + H)}
+
+
+def block_bytes(N: int, cz: int, H: int, c: int) -> dict:
+    """Minimum HBM bytes of the projection stages (each tensor read or written
+    once; the attention stages are reported by the attention line)."""
+    R, hc = N * N, H * c
+    act, pair, bias = R * cz * 2, R * hc * 2, R * H * 2
+    return {"proj_in_fwd": act + act + R * 8 + 4 * pair + bias,     # z; x, stats, q|k|v|g, bias
+            "proj_out_fwd": pair + act,                             # o; y
+            "proj_out_bwd": pair + act + pair,                      # o, dy; do
+            "proj_in_bwd": act + act + R * 8 + 4 * pair + bias + act}   # z, x, stats, grads; dz
+
+
+def run_block(args, rank, world, local):
+    """One step: the whole triangle-attention block around the attention,
+    forward and backward, N=768 (starting node, no mask), cz=128, H=4, c=32:
+    LayerNorm and the q/k/v/gate/bias projections, the attention, the output
+    projection, then the backward of each in reverse order."""
+    import triangle_attention_b200 as ta
+    N, cz, H, c = 768, 128, 4, 32
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = tri_inputs.make_block_inputs(N, cz, H, c, None, seed=11 + rank)
+    g = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in d.items()}
+    stream = torch.cuda.current_stream()
+    prob = ta.proj_problem(g["z"], H, c)
+    ws_p = ta.workspace(ta.proj_workspace_size(prob), dev)
+    x, stats, q, k, v, gate, bias = ta.proj_in_fwd(g["z"], g["gamma"], g["beta"], g["w_qkvg"],
+                                                   g["b_g"], g["w_b"], ws=ws_p)
+    aprob = ta.problem(q, None, ta.STARTING)
+    ws_f = ta.workspace(ta.fwd_workspace_size(aprob), dev)
+    ws_b = ta.workspace(ta.bwd_workspace_size(aprob), dev)
+    o, lse = ta.fwd(q, k, v, bias, gate, None, ta.STARTING, ws=ws_f)
+    y = ta.proj_out_fwd(o, g["w_o"], g["b_o"], ws=ws_p)
+    og = ta.proj_out_bwd(o, g["w_o"], g["dy"], ws=ws_p)
+    ag = ta.bwd(q, k, v, bias, gate, None, o, lse, og[0], ta.STARTING, ws=ws_b)
+    ig = ta.proj_in_bwd(g["z"], g["gamma"], g["w_qkvg"], g["w_b"], x, stats, ag[0], ag[1],
+                        ag[2], ag[4], ag[3], grads=None, ws=ws_p)
+    stages = {
+        "proj_in_fwd": lambda: ta.proj_in_fwd(g["z"], g["gamma"], g["beta"], g["w_qkvg"],
+                                              g["b_g"], g["w_b"],
+                                              outs=(x, stats, q, k, v, gate, bias), ws=ws_p),
+        "attention_fwd": lambda: ta.fwd(q, k, v, bias, gate, None, ta.STARTING, out=o, lse=lse,
+                                        ws=ws_f),
+        "proj_out_fwd": lambda: ta.proj_out_fwd(o, g["w_o"], g["b_o"], y=y, ws=ws_p),
+        "proj_out_bwd": lambda: ta.proj_out_bwd(o, g["w_o"], g["dy"], grads=og, ws=ws_p),
+        "attention_bwd": lambda: ta.bwd(q, k, v, bias, gate, None, o, lse, og[0], ta.STARTING,
+                                        grads=ag, ws=ws_b),
+        "proj_in_bwd": lambda: ta.proj_in_bwd(g["z"], g["gamma"], g["w_qkvg"], g["w_b"], x,
+                                              stats, ag[0], ag[1], ag[2], ag[4], ag[3],
+                                              grads=ig, ws=ws_p),
+    }
+    names = list(stages)
+
+    def step(events=None):
+        for i, n in enumerate(names):
+            if events:
+                events[i][0].record(stream)
+            stages[n]()
+            if events:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
+    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark()
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in names]
+          for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    for ws in (ws_p, ws_f, ws_b):
+        if ta.read_status(ws):
+            raise RuntimeError("device status set in the timed region")
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    stage_ms = {n: float(np.median([ev[i][j][0].elapsed_time(ev[i][j][1])
+                                    for i in range(args.steps)])) for j, n in enumerate(names)}
+    fl = block_flops(N, cz, H, c)
+    by = block_bytes(N, cz, H, c)
+    peaks = load_peaks()
+    proj = {n: {"ms": stage_ms[n], "GB/s": by[n] / (stage_ms[n] * 1e-3) / 1e9,
+                "frac_hbm": by[n] / (stage_ms[n] * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+            for n in by}
+    top = max(by, key=lambda n: stage_ms[n])
+    launches = {"proj_in_fwd": 2, "attention_fwd": ta.kernel_launches(aprob, False, False),
+                "proj_out_fwd": 1, "proj_out_bwd": 5,
+                "attention_bwd": ta.kernel_launches(aprob, True, False), "proj_in_bwd": 9}
+    return {"metric": BLOCK_METRIC, "value": whole_job_tflops(world, sum(fl.values()), ms),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded, tri_inputs.make_block_inputs)",
+            "config": {"workload": "block_n768_cz128", "N": N, "cz": cz, "H": H, "c": c,
+                       "variant": "starting", "mask": "none",
+                       "l2": "inputs larger than L2 (z 151 MB, q/k/v/g 151 MB each)",
+                       "parallelism": "independent replica per GPU"},
+            "stage_ms": stage_ms, "projection_stages": proj,
+            "roofline": {"bound": "hbm", "kernel": top, "achieved": proj[top]["GB/s"],
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": proj[top]["frac_hbm"], "traffic": None,
+                         "note": "algorithmic bytes of the whole stage over its event time"},
+            "clocks": clk, "gpu_launches": sum(launches.values()) * args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["attention", "trimul"], default="attention",
-                    help="attention (the default line) or the triangle multiplication")
+    ap.add_argument("--op", choices=["attention", "trimul", "block"], default="attention",
+                    help="attention (the default line), the triangle multiplication, or the "
+                         "whole block around the attention")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget-s", type=float, default=150.0,
@@ -579,8 +707,12 @@ def main():
 
     rank, world, local = dist_setup()
     try:
-        line = (run_trimul(args, rank, world, local) if args.op == "trimul"
-                else run_ours(args, rank, world, local, w))
+        if args.op == "trimul":
+            line = run_trimul(args, rank, world, local)
+        elif args.op == "block":
+            line = run_block(args, rank, world, local)
+        else:
+            line = run_ours(args, rank, world, local, w)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -290,6 +290,93 @@ tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const vo
                             const void *dt, void *da, void *db, void *workspace,
                             size_t workspace_bytes, tri_attn_stream_t stream);
 
+/* ------------------------------------------ LayerNorm and projections --
+ *
+ * The steps either side of the attention. The pages put LayerNorm at 14% of
+ * AlphaFold training time, at 10% of its theoretical speed before optimisation
+ * ("알파폴드 초기 학습 시간을 10시간으로 단축하는 ScaleFold", Stats), and fuse
+ * the gated self-attention with the projections around it ("HelixFold: An
+ * Efficient Implementation of AlphaFold2 using PaddlePaddle", proposed methods);
+ * they print neither, and this is the standard AlphaFold-family block. Per pair
+ * position (a row of z, cz channels; rows = N*N per batch element):
+ *
+ *   input side   x       = (z - mean) / sqrt(var + eps) * gamma + beta
+ *                          (biased variance over the cz channels)
+ *                q|k|v|g = x w_qkvg (+ b_g on g only)   -> [rows][H*c] each
+ *                bias[h] = x w_b[:, h]                  -> [batch][H][rows]
+ *   output side  y       = o w_o + b_o                  -> [rows][cz]
+ *
+ * q, k, v, g and bias are laid out exactly as tri_attn_fwd takes them (g are
+ * the gate logits; [rows][H*c] is [N, N, H, c]); o is the attention's output.
+ * The backward entry points return the gradient of L = sum(dq q) + sum(dk k) +
+ * sum(dv v) + sum(dg g) + sum(dbias bias), or L = sum(dy y).
+ *
+ * Types: z, x, q, k, v, g, bias, o, y and every activation gradient are bf16;
+ * w_qkvg, w_b, w_o are bf16; gamma, beta, b_g, b_o, stats and every parameter
+ * gradient are float32. LayerNorm statistics and the row sums are fp32; the
+ * products run on the tensor cores with fp32 accumulation. x is rounded to bf16
+ * once and both the projections and the bias read that rounded x.
+ *
+ * Layouts (row-major, no padding): z, x, y, dz, dy [batch*rows][cz];
+ * q, k, v, g and their gradients, o, do [batch*rows][H*c]; bias, dbias
+ * [batch][H][rows]; stats [batch*rows][2] = (mean, 1/sqrt(var + eps));
+ * w_qkvg [cz][4*H*c] (the q, k, v, g blocks side by side); b_g [H*c];
+ * w_b [cz][H]; w_o [H*c][cz]; gamma, beta, b_o [cz]. Parameter gradients have
+ * their parameter's shape.
+ *
+ * Limits (TRI_ATTN_ERR_UNSUPPORTED otherwise): cz in {64, 128, 192, 256};
+ * 1 <= H <= 8; H*c in {64, 128, 192, 256}; batch*rows < 2^31. rows = 0 or batch = 0
+ * computes nothing but still zeroes the parameter gradients; the activation
+ * pointers may then be NULL (those of the parameters and their gradients may not).
+ *
+ * Ownership, errors, determinism: as for the attention. Every pointer is a
+ * caller-owned, 16-byte aligned device pointer (x and stats too: the forward
+ * writes them, the backward reads them). The workspace (tri_proj_workspace_size
+ * bytes, one size for all four calls) holds the status word and the fp32
+ * partial sums; parameter gradients are summed over the rows in a fixed order
+ * (per-warp or per-split partials, then one ordered sum), so repeated calls are
+ * bit-identical.
+ */
+typedef struct {
+    int64_t rows;   /* pair positions per batch element (N*N) */
+    int32_t batch;  /* independent pair maps, >= 0 */
+    int32_t cz;     /* channels of z */
+    int32_t H;      /* heads */
+    int32_t c;      /* channels per head */
+    float eps;      /* LayerNorm epsilon (> 0) */
+    int32_t reserved; /* must be 0 */
+} tri_proj_problem;
+
+tri_attn_status tri_proj_workspace_size(const tri_proj_problem *prob, size_t *bytes);
+
+/* x, stats, q, k, v, g, bias from z. */
+tri_attn_status tri_proj_in_fwd(const tri_proj_problem *prob, const void *z, const float *gamma,
+                                const float *beta, const void *w_qkvg, const float *b_g,
+                                const void *w_b, void *x, float *stats, void *q, void *k,
+                                void *v, void *g, void *bias, void *workspace,
+                                size_t workspace_bytes, tri_attn_stream_t stream);
+
+/* dz and the parameter gradients from dq, dk, dv, dg, dbias (x and stats as
+ * the forward wrote them). */
+tri_attn_status tri_proj_in_bwd(const tri_proj_problem *prob, const void *z, const float *gamma,
+                                const void *w_qkvg, const void *w_b, const void *x,
+                                const float *stats, const void *dq, const void *dk,
+                                const void *dv, const void *dg, const void *dbias, void *dz,
+                                float *dgamma, float *dbeta, float *dw_qkvg, float *db_g,
+                                float *dw_b, void *workspace, size_t workspace_bytes,
+                                tri_attn_stream_t stream);
+
+/* y = o w_o + b_o. */
+tri_attn_status tri_proj_out_fwd(const tri_proj_problem *prob, const void *o, const void *w_o,
+                                 const float *b_o, void *y, void *workspace,
+                                 size_t workspace_bytes, tri_attn_stream_t stream);
+
+/* do, dw_o, db_o from dy. */
+tri_attn_status tri_proj_out_bwd(const tri_proj_problem *prob, const void *o, const void *w_o,
+                                 const void *dy, void *do_, float *dw_o, float *db_o,
+                                 void *workspace, size_t workspace_bytes,
+                                 tri_attn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,3 +60,40 @@ def test_triangle_multiplication_autograd():
             assert rel_l2(np64(t[i]), ref_t) <= 4e-3
             assert rel_l2(np64(la.grad[i]), ref_da) <= 4e-3
             assert rel_l2(np64(lb.grad[i]), ref_db) <= 4e-3
+
+
+@pytest.mark.parametrize("variant", [STARTING, ENDING])
+def test_attention_block_matches_the_oracle_chain(variant):
+    """LayerNorm -> projections -> attention -> output projection through
+    autograd, against the oracles chained in fp64. Each GPU step rounds its
+    outputs to bf16, so the bound is twice the single-kernel one."""
+    from tri_inputs import full_mask, make_block_inputs
+    N, cz, H, c, eps = 40, 128, 4, 32, 1e-5
+    R, hc, shape = N * N, H * c, (N, N, H, c)
+    d = make_block_inputs(N, cz, H, c, None, seed=50 + variant)
+    mask = full_mask(N, seed=9, keep_prob=0.9)
+    names = ("z", "gamma", "beta", "w_qkvg", "b_g", "w_b", "w_o", "b_o")
+    leaves = {k: d[k].cuda().requires_grad_(True) for k in names}
+    y = ta.triangle_attention_block(*(leaves[k] for k in names), mask.cuda(), variant, eps)
+    y.backward(d["dy"].cuda())
+    torch.cuda.synchronize()
+
+    f = oracle.proj_in_fwd(d["z"].reshape(R, cz), d["gamma"], d["beta"], d["w_qkvg"], d["b_g"],
+                           d["w_b"], eps)
+    q, k, v, gate = (f[n].reshape(shape) for n in ("q", "k", "v", "gate"))
+    bias = f["bias"].reshape(H, N, N)
+    out, _ = oracle.fwd(q, k, v, bias, gate, mask, variant)
+    out = oracle.to_storage(out, variant).reshape(R, hc)
+    y_ref = oracle.proj_out_fwd(out, d["w_o"], d["b_o"])
+    ob = oracle.proj_out_bwd(out, d["w_o"], d["dy"].reshape(R, cz))
+    dq, dk, dv, dg, db = oracle.bwd(q, k, v, bias, gate, ob["do"].reshape(shape), mask, variant)
+    dq, dk, dv, dg = (oracle.to_storage(t, variant).reshape(R, hc) for t in (dq, dk, dv, dg))
+    ib = oracle.proj_in_bwd(d["z"].reshape(R, cz), d["gamma"], d["beta"], d["w_qkvg"], d["w_b"],
+                            eps, dq, dk, dv, dg, db.reshape(H, R))
+    tol = 2 * BF16_REL
+    assert rel_l2(np64(y).reshape(R, cz), y_ref) <= tol
+    ref = {"z": ib["dz"], "gamma": ib["dgamma"], "beta": ib["dbeta"], "w_qkvg": ib["dw_qkvg"],
+           "b_g": ib["db_g"], "w_b": ib["dw_b"], "w_o": ob["dw_o"], "b_o": ob["db_o"]}
+    for k in names:
+        err = rel_l2(np64(leaves[k].grad).reshape(ref[k].shape), ref[k])
+        assert err <= tol, f"d{k}: relative L2 error {err:.3e}"

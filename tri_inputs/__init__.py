@@ -123,3 +123,38 @@ def full_mask(N: int, seed: int, keep_prob: float = 0.8, fully_masked_rows=()) -
     for r in fully_masked_rows:
         m[r, :] = 0
     return torch.from_numpy(m)
+
+
+def make_block_inputs(N: int, cz: int = 128, H: int = 4, c: int = 32, batch: Optional[int] = None,
+                      seed: int = 0) -> dict:
+    """Draw the pair representation, the parameters of the block around the
+    attention (LayerNorm and projections) and the gradients that flow into it.
+
+    Draw order: z, gamma, beta, w_qkvg, b_g, w_b, w_o, b_o, then the incoming
+    gradients dq, dk, dv, dg, dbias (same shapes as q, k, v, g, bias) and dy.
+    z ~ N(0, 1) + a per-row offset N(0, 1) (LayerNorm must remove it); gamma ~
+    1 + 0.1 N(0, 1); beta, b_g, b_o ~ 0.1 N(0, 1); weights ~ N(0, 1/fan_in);
+    gradients ~ N(0, 1). Activations and weights are bf16, the LayerNorm
+    parameters and biases float32. With batch=None the pair tensors are
+    [N, N, ...], else [batch, N, N, ...]."""
+    rng = np.random.default_rng(seed)
+    lead = (N, N) if batch is None else (batch, N, N)
+    hc = H * c
+
+    def draw(shape, s=1.0, shift=0.0, dtype="bf16"):
+        x = rng.standard_normal(shape, dtype=np.float32) * np.float32(s) + np.float32(shift)
+        return _round(x, dtype)
+
+    z = rng.standard_normal(lead + (cz,), dtype=np.float32)
+    z += rng.standard_normal(lead + (1,), dtype=np.float32)
+    out = {"z": _round(z, "bf16"),
+           "gamma": draw((cz,), 0.1, 1.0, "f32"), "beta": draw((cz,), 0.1, 0.0, "f32"),
+           "w_qkvg": draw((cz, 4 * hc), cz ** -0.5), "b_g": draw((hc,), 0.1, 0.0, "f32"),
+           "w_b": draw((cz, H), cz ** -0.5), "w_o": draw((hc, cz), hc ** -0.5),
+           "b_o": draw((cz,), 0.1, 0.0, "f32")}
+    for name in ("dq", "dk", "dv", "dg"):
+        out[name] = draw(lead + (H, c))
+    out["dbias"] = draw(lead[:-2] + (H, N, N))
+    out["dy"] = draw(lead + (cz,))
+    out["meta"] = dict(N=N, cz=cz, H=H, c=c, batch=batch, seed=seed)
+    return out

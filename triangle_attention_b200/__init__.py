@@ -10,6 +10,9 @@ Entry points (names follow the C ABI in include/tri_attn.h):
     bwd(q, k, v, bias, gate, mask, out, lse, dout, variant) -> (dq, dk, dv, dbias, dgate)
     fwd_workspace_size / bwd_workspace_size / read_status
     TriangleAttention: torch.autograd.Function over fwd/bwd.
+    mul_fwd / mul_bwd, TriangleMultiplication: the triangle multiplicative update.
+    proj_in_fwd / proj_in_bwd / proj_out_fwd / proj_out_bwd: LayerNorm and the
+    projections around the attention; TriangleAttentionBlock chains them.
 """
 
 from __future__ import annotations
@@ -77,6 +80,12 @@ class MulProblem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("C", ctypes.c_int32), ("direction", ctypes.c_int32)]
 
 
+class ProjProblem(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int64), ("batch", ctypes.c_int32), ("cz", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("c", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("reserved", ctypes.c_int32)]
+
+
 class Problem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int32), ("c", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("variant", ctypes.c_int32),
@@ -112,11 +121,18 @@ def lib():
         L.tri_mul_workspace_size.argtypes = [MP, ctypes.POINTER(sz)]
         L.tri_mul_fwd.argtypes = [MP, P, P, P, P, sz, P]
         L.tri_mul_bwd.argtypes = [MP, P, P, P, P, P, P, sz, P]
+        JP = ctypes.POINTER(ProjProblem)
+        L.tri_proj_workspace_size.argtypes = [JP, ctypes.POINTER(sz)]
+        L.tri_proj_in_fwd.argtypes = [JP] + [P] * 13 + [P, sz, P]
+        L.tri_proj_in_bwd.argtypes = [JP] + [P] * 17 + [P, sz, P]
+        L.tri_proj_out_fwd.argtypes = [JP] + [P] * 4 + [P, sz, P]
+        L.tri_proj_out_bwd.argtypes = [JP] + [P] * 6 + [P, sz, P]
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
                   L.tri_attn_kernel_launches, L.tri_attn_read_status,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
-                  L.tri_mul_bwd):
+                  L.tri_mul_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
+                  L.tri_proj_in_bwd, L.tri_proj_out_fwd, L.tri_proj_out_bwd):
             f.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -287,6 +303,31 @@ def mul_bwd(a, b, dt, direction: int = OUTGOING, grads=None, ws=None, stream=Non
     return da, db
 
 
+def _attention_fwd(q, k, v, bias, gate, mask, variant):
+    """fwd, unbatched or over a leading batch dimension (each element in turn)."""
+    if q.dim() == 4:
+        return fwd(q, k, v, bias, gate, mask, variant)
+    out = torch.empty_like(q)
+    B, N, _, H, _ = q.shape
+    lse = torch.empty((B, N, H, N), dtype=torch.float32, device=q.device)
+    for i in range(B):
+        fwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i], variant,
+            out=out[i], lse=lse[i])
+    return out, lse
+
+
+def _attention_bwd(q, k, v, bias, gate, mask, out, lse, dout, variant):
+    """bwd, unbatched or over a leading batch dimension."""
+    if q.dim() == 4:
+        return bwd(q, k, v, bias, gate, mask, out, lse, dout, variant)
+    dq, dk, dv, dgate = (torch.empty_like(t) for t in (q, k, v, gate))
+    dbias = torch.empty_like(bias)
+    for i in range(q.shape[0]):
+        bwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i], out[i],
+            lse[i], dout[i], variant, grads=(dq[i], dk[i], dv[i], dbias[i], dgate[i]))
+    return dq, dk, dv, dbias, dgate
+
+
 class TriangleAttention(torch.autograd.Function):
     """out = TriangleAttention.apply(q, k, v, bias, gate, mask, variant).
 
@@ -297,37 +338,17 @@ class TriangleAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, bias, gate, mask=None, variant=STARTING):
-        batched = q.dim() == 5
-        ctx.batched = batched
         ctx.mask = mask
         ctx.variant = variant
-        if not batched:
-            out, lse = fwd(q, k, v, bias, gate, mask, variant)
-        else:
-            out = torch.empty_like(q)
-            B, N, _, H, _ = q.shape
-            lse = torch.empty((B, N, H, N), dtype=torch.float32, device=q.device)
-            for i in range(B):
-                fwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i],
-                    variant, out=out[i], lse=lse[i])
+        out, lse = _attention_fwd(q, k, v, bias, gate, mask, variant)
         ctx.save_for_backward(q, k, v, bias, gate, out, lse)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, bias, gate, out, lse = ctx.saved_tensors
-        dout = dout.contiguous()
-        mask = ctx.mask
-        if not ctx.batched:
-            dq, dk, dv, dbias, dgate = bwd(q, k, v, bias, gate, mask, out, lse, dout,
-                                           ctx.variant)
-        else:
-            dq, dk, dv, dgate = (torch.empty_like(t) for t in (q, k, v, gate))
-            dbias = torch.empty_like(bias)
-            for i in range(q.shape[0]):
-                bwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i],
-                    out[i], lse[i], dout[i], ctx.variant,
-                    grads=(dq[i], dk[i], dv[i], dbias[i], dgate[i]))
+        dq, dk, dv, dbias, dgate = _attention_bwd(q, k, v, bias, gate, ctx.mask, out, lse,
+                                                  dout.contiguous(), ctx.variant)
         return dq, dk, dv, dbias, dgate, None, None
 
 
@@ -363,3 +384,141 @@ class TriangleMultiplication(torch.autograd.Function):
             for i in range(a.shape[0]):
                 mul_bwd(a[i], b[i], dt[i], ctx.direction, grads=(da[i], db[i]))
         return da, db, None
+
+
+# ------------------------------------------------ LayerNorm and projections --
+
+def proj_problem(z_or_y: torch.Tensor, H: int, c: int, eps: float = 1e-5) -> ProjProblem:
+    """Problem of a pair tensor [N, N, cz] or [B, N, N, cz] (rows = N*N per batch
+    element)."""
+    if z_or_y.dim() not in (3, 4) or z_or_y.shape[-3] != z_or_y.shape[-2]:
+        raise ValueError("pair tensors are [N, N, cz] or [B, N, N, cz]")
+    B = z_or_y.shape[0] if z_or_y.dim() == 4 else 1
+    N, cz = z_or_y.shape[-2], z_or_y.shape[-1]
+    return ProjProblem(N * N, B, cz, H, c, eps, 0)
+
+
+def proj_workspace_size(prob: ProjProblem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().tri_proj_workspace_size(ctypes.byref(prob), ctypes.byref(n)),
+           "tri_proj_workspace_size")
+    return n.value
+
+
+def _proj_ws(prob, ws, device):
+    return ws if ws is not None else workspace(proj_workspace_size(prob), device)
+
+
+def proj_in_fwd(z, gamma, beta, w_qkvg, b_g, w_b, eps: float = 1e-5, outs=None, ws=None,
+                stream=None) -> tuple:
+    """LayerNorm of the pair representation z ([N, N, cz] or [B, N, N, cz], bf16)
+    and its projections: returns (x, stats, q, k, v, g, bias) with x like z,
+    stats float32 [.., N, N, 2], q/k/v/g [.., N, N, H, c] bf16 (g: gate logits),
+    bias [.., H, N, N] bf16. w_qkvg [cz, 4*H*c] bf16; b_g [H*c] and gamma, beta
+    [cz] float32; w_b [cz, H] bf16."""
+    H = w_b.shape[1]
+    c = w_qkvg.shape[1] // (4 * H)
+    prob = proj_problem(z, H, c, eps)
+    lead = z.shape[:-1]
+    if outs is None:
+        x = torch.empty_like(z)
+        stats = torch.empty(lead + (2,), dtype=torch.float32, device=z.device)
+        q, k, v, g = (torch.empty(lead + (H, c), dtype=z.dtype, device=z.device)
+                      for _ in range(4))
+        bias = torch.empty(lead[:-2] + (H,) + lead[-2:], dtype=z.dtype, device=z.device)
+        outs = (x, stats, q, k, v, g, bias)
+    _contig(z, gamma, beta, w_qkvg, b_g, w_b, *outs)
+    ws = _proj_ws(prob, ws, z.device)
+    _check(lib().tri_proj_in_fwd(ctypes.byref(prob), _p(z), _p(gamma), _p(beta), _p(w_qkvg),
+                                 _p(b_g), _p(w_b), *map(_p, outs), _p(ws), ws.numel(),
+                                 _stream(stream)), "tri_proj_in_fwd")
+    return outs
+
+
+def proj_in_bwd(z, gamma, w_qkvg, w_b, x, stats, dq, dk, dv, dg, dbias, eps: float = 1e-5,
+                grads=None, ws=None, stream=None) -> tuple:
+    """(dz, dgamma, dbeta, dw_qkvg, db_g, dw_b) of the input side, given the
+    gradients of q, k, v, g and bias; x and stats as proj_in_fwd returned them.
+    Parameter gradients are float32 with their parameter's shape."""
+    H = w_b.shape[1]
+    c = w_qkvg.shape[1] // (4 * H)
+    prob = proj_problem(z, H, c, eps)
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=z.device)
+        grads = (torch.empty_like(z), torch.empty(gamma.shape, **f32),
+                 torch.empty(gamma.shape, **f32), torch.empty(w_qkvg.shape, **f32),
+                 torch.empty((H * c,), **f32), torch.empty(w_b.shape, **f32))
+    _contig(z, gamma, w_qkvg, w_b, x, stats, dq, dk, dv, dg, dbias, *grads)
+    ws = _proj_ws(prob, ws, z.device)
+    _check(lib().tri_proj_in_bwd(ctypes.byref(prob), _p(z), _p(gamma), _p(w_qkvg), _p(w_b),
+                                 _p(x), _p(stats), _p(dq), _p(dk), _p(dv), _p(dg), _p(dbias),
+                                 *map(_p, grads), _p(ws), ws.numel(), _stream(stream)),
+           "tri_proj_in_bwd")
+    return grads
+
+
+def proj_out_fwd(o, w_o, b_o, y=None, ws=None, stream=None) -> torch.Tensor:
+    """y = o w_o + b_o: o [.., N, N, H, c] bf16 (the attention output), w_o
+    [H*c, cz] bf16, b_o [cz] float32; y [.., N, N, cz] bf16."""
+    H, c = o.shape[-2], o.shape[-1]
+    cz = w_o.shape[1]
+    if y is None:
+        y = torch.empty(o.shape[:-2] + (cz,), dtype=o.dtype, device=o.device)
+    prob = proj_problem(y, H, c)
+    _contig(o, w_o, b_o, y)
+    ws = _proj_ws(prob, ws, o.device)
+    _check(lib().tri_proj_out_fwd(ctypes.byref(prob), _p(o), _p(w_o), _p(b_o), _p(y), _p(ws),
+                                  ws.numel(), _stream(stream)), "tri_proj_out_fwd")
+    return y
+
+
+def proj_out_bwd(o, w_o, dy, grads=None, ws=None, stream=None) -> tuple:
+    """(do, dw_o, db_o) of L = sum(dy * y) for y = proj_out_fwd(o, w_o, b_o)."""
+    H, c = o.shape[-2], o.shape[-1]
+    prob = proj_problem(dy, H, c)
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=o.device)
+        grads = (torch.empty_like(o), torch.empty(w_o.shape, **f32),
+                 torch.empty((w_o.shape[1],), **f32))
+    _contig(o, w_o, dy, *grads)
+    ws = _proj_ws(prob, ws, o.device)
+    _check(lib().tri_proj_out_bwd(ctypes.byref(prob), _p(o), _p(w_o), _p(dy), *map(_p, grads),
+                                  _p(ws), ws.numel(), _stream(stream)), "tri_proj_out_bwd")
+    return grads
+
+
+class TriangleAttentionBlock(torch.autograd.Function):
+    """y = TriangleAttentionBlock.apply(z, gamma, beta, w_qkvg, b_g, w_b, w_o, b_o,
+    mask, variant, eps): LayerNorm, the q/k/v/gate/bias projections, gated
+    triangle attention and the output projection; z [N, N, cz] or [B, N, N, cz]
+    bf16 -> y like z (the update that is added to z). Every step runs in the
+    library; parameter gradients are computed in float32."""
+
+    @staticmethod
+    def forward(ctx, z, gamma, beta, w_qkvg, b_g, w_b, w_o, b_o, mask=None, variant=STARTING,
+                eps=1e-5):
+        z = z.contiguous()
+        x, stats, q, k, v, g, bias = proj_in_fwd(z, gamma, beta, w_qkvg, b_g, w_b, eps)
+        o, lse = _attention_fwd(q, k, v, bias, g, mask, variant)
+        y = proj_out_fwd(o, w_o, b_o)
+        ctx.eps, ctx.mask, ctx.variant = eps, mask, variant
+        ctx.save_for_backward(z, gamma, w_qkvg, w_b, w_o, x, stats, q, k, v, g, bias, o, lse)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        z, gamma, w_qkvg, w_b, w_o, x, stats, q, k, v, g, bias, o, lse = ctx.saved_tensors
+        do, dw_o, db_o = proj_out_bwd(o, w_o, dy.contiguous())
+        dq, dk, dv, dbias, dg = _attention_bwd(q, k, v, bias, g, ctx.mask, o, lse, do,
+                                               ctx.variant)
+        dz, dgamma, dbeta, dw_qkvg, db_g, dw_b = proj_in_bwd(z, gamma, w_qkvg, w_b, x, stats, dq,
+                                                             dk, dv, dg, dbias, ctx.eps)
+        return dz, dgamma, dbeta, dw_qkvg, db_g, dw_b, dw_o, db_o, None, None, None
+
+
+def triangle_attention_block(z, gamma, beta, w_qkvg, b_g, w_b, w_o, b_o, mask=None,
+                             variant: int = STARTING, eps: float = 1e-5) -> torch.Tensor:
+    """Differentiable LayerNorm -> projections -> gated triangle attention ->
+    output projection; see TriangleAttentionBlock."""
+    return TriangleAttentionBlock.apply(z, gamma, beta, w_qkvg, b_g, w_b, w_o, b_o, mask,
+                                        variant, eps)

@@ -5,6 +5,8 @@
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
+#include <utility>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -13,6 +15,7 @@
 #include "bf16.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "proj.cuh"
 
 namespace {
 
@@ -229,14 +232,14 @@ bool encode_operand(CUtensorMap *m, const void *base, bool mn_major, int64_t mn,
 tri_attn_status gemm_bf16(const void *x, bool x_mn, const void *y, bool y_mn, void *out,
                           int64_t M, int64_t Nn, int64_t K, int64_t batch, int32_t *status,
                           cudaStream_t stream) {
-  CUtensorMap my;
-  tri::GemmXs xs;
+  tri::GemmMaps ys;
+  tri::GemmMaps xs;
   tri::GemmOuts outs;
   if (!encode_operand(&xs.map[0], x, x_mn, M, K, batch) ||
-      !encode_operand(&my, y, y_mn, Nn, K, batch) ||
+      !encode_operand(&ys.map[0], y, y_mn, Nn, K, batch) ||
       !encode_stack(&outs.map[0], out, false, Nn, M, batch, 64, 32))
     return TRI_ATTN_ERR_CUDA;
-  tri::GemmArgs args;
+  tri::GemmArgs args{};
   args.M = (int)M;
   args.Nn = (int)Nn;
   args.K = (int)K;
@@ -246,7 +249,7 @@ tri_attn_status gemm_bf16(const void *x, bool x_mn, const void *y, bool y_mn, vo
   args.k_per_x = 1 << 30;           // one X tensor: every K slice comes from map 0
   args.col_bias = nullptr;
   args.status = status;
-  return cuda_status(tri::launch_gemm_tc(x_mn, y_mn, false, xs, my, outs, args, stream));
+  return cuda_status(tri::launch_gemm_tc(x_mn, y_mn, false, xs, ys, outs, args, stream));
 }
 
 tri_attn_status check_mul(const tri_mul_problem *p) {
@@ -631,6 +634,367 @@ tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const vo
     if (st == TRI_ATTN_OK) st = mul_product(prob, a, false, dt, true, db, status, stream);
   }
   return st;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------ LayerNorm and projections --
+
+namespace {
+
+constexpr int kGemmTileM = 128, kGemmTileN = 256, kGemmTileK = 64;
+constexpr int kSplitTargetCtas = 2 * 148;      // two CTAs per SM
+
+int64_t proj_total_rows(const tri_proj_problem *p) { return p->rows * (int64_t)p->batch; }
+
+tri_attn_status check_proj(const tri_proj_problem *p) {
+  if (!p) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->rows < 0 || p->batch < 0 || p->cz < 1 || p->H < 1 || p->c < 1 || !(p->eps > 0.0f) ||
+      !std::isfinite(p->eps) || p->reserved != 0)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->cz % 64 || p->cz > 256 || p->H > 8 || p->c > 256 || (p->H * p->c) % 64 ||
+      p->H * p->c > 256)
+    return TRI_ATTN_ERR_UNSUPPORTED;
+  if (p->rows > 0 && p->batch > 0 && proj_total_rows(p) >= (int64_t(1) << 31))
+    return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
+// Split of a weight-gradient product (M x Nn, summed over K rows) into batches
+// of k_split rows (a multiple of the 64-row K step) so that the grid fills two
+// CTAs per SM; every batch gets at least one row.
+struct KSplit {
+  int k_split, n;
+};
+KSplit split_k(int64_t M, int64_t Nn, int64_t K) {
+  const int64_t tiles = ((M + kGemmTileM - 1) / kGemmTileM) * ((Nn + kGemmTileN - 1) / kGemmTileN);
+  int64_t s = kSplitTargetCtas / tiles;
+  if (s < 1) s = 1;
+  int64_t ks = (K + s - 1) / s;
+  ks = (ks + kGemmTileK - 1) / kGemmTileK * kGemmTileK;
+  if (ks < kGemmTileK) ks = kGemmTileK;
+  return {(int)ks, (int)((K + ks - 1) / ks)};
+}
+
+struct ProjWs {
+  int32_t *status;
+  float *dx;      // [R][cz] fp32
+  float *part;    // partial sums
+};
+
+// Workspace: the status word, dx, and the largest set of partial sums.
+size_t carve_proj(const tri_proj_problem *p, void *base, ProjWs *ws) {
+  const int64_t R = proj_total_rows(p), cz = p->cz, hc = (int64_t)p->H * p->c;
+  const int64_t warps = tri::proj_partials();
+  int64_t part = warps * cz * (2 + p->H);
+  part = std::max(part, warps * std::max(hc, cz));
+  if (R > 0) {
+    const KSplit si = split_k(cz, 4 * hc, R), so = split_k(hc, cz, R);
+    part = std::max(part, (int64_t)si.n * cz * 4 * hc);
+    part = std::max(part, (int64_t)so.n * hc * cz);
+  }
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + kAlign - 1) / kAlign * kAlign;
+    return o;
+  };
+  const size_t o_status = take(sizeof(int32_t));
+  const size_t o_dx = take((size_t)R * cz * sizeof(float));
+  const size_t o_part = take((size_t)part * sizeof(float));
+  if (ws && base) {
+    char *b = static_cast<char *>(base);
+    ws->status = reinterpret_cast<int32_t *>(b + o_status);
+    ws->dx = reinterpret_cast<float *>(b + o_dx);
+    ws->part = reinterpret_cast<float *>(b + o_part);
+  }
+  return off;
+}
+
+tri_attn_status proj_begin(const tri_proj_problem *p, void *workspace, size_t workspace_bytes,
+                           ProjWs *ws) {
+  tri_attn_status st = check_proj(p);
+  if (st != TRI_ATTN_OK) return st;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < carve_proj(p, nullptr, nullptr))
+    return TRI_ATTN_ERR_WORKSPACE;
+  carve_proj(p, workspace, ws);
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status zero_f32(float *p, size_t n, cudaStream_t s) {
+  return cuda_status(cudaMemsetAsync(p, 0, n * sizeof(float), s));
+}
+
+// fp32 weight gradient D[M][Nn] = sum over the K rows of X[k][m] Y[k][n], X
+// stored [K][M], Y as ny tensors [K][Nn / ny] side by side along n: split-K
+// partials into ws->part, then one ordered sum into out [M][Nn].
+tri_attn_status weight_grad(const void *x, const void *const *y, int ny, int64_t M, int64_t Nn,
+                            int64_t K, float *out, const ProjWs &ws, cudaStream_t stream) {
+  const KSplit sp = split_k(M, Nn, K);
+  const int64_t per_y = Nn / ny;
+  tri::GemmMaps xs, ys;
+  tri::GemmOuts outs;
+  if (!encode_operand(&xs.map[0], x, true, M, K, 1) ||
+      !encode_stack(&outs.map[0], ws.part, true, Nn, M, sp.n, 32, 32))
+    return TRI_ATTN_ERR_CUDA;
+  for (int i = 0; i < ny; ++i)
+    if (!encode_operand(&ys.map[i], y[i], true, per_y, K, 1)) return TRI_ATTN_ERR_CUDA;
+  tri::GemmArgs args{};
+  args.M = (int)M;
+  args.Nn = (int)Nn;
+  args.K = (int)K;
+  args.batch = sp.n;
+  args.nouts = 1;
+  args.cols_per_out = (int)Nn;
+  args.k_per_x = 1 << 30;
+  args.n_per_y = ny > 1 ? (int)per_y : 0;
+  args.ny = ny;
+  args.k_split = sp.k_split;
+  args.status = ws.status;
+  tri_attn_status st = cuda_status(tri::launch_gemm_tc(true, true, true, xs, ys, outs, args, stream));
+  if (st != TRI_ATTN_OK) return st;
+  return cuda_status(
+      tri::launch_ordered_sum(ws.part, sp.n, M * Nn, M * Nn, out, M * Nn, M * Nn, stream));
+}
+
+// Column sums of a bf16 [R][cols] matrix into out[cols], in a fixed order.
+tri_attn_status column_sums(const void *m, int64_t R, int64_t cols, float *out, const ProjWs &ws,
+                            cudaStream_t stream) {
+  const int warps = tri::proj_partials();
+  cudaError_t e = tri::launch_colsum(static_cast<const __nv_bfloat16 *>(m), R, (int)cols,
+                                     ws.part, stream);
+  if (e == cudaSuccess)
+    e = tri::launch_ordered_sum(ws.part, warps, cols, cols, out, cols, cols, stream);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_attn_status tri_proj_workspace_size(const tri_proj_problem *prob, size_t *bytes) {
+  tri_attn_status st = check_proj(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!bytes) return TRI_ATTN_ERR_INVALID_ARG;
+  *bytes = carve_proj(prob, nullptr, nullptr);
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status tri_proj_in_fwd(const tri_proj_problem *prob, const void *z, const float *gamma,
+                                const float *beta, const void *w_qkvg, const float *b_g,
+                                const void *w_b, void *x, float *stats, void *q, void *k,
+                                void *v, void *g, void *bias, void *workspace,
+                                size_t workspace_bytes, tri_attn_stream_t stream_) {
+  ProjWs ws;
+  tri_attn_status st = proj_begin(prob, workspace, workspace_bytes, &ws);
+  if (st != TRI_ATTN_OK) return st;
+  for (const void *p : {(const void *)gamma, (const void *)beta, w_qkvg, (const void *)b_g, w_b})
+    TRI_CHECK_PTR(p);
+  const int64_t R = proj_total_rows(prob), cz = prob->cz, hc = (int64_t)prob->H * prob->c;
+  if (R == 0) return TRI_ATTN_OK;      // no rows: nothing to do, nothing enqueued
+  for (const void *p : {z, (const void *)x, (const void *)stats, (const void *)q, (const void *)k,
+                        (const void *)v, (const void *)g, (const void *)bias})
+    TRI_CHECK_PTR(p);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaMemsetAsync(ws.status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return TRI_ATTN_ERR_CUDA;
+  tri::ProjArgs a{};
+  a.rows = R;
+  a.rows_per = prob->rows;
+  a.cz = prob->cz;
+  a.H = prob->H;
+  a.eps = prob->eps;
+  a.z = static_cast<const __nv_bfloat16 *>(z);
+  a.gamma = gamma;
+  a.beta = beta;
+  a.w_b = static_cast<const __nv_bfloat16 *>(w_b);
+  a.x = static_cast<__nv_bfloat16 *>(x);
+  a.stats = stats;
+  a.bias = static_cast<__nv_bfloat16 *>(bias);
+  st = cuda_status(tri::launch_ln_fwd(a, stream));
+  if (st != TRI_ATTN_OK) return st;
+  // q | k | v | g = x w_qkvg: x K-major, w_qkvg [cz][4Hc] MN-major, each
+  // 64-column box of the product routed to its output, b_g added to g
+  tri::GemmMaps ys;
+  tri::GemmMaps xs;
+  tri::GemmOuts outs;
+  void *dst[4] = {q, k, v, g};
+  if (!encode_operand(&xs.map[0], x, false, R, cz, 1) ||
+      !encode_operand(&ys.map[0], w_qkvg, true, 4 * hc, cz, 1))
+    return TRI_ATTN_ERR_CUDA;
+  for (int o = 0; o < 4; ++o)
+    if (!encode_stack(&outs.map[o], dst[o], false, hc, R, 1, 64, 32)) return TRI_ATTN_ERR_CUDA;
+  tri::GemmArgs args{};
+  args.M = (int)R;
+  args.Nn = (int)(4 * hc);
+  args.K = (int)cz;
+  args.batch = 1;
+  args.nouts = 4;
+  args.cols_per_out = (int)hc;
+  args.k_per_x = 1 << 30;
+  args.col_bias = b_g;
+  args.col_bias_from = (int)(3 * hc);
+  args.status = ws.status;
+  return cuda_status(tri::launch_gemm_tc(false, true, false, xs, ys, outs, args, stream));
+}
+
+tri_attn_status tri_proj_in_bwd(const tri_proj_problem *prob, const void *z, const float *gamma,
+                                const void *w_qkvg, const void *w_b, const void *x,
+                                const float *stats, const void *dq, const void *dk,
+                                const void *dv, const void *dg, const void *dbias, void *dz,
+                                float *dgamma, float *dbeta, float *dw_qkvg, float *db_g,
+                                float *dw_b, void *workspace, size_t workspace_bytes,
+                                tri_attn_stream_t stream_) {
+  ProjWs ws;
+  tri_attn_status st = proj_begin(prob, workspace, workspace_bytes, &ws);
+  if (st != TRI_ATTN_OK) return st;
+  for (const void *p : {(const void *)gamma, w_qkvg, w_b, (const void *)dgamma,
+                        (const void *)dbeta, (const void *)dw_qkvg, (const void *)db_g,
+                        (const void *)dw_b})
+    TRI_CHECK_PTR(p);
+  const int64_t R = proj_total_rows(prob), cz = prob->cz, hc = (int64_t)prob->H * prob->c;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (R == 0) {
+    // no rows: every parameter gradient is an empty sum
+    for (auto t : {std::make_pair(dgamma, cz), std::make_pair(dbeta, cz),
+                   std::make_pair(dw_qkvg, cz * 4 * hc), std::make_pair(db_g, hc),
+                   std::make_pair(dw_b, cz * prob->H)})
+      if ((st = zero_f32(t.first, (size_t)t.second, stream)) != TRI_ATTN_OK) return st;
+    return TRI_ATTN_OK;
+  }
+  for (const void *p : {z, x, (const void *)stats, dq, dk, dv, dg, dbias, (const void *)dz})
+    TRI_CHECK_PTR(p);
+  if (cudaMemsetAsync(ws.status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return TRI_ATTN_ERR_CUDA;
+  // dx = [dq dk dv dg] w_qkvg^T (fp32): four K-major X maps along K, w_qkvg K-major
+  {
+    tri::GemmMaps ys;
+    tri::GemmMaps xs;
+    tri::GemmOuts outs;
+    const void *src[4] = {dq, dk, dv, dg};
+    for (int o = 0; o < 4; ++o)
+      if (!encode_operand(&xs.map[o], src[o], false, R, hc, 1)) return TRI_ATTN_ERR_CUDA;
+    if (!encode_operand(&ys.map[0], w_qkvg, false, cz, 4 * hc, 1) ||
+        !encode_stack(&outs.map[0], ws.dx, true, cz, R, 1, 32, 32))
+      return TRI_ATTN_ERR_CUDA;
+    tri::GemmArgs args{};
+    args.M = (int)R;
+    args.Nn = (int)cz;
+    args.K = (int)(4 * hc);
+    args.batch = 1;
+    args.nouts = 1;
+    args.cols_per_out = (int)cz;
+    args.k_per_x = (int)hc;
+    args.status = ws.status;
+    st = cuda_status(tri::launch_gemm_tc(false, false, true, xs, ys, outs, args, stream));
+    if (st != TRI_ATTN_OK) return st;
+  }
+  // LayerNorm backward: dz, and per-warp partials of dgamma | dbeta | dw_b
+  tri::ProjArgs a{};
+  a.rows = R;
+  a.rows_per = prob->rows;
+  a.cz = prob->cz;
+  a.H = prob->H;
+  a.eps = prob->eps;
+  a.z = static_cast<const __nv_bfloat16 *>(z);
+  a.gamma = gamma;
+  a.w_b = static_cast<const __nv_bfloat16 *>(w_b);
+  a.x = static_cast<__nv_bfloat16 *>(const_cast<void *>(x));
+  a.stats = const_cast<float *>(stats);
+  a.dx = ws.dx;
+  a.dbias = static_cast<const __nv_bfloat16 *>(dbias);
+  a.dz = static_cast<__nv_bfloat16 *>(dz);
+  a.part = ws.part;
+  cudaError_t e = tri::launch_ln_bwd(a, stream);
+  const int64_t warps = tri::proj_partials(), pw = cz * (2 + prob->H);
+  if (e == cudaSuccess) e = tri::launch_ordered_sum(ws.part, warps, pw, cz, dgamma, cz, cz, stream);
+  if (e == cudaSuccess)
+    e = tri::launch_ordered_sum(ws.part + cz, warps, pw, cz, dbeta, cz, cz, stream);
+  if (e == cudaSuccess)
+    e = tri::launch_ordered_sum(ws.part + 2 * cz, warps, pw, cz * prob->H, dw_b, cz * prob->H,
+                                cz * prob->H, stream);
+  if ((st = cuda_status(e)) != TRI_ATTN_OK) return st;
+  if ((st = column_sums(dg, R, hc, db_g, ws, stream)) != TRI_ATTN_OK) return st;
+  // dw_qkvg = x^T [dq dk dv dg]
+  const void *grads[4] = {dq, dk, dv, dg};
+  return weight_grad(x, grads, 4, cz, 4 * hc, R, dw_qkvg, ws, stream);
+}
+
+tri_attn_status tri_proj_out_fwd(const tri_proj_problem *prob, const void *o, const void *w_o,
+                                 const float *b_o, void *y, void *workspace,
+                                 size_t workspace_bytes, tri_attn_stream_t stream_) {
+  ProjWs ws;
+  tri_attn_status st = proj_begin(prob, workspace, workspace_bytes, &ws);
+  if (st != TRI_ATTN_OK) return st;
+  for (const void *p : {w_o, (const void *)b_o}) TRI_CHECK_PTR(p);
+  const int64_t R = proj_total_rows(prob), cz = prob->cz, hc = (int64_t)prob->H * prob->c;
+  if (R == 0) return TRI_ATTN_OK;      // no rows: nothing to do, nothing enqueued
+  for (const void *p : {o, (const void *)y}) TRI_CHECK_PTR(p);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaMemsetAsync(ws.status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return TRI_ATTN_ERR_CUDA;
+  // y = o w_o + b_o: o K-major, w_o [Hc][cz] MN-major
+  tri::GemmMaps ys;
+  tri::GemmMaps xs;
+  tri::GemmOuts outs;
+  if (!encode_operand(&xs.map[0], o, false, R, hc, 1) ||
+      !encode_operand(&ys.map[0], w_o, true, cz, hc, 1) ||
+      !encode_stack(&outs.map[0], y, false, cz, R, 1, 64, 32))
+    return TRI_ATTN_ERR_CUDA;
+  tri::GemmArgs args{};
+  args.M = (int)R;
+  args.Nn = (int)cz;
+  args.K = (int)hc;
+  args.batch = 1;
+  args.nouts = 1;
+  args.cols_per_out = (int)cz;
+  args.k_per_x = 1 << 30;
+  args.col_bias = b_o;
+  args.col_bias_from = 0;
+  args.status = ws.status;
+  return cuda_status(tri::launch_gemm_tc(false, true, false, xs, ys, outs, args, stream));
+}
+
+tri_attn_status tri_proj_out_bwd(const tri_proj_problem *prob, const void *o, const void *w_o,
+                                 const void *dy, void *do_, float *dw_o, float *db_o,
+                                 void *workspace, size_t workspace_bytes,
+                                 tri_attn_stream_t stream_) {
+  ProjWs ws;
+  tri_attn_status st = proj_begin(prob, workspace, workspace_bytes, &ws);
+  if (st != TRI_ATTN_OK) return st;
+  for (const void *p : {w_o, (const void *)dw_o, (const void *)db_o}) TRI_CHECK_PTR(p);
+  const int64_t R = proj_total_rows(prob), cz = prob->cz, hc = (int64_t)prob->H * prob->c;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (R == 0) {
+    if ((st = zero_f32(dw_o, (size_t)(hc * cz), stream)) != TRI_ATTN_OK) return st;
+    return zero_f32(db_o, (size_t)cz, stream);
+  }
+  for (const void *p : {o, dy, (const void *)do_}) TRI_CHECK_PTR(p);
+  if (cudaMemsetAsync(ws.status, 0, sizeof(int32_t), stream) != cudaSuccess)
+    return TRI_ATTN_ERR_CUDA;
+  // do = dy w_o^T: dy K-major, w_o [Hc][cz] K-major
+  {
+    tri::GemmMaps ys;
+    tri::GemmMaps xs;
+    tri::GemmOuts outs;
+    if (!encode_operand(&xs.map[0], dy, false, R, cz, 1) ||
+        !encode_operand(&ys.map[0], w_o, false, hc, cz, 1) ||
+        !encode_stack(&outs.map[0], do_, false, hc, R, 1, 64, 32))
+      return TRI_ATTN_ERR_CUDA;
+    tri::GemmArgs args{};
+    args.M = (int)R;
+    args.Nn = (int)hc;
+    args.K = (int)cz;
+    args.batch = 1;
+    args.nouts = 1;
+    args.cols_per_out = (int)hc;
+    args.k_per_x = 1 << 30;
+    args.status = ws.status;
+    st = cuda_status(tri::launch_gemm_tc(false, false, false, xs, ys, outs, args, stream));
+    if (st != TRI_ATTN_OK) return st;
+  }
+  if ((st = weight_grad(o, &dy, 1, hc, cz, R, dw_o, ws, stream)) != TRI_ATTN_OK) return st;
+  return column_sums(dy, R, cz, db_o, ws, stream);
 }
 
 }  // extern "C"

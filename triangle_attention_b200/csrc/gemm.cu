@@ -87,6 +87,21 @@ __device__ __forceinline__ void load_slice(uint8_t *dst, const CUtensorMap *map,
   }
 }
 
+// The Y slice when Y is several tensors along n: each box (64 rows MN-major,
+// 128 K-major) comes from the tensor holding its first row; rows past the last
+// tensor read past its extent, which the copy fills with zeros.
+template <bool MN>
+__device__ __forceinline__ void load_y_slice(uint8_t *dst, const GemmMaps &ys, const GemmArgs &a,
+                                             uint64_t *bar, int n0, int k0, int c) {
+  constexpr int kBox = MN ? 64 : 128;
+#pragma unroll
+  for (int h = 0; h < kTN / kBox; ++h) {
+    const int n = n0 + kBox * h;
+    const int yi = min(n / a.n_per_y, a.ny - 1);
+    load_slice<MN, kBox>(dst + h * (kBox * kTK * 2), &ys.map[yi], bar, n - yi * a.n_per_y, k0, c);
+  }
+}
+
 // Descriptor of the 16-wide K step ks of a slice (128-byte swizzle). K-major:
 // rows of 128 bytes, 8-row groups 1 KB apart, the K step 32 bytes along a row.
 // MN-major: 64-wide MN atom columns 8 KB apart, 8 k-rows per 1 KB group, the K
@@ -99,7 +114,7 @@ __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
 
 template <bool XMN, bool YMN, bool F32>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
-gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtensorMap tm_y,
+gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ GemmMaps ys,
                const __grid_constant__ GemmOuts outs, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -108,7 +123,12 @@ gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtens
   volatile uint32_t *abort_flag = &ctl.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * kTN, c = blockIdx.z;
-  const int nk = (a.K + kTK - 1) / kTK;
+  // split-K: batch index c takes K columns [kbeg, kend) of operands that have no
+  // batch dimension of their own; otherwise c is every tensor's batch coordinate
+  const int kbeg = a.k_split ? c * a.k_split : 0;
+  const int kend = a.k_split ? min(a.K, kbeg + a.k_split) : a.K;
+  const int cin = a.k_split ? 0 : c;
+  const int nk = (kend - kbeg + kTK - 1) / kTK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -133,7 +153,7 @@ gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtens
     // ------------------------------------------------------------ producer --
     if (elect_one()) {
       tma_prefetch_desc(&xs.map[0]);
-      tma_prefetch_desc(&tm_y);
+      tma_prefetch_desc(&ys.map[0]);
       int armed[kStages];
       for (int s = 0; s < kStages; ++s) armed[s] = -1;
       bool ok = true;
@@ -146,9 +166,13 @@ gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtens
         }
         uint8_t *dst = smem + st * kStageBytes;
         mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
-        const int xi = (kt * kTK) / a.k_per_x;       // the X tensor holding this K slice
-        load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], m0, kt * kTK - xi * a.k_per_x, c);
-        load_slice<YMN, kTN>(dst + kXBytes, &tm_y, &ctl.full[st], n0, kt * kTK, c);
+        const int k = kbeg + kt * kTK;
+        const int xi = k / a.k_per_x;                  // the X tensor holding this K slice
+        load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], m0, k - xi * a.k_per_x, cin);
+        if (a.n_per_y)
+          load_y_slice<YMN>(dst + kXBytes, ys, a, &ctl.full[st], n0, k, cin);
+        else
+          load_slice<YMN, kTN>(dst + kXBytes, &ys.map[0], &ctl.full[st], n0, k, cin);
         armed[st] = kt / kStages;
       }
       if (!ok)
@@ -220,10 +244,12 @@ gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtens
         } else {
           uint8_t *box = stage + (cb >> 1) * (32 * 128);
           if (a.col_bias) {
-            const float *cbias = a.col_bias + n0 + cb * 32;
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (n0 + cb * 32 + e < a.Nn) v[e] = __float_as_uint(__uint_as_float(v[e]) + cbias[e]);
+            for (int e = 0; e < 32; ++e) {
+              const int col = n0 + cb * 32 + e;
+              if (col >= a.col_bias_from && col < a.Nn)
+                v[e] = __float_as_uint(__uint_as_float(v[e]) + a.col_bias[col - a.col_bias_from]);
+            }
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -261,7 +287,7 @@ gemm_tc_kernel(const __grid_constant__ GemmXs xs, const __grid_constant__ CUtens
 }
 
 template <bool XMN, bool YMN, bool F32>
-cudaError_t launch(const GemmXs &x, const CUtensorMap &y, const GemmOuts &d,
+cudaError_t launch(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
                    const GemmArgs &args, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -273,10 +299,16 @@ cudaError_t launch(const GemmXs &x, const CUtensorMap &y, const GemmOuts &d,
 
 }  // namespace
 
-cudaError_t launch_gemm_tc(bool x_mn, bool y_mn, bool f32_out, const GemmXs &x,
-                           const CUtensorMap &y, const GemmOuts &d, const GemmArgs &args,
+cudaError_t launch_gemm_tc(bool x_mn, bool y_mn, bool f32_out, const GemmMaps &x,
+                           const GemmMaps &y, const GemmOuts &d, const GemmArgs &args,
                            cudaStream_t stream) {
   if (args.M == 0 || args.Nn == 0 || args.batch == 0) return cudaSuccess;
+  // an empty K range would leave the accumulator unwritten: callers zero such outputs
+  if (args.K <= 0 || (args.k_split && (args.k_split % kTK || (int64_t)(args.batch - 1) * args.k_split >= args.K)))
+    return cudaErrorInvalidValue;
+  if (args.k_per_x <= 0 || args.k_per_x % kTK) return cudaErrorInvalidValue;
+  if (args.n_per_y && (args.ny < 1 || args.ny > 4 || args.n_per_y % (y_mn ? 64 : 128)))
+    return cudaErrorInvalidValue;
   if (f32_out) {
     if (!x_mn && !y_mn) return launch<false, false, true>(x, y, d, args, stream);
     if (!x_mn && y_mn) return launch<false, true, true>(x, y, d, args, stream);

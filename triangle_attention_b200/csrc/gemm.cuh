@@ -14,12 +14,19 @@ struct GemmArgs {
   int cols_per_out;                  // columns of D per bf16 output tensor (multiple of 64)
   int k_per_x;                       // K columns per X tensor map (multiple of 64): X may
                                      // be up to four tensors laid side by side along K
-  const float *col_bias;             // bf16 outputs: added to column n before rounding, or null
+  int n_per_y, ny;                   // Y may be ny <= 4 tensors of n_per_y rows n each
+                                     // (a multiple of 64 MN-major, of 128 K-major)
+  int k_split;                       // > 0: split-K, batch index b sums K columns
+                                     // [b*k_split, min(K, (b+1)*k_split)) of operands with no
+                                     // batch dimension (multiple of 64); 0: a true batch
+  const float *col_bias;             // bf16 outputs: col_bias[n - col_bias_from] is added to
+  int col_bias_from;                 // column n >= col_bias_from before rounding (or null)
   int32_t *status;
 };
 
-// X operand maps: K columns [i*k_per_x, (i+1)*k_per_x) come from map i.
-struct GemmXs {
+// Operand maps. X: K columns [i*k_per_x, (i+1)*k_per_x) come from map i.
+// Y: rows n in [i*n_per_y, (i+1)*n_per_y) come from map i (n_per_y = 0: one map).
+struct GemmMaps {
   CUtensorMap map[4];
 };
 
@@ -32,8 +39,8 @@ struct GemmOuts {
 // x_mn / y_mn: the operand's stored matrix has k as its rows (MN-major) instead
 // of its columns (K-major); the maps come with the matching boxes (64 x 128
 // K-major, 64 x 64 MN-major).
-cudaError_t launch_gemm_tc(bool x_mn, bool y_mn, bool f32_out, const GemmXs &x,
-                           const CUtensorMap &y, const GemmOuts &d, const GemmArgs &args,
+cudaError_t launch_gemm_tc(bool x_mn, bool y_mn, bool f32_out, const GemmMaps &x,
+                           const GemmMaps &y, const GemmOuts &d, const GemmArgs &args,
                            cudaStream_t stream);
 
 }  // namespace tri

@@ -1,0 +1,389 @@
+// LayerNorm of the pair representation and the small projections around the
+// attention's input projections (the large ones run on the tensor cores, see
+// gemm.cu). The pages put LayerNorm at 14% of AlphaFold training time, at 10%
+// of its theoretical speed before optimisation ("알파폴드 초기 학습 시간을
+// 10시간으로 단축하는 ScaleFold", Stats), and fuse the gated attention with its
+// projections ("HelixFold: An Efficient Implementation of AlphaFold2 using
+// PaddlePaddle", proposed methods).
+//
+// One warp per pair position (row of z [rows][cz]); lane l holds channels
+// l*CPL .. l*CPL + CPL - 1, so a warp reads and writes whole rows contiguously.
+// Reductions over rows (dgamma, dbeta, the bias weights, the gate bias) are
+// accumulated per warp over a fixed set of rows and summed over the warps in a
+// fixed order: repeated calls are bit-identical.
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ptx.cuh"
+#include "proj.cuh"
+
+namespace tri {
+namespace {
+
+constexpr int kMaxHeads = 8;
+constexpr int kRowsPerWarp = 4;      // rows whose loads a warp keeps in flight
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float bf16_round(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+// bias and dbias are [batch][H][rows_per]: entry (h, row) sits at
+// bias_base(row) + h * rows_per (rows < 2^31, so 32-bit division suffices)
+__device__ __forceinline__ int64_t bias_base(const ProjArgs &a, int64_t row) {
+  const uint32_t b = (uint32_t)row / (uint32_t)a.rows_per;
+  return row + (int64_t)b * (a.H - 1) * a.rows_per;
+}
+
+// CPL consecutive bf16 channels of one row: 4 to 16 bytes per lane, one or
+// more vector loads.
+template <int CPL>
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&v)[CPL]) {
+  uint32_t w[CPL / 2];
+  if constexpr (CPL == 8) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(p);
+    w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
+  } else if constexpr (CPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(p);
+    w[0] = u.x, w[1] = u.y;
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPL / 2; ++e) w[e] = reinterpret_cast<const uint32_t *>(p)[e];
+  }
+#pragma unroll
+  for (int e = 0; e < CPL / 2; ++e) {
+    v[2 * e] = bf16lo(w[e]);
+    v[2 * e + 1] = bf16hi(w[e]);
+  }
+}
+
+template <int CPL>
+__device__ __forceinline__ void store_row(__nv_bfloat16 *p, const float (&v)[CPL]) {
+  uint32_t w[CPL / 2];
+#pragma unroll
+  for (int e = 0; e < CPL / 2; ++e) w[e] = pack_bf16(v[2 * e], v[2 * e + 1]);
+  if constexpr (CPL == 8) {
+    *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (CPL == 4) {
+    *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPL / 2; ++e) reinterpret_cast<uint32_t *>(p)[e] = w[e];
+  }
+}
+
+template <int CPL>
+__device__ __forceinline__ void load_row_f32(const float *p, float (&v)[CPL]) {
+  if constexpr (CPL % 4 == 0) {
+#pragma unroll
+    for (int e = 0; e < CPL; e += 4) {
+      const float4 u = *reinterpret_cast<const float4 *>(p + e);
+      v[e] = u.x, v[e + 1] = u.y, v[e + 2] = u.z, v[e + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < CPL; e += 2) {
+      const float2 u = *reinterpret_cast<const float2 *>(p + e);
+      v[e] = u.x, v[e + 1] = u.y;
+    }
+  }
+}
+
+// This lane's rows of w_b [cz][H] (channels c0 .. c0 + CPL - 1), zero past H.
+template <int CPL, int HM>
+__device__ __forceinline__ void load_wb(const ProjArgs &a, int c0, float (&wb)[CPL][HM]) {
+#pragma unroll
+  for (int e = 0; e < CPL; ++e)
+#pragma unroll
+    for (int h = 0; h < HM; ++h)
+      wb[e][h] = h < a.H ? __bfloat162float(a.w_b[(c0 + e) * a.H + h]) : 0.0f;
+}
+
+// Rows are taken in groups of kRowsPerWarp by the warps in turn: group g goes
+// to warp g mod (number of warps), so a warp keeps kRowsPerWarp rows of loads
+// in flight.
+__device__ __forceinline__ int64_t first_group() {
+  return blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
+}
+__device__ __forceinline__ int64_t group_stride() { return (int64_t)gridDim.x * (blockDim.x >> 5); }
+
+// x = LayerNorm(z) * gamma + beta (bf16), stats = (mean, rstd), and
+// bias[h][row] = sum_c x[c] w_b[c][h] from the rounded x the GEMM also reads.
+template <int CPL, int HM>
+__global__ void __launch_bounds__(256, CPL <= 4 ? 4 : 2) ln_fwd_kernel(ProjArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int c0 = lane * CPL;
+  float wb[CPL][HM];
+  load_wb<CPL, HM>(a, c0, wb);
+  float g[CPL], bt[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) {
+    g[e] = a.gamma[c0 + e];
+    bt[e] = a.beta[c0 + e];
+  }
+  const int64_t groups = (a.rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  for (int64_t grp = first_group(); grp < groups; grp += group_stride()) {
+    const int64_t r0 = grp * kRowsPerWarp;
+    float v[kRowsPerWarp][CPL];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+      if (r0 + r < a.rows) load_row<CPL>(a.z + (r0 + r) * a.cz + c0, v[r]);
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const int64_t row = r0 + r;
+      if (row >= a.rows) break;                    // warp-uniform
+      float s = 0.0f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) s += v[r][e];
+      const float mean = warp_sum(s) / a.cz;
+      float q = 0.0f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) q += (v[r][e] - mean) * (v[r][e] - mean);
+      const float rstd = rsqrtf(warp_sum(q) / a.cz + a.eps);
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) v[r][e] = bf16_round((v[r][e] - mean) * rstd * g[e] + bt[e]);
+      store_row<CPL>(a.x + row * a.cz + c0, v[r]);
+      if (lane == 0) reinterpret_cast<float2 *>(a.stats)[row] = make_float2(mean, rstd);
+#pragma unroll
+      for (int h = 0; h < HM; ++h) {
+        if (h >= a.H) break;
+        float d = 0.0f;
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) d += v[r][e] * wb[e][h];
+        d = warp_sum(d);
+        if (lane == 0) a.bias[bias_base(a, row) + h * a.rows_per] = __float2bfloat16_rn(d);
+      }
+    }
+  }
+}
+
+// dz from dx (the projections' gradient w.r.t. x, fp32) plus the bias term
+// sum_h dbias[h][row] w_b[c][h]; partial sums of dgamma, dbeta and
+// dw_b[c][h] = sum_rows x[c] dbias[h][row] (x as the forward stored it), one
+// set per block: each warp accumulates its rows, then the block's warps are
+// added in warp order.
+template <int CPL, int HM>
+__global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs a) {
+  __shared__ float acc[256 * (2 + kMaxHeads)];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = lane * CPL;
+  float wb[CPL][HM];
+  load_wb<CPL, HM>(a, c0, wb);
+  float g[CPL], dg[CPL], db[CPL], dwb[CPL][HM];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) {
+    g[e] = a.gamma[c0 + e];
+    dg[e] = db[e] = 0.0f;
+#pragma unroll
+    for (int h = 0; h < HM; ++h) dwb[e][h] = 0.0f;
+  }
+  const int64_t groups = (a.rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  for (int64_t grp = first_group(); grp < groups; grp += group_stride()) {
+    const int64_t r0 = grp * kRowsPerWarp;
+    float z[kRowsPerWarp][CPL], dx[kRowsPerWarp][CPL];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+      if (r0 + r < a.rows) {
+        load_row<CPL>(a.z + (r0 + r) * a.cz + c0, z[r]);
+        load_row_f32<CPL>(a.dx + (r0 + r) * a.cz + c0, dx[r]);
+      }
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r) {
+      const int64_t row = r0 + r;
+      if (row >= a.rows) break;                    // warp-uniform
+      float x[CPL];
+      load_row<CPL>(a.x + row * a.cz + c0, x);
+      const float2 st = reinterpret_cast<const float2 *>(a.stats)[row];
+      const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
+#pragma unroll
+      for (int h = 0; h < HM; ++h) {
+        if (h >= a.H) break;
+        const float dbh = __bfloat162float(dbias[h * a.rows_per]);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+          dx[r][e] += dbh * wb[e][h];
+          dwb[e][h] += x[e] * dbh;
+        }
+      }
+      float s1 = 0.0f, s2 = 0.0f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) {
+        const float xh = (z[r][e] - st.x) * st.y;
+        z[r][e] = xh;
+        dg[e] += dx[r][e] * xh;
+        db[e] += dx[r][e];
+        const float gx = dx[r][e] * g[e];
+        s1 += gx;
+        s2 += gx * xh;
+      }
+      const float m1 = warp_sum(s1) / a.cz, m2 = warp_sum(s2) / a.cz;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) z[r][e] = st.y * (dx[r][e] * g[e] - m1 - z[r][e] * m2);
+      store_row<CPL>(a.dz + row * a.cz + c0, z[r]);
+    }
+  }
+  // block partials [dgamma cz | dbeta cz | dw_b cz*H], warps added in order
+  const int len = a.cz * (2 + a.H);
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    if (warp == w) {
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) {
+        float *p0 = &acc[c0 + e], *p1 = &acc[a.cz + c0 + e];
+        *p0 = (w ? *p0 : 0.0f) + dg[e];
+        *p1 = (w ? *p1 : 0.0f) + db[e];
+#pragma unroll
+        for (int h = 0; h < HM; ++h)
+          if (h < a.H) {
+            float *p2 = &acc[2 * a.cz + (c0 + e) * a.H + h];
+            *p2 = (w ? *p2 : 0.0f) + dwb[e][h];
+          }
+      }
+    }
+    __syncthreads();
+  }
+  float *part = a.part + blockIdx.x * (int64_t)len;
+  for (int i = threadIdx.x; i < len; i += blockDim.x) part[i] = acc[i];
+}
+
+// Per-warp partial column sums of a [rows][cols] bf16 matrix (cols = 32*CPL),
+// added per block in warp order: one partial row per block.
+template <int CPL>
+__global__ void __launch_bounds__(256) colsum_kernel(const __nv_bfloat16 *m, int64_t rows,
+                                                     int cols, float *part) {
+  __shared__ float acc[256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c0 = lane * CPL;
+  float s[CPL];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) s[e] = 0.0f;
+  const int64_t groups = (rows + kRowsPerWarp - 1) / kRowsPerWarp;
+  for (int64_t grp = first_group(); grp < groups; grp += group_stride()) {
+    const int64_t r0 = grp * kRowsPerWarp;
+    float v[kRowsPerWarp][CPL];
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+      if (r0 + r < rows) load_row<CPL>(m + (r0 + r) * cols + c0, v[r]);
+#pragma unroll
+    for (int r = 0; r < kRowsPerWarp; ++r)
+      if (r0 + r < rows)
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) s[e] += v[r][e];
+  }
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    if (warp == w)
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[c0 + e] = (w ? acc[c0 + e] : 0.0f) + s[e];
+    __syncthreads();
+  }
+  for (int i = threadIdx.x; i < cols; i += blockDim.x) part[blockIdx.x * (int64_t)cols + i] = acc[i];
+}
+
+// out[i] = sum over k < n of part[k * part_stride + i], element i landing at
+// out + (i / width) * out_stride + i % width. A block of 32 warps takes 32
+// consecutive elements (one per lane); warp w adds the k of its fixed share
+// [w n / 32, (w + 1) n / 32) in order, then the 32 warp sums are added in warp
+// order, so the result does not depend on scheduling.
+__global__ void __launch_bounds__(1024) ordered_sum_kernel(const float *part, int64_t n,
+                                                           int64_t part_stride, int64_t len,
+                                                           float *out, int64_t width,
+                                                           int64_t out_stride) {
+  __shared__ float ws[32][33];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t i = blockIdx.x * 32ll + lane;
+  const int64_t k0 = warp * n / 32, k1 = (warp + 1) * n / 32;
+  float s = 0.0f;
+  if (i < len) {
+    const float *p = part + i;
+    int64_t k = k0;
+    for (; k + 4 <= k1; k += 4) {
+      const float v0 = p[k * part_stride], v1 = p[(k + 1) * part_stride];
+      const float v2 = p[(k + 2) * part_stride], v3 = p[(k + 3) * part_stride];
+      s += v0;
+      s += v1;
+      s += v2;
+      s += v3;
+    }
+    for (; k < k1; ++k) s += p[k * part_stride];
+  }
+  ws[warp][lane] = s;
+  __syncthreads();
+  if (warp == 0 && i < len) {
+    float t = 0.0f;
+    for (int w = 0; w < 32; ++w) t += ws[w][lane];
+    out[(i / width) * out_stride + i % width] = t;
+  }
+}
+
+}  // namespace
+
+int proj_partials() { return kProjBlocks; }
+
+template <int HM>
+cudaError_t launch_ln_fwd_h(const ProjArgs &a, cudaStream_t stream) {
+  const int blocks = kProjBlocks;
+  if (a.cz % 64) return cudaErrorInvalidValue;
+  switch (a.cz / 32) {
+    case 2: ln_fwd_kernel<2, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 4: ln_fwd_kernel<4, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 6: ln_fwd_kernel<6, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 8: ln_fwd_kernel<8, HM><<<blocks, 256, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_fwd(const ProjArgs &a, cudaStream_t stream) {
+  if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
+  return a.H <= 4 ? launch_ln_fwd_h<4>(a, stream) : launch_ln_fwd_h<kMaxHeads>(a, stream);
+}
+
+template <int HM>
+cudaError_t launch_ln_bwd_h(const ProjArgs &a, cudaStream_t stream) {
+  const int blocks = kProjBlocks;
+  if (a.cz % 64) return cudaErrorInvalidValue;
+  switch (a.cz / 32) {
+    case 2: ln_bwd_kernel<2, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 4: ln_bwd_kernel<4, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 6: ln_bwd_kernel<6, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 8: ln_bwd_kernel<8, HM><<<blocks, 256, 0, stream>>>(a); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ln_bwd(const ProjArgs &a, cudaStream_t stream) {
+  if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
+  return a.H <= 4 ? launch_ln_bwd_h<4>(a, stream) : launch_ln_bwd_h<kMaxHeads>(a, stream);
+}
+
+cudaError_t launch_colsum(const __nv_bfloat16 *m, int64_t rows, int cols, float *part,
+                          cudaStream_t stream) {
+  const int blocks = kProjBlocks;
+  if (cols % 64) return cudaErrorInvalidValue;
+  switch (cols / 32) {
+    case 2: colsum_kernel<2><<<blocks, 256, 0, stream>>>(m, rows, cols, part); break;
+    case 4: colsum_kernel<4><<<blocks, 256, 0, stream>>>(m, rows, cols, part); break;
+    case 6: colsum_kernel<6><<<blocks, 256, 0, stream>>>(m, rows, cols, part); break;
+    case 8: colsum_kernel<8><<<blocks, 256, 0, stream>>>(m, rows, cols, part); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ordered_sum(const float *part, int64_t n, int64_t part_stride, int64_t len,
+                               float *out, int64_t width, int64_t out_stride,
+                               cudaStream_t stream) {
+  if (len == 0) return cudaSuccess;
+  const int64_t blocks = (len + 31) / 32;
+  ordered_sum_kernel<<<(unsigned)blocks, 1024, 0, stream>>>(part, n, part_stride, len, out,
+                                                           width, out_stride);
+  return cudaGetLastError();
+}
+
+}  // namespace tri
