@@ -24,12 +24,6 @@ namespace {
 constexpr int kMaxHeads = 8;
 constexpr int kRowsPerWarp = 4;      // rows whose loads a warp keeps in flight
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ float bf16_round(float v) {
   return __bfloat162float(__float2bfloat16_rn(v));
 }
@@ -41,11 +35,10 @@ __device__ __forceinline__ int64_t bias_base(const ProjArgs &a, int64_t row) {
   return row + (int64_t)b * (a.H - 1) * a.rows_per;
 }
 
-// CPL consecutive bf16 channels of one row: 4 to 16 bytes per lane, one or
-// more vector loads.
+// CPL consecutive bf16 channels of one row, packed in pairs: one vector load
+// of 4 to 16 bytes per lane.
 template <int CPL>
-__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&v)[CPL]) {
-  uint32_t w[CPL / 2];
+__device__ __forceinline__ void load_raw(const __nv_bfloat16 *p, uint32_t (&w)[CPL / 2]) {
   if constexpr (CPL == 8) {
     const uint4 u = *reinterpret_cast<const uint4 *>(p);
     w[0] = u.x, w[1] = u.y, w[2] = u.z, w[3] = u.w;
@@ -56,11 +49,22 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&v)[CPL]
 #pragma unroll
     for (int e = 0; e < CPL / 2; ++e) w[e] = reinterpret_cast<const uint32_t *>(p)[e];
   }
+}
+
+template <int CPL>
+__device__ __forceinline__ void unpack(const uint32_t (&w)[CPL / 2], float (&v)[CPL]) {
 #pragma unroll
   for (int e = 0; e < CPL / 2; ++e) {
     v[2 * e] = bf16lo(w[e]);
     v[2 * e + 1] = bf16hi(w[e]);
   }
+}
+
+template <int CPL>
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *p, float (&v)[CPL]) {
+  uint32_t w[CPL / 2];
+  load_raw<CPL>(p, w);
+  unpack<CPL>(w, v);
 }
 
 template <int CPL>
@@ -95,6 +99,35 @@ __device__ __forceinline__ void load_row_f32(const float *p, float (&v)[CPL]) {
   }
 }
 
+constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
+
+// Warp sum of NV values at once (NV a power of two, at most 32) by recursive
+// halving: at lane offsets 16, 8, ... each lane keeps half of its values and
+// adds its partner's copy of that half, then the single value left is summed
+// over the remaining offsets. NV - 1 + 5 - log2(NV) shuffles instead of 5 NV.
+// Lane l returns the total of value l >> (5 - log2 NV); the order of the
+// additions is fixed, so the result does not depend on scheduling.
+template <int NV>
+__device__ __forceinline__ float reduce_scatter(float (&v)[NV], int lane) {
+  constexpr int L = ilog2(NV);
+  static_assert((1 << L) == NV && NV <= 32, "NV must be a power of two <= 32");
+#pragma unroll
+  for (int st = 0, n = NV; st < L; ++st, n >>= 1) {
+    const int off = 16 >> st;
+    const bool upper = lane & off;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float keep = upper ? v[j + n / 2] : v[j];
+      const float send = upper ? v[j] : v[j + n / 2];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float t = v[0];
+#pragma unroll
+  for (int off = 16 >> L; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
+}
+
 // This lane's rows of w_b [cz][H] (channels c0 .. c0 + CPL - 1), zero past H.
 template <int CPL, int HM>
 __device__ __forceinline__ void load_wb(const ProjArgs &a, int c0, float (&wb)[CPL][HM]) {
@@ -105,20 +138,38 @@ __device__ __forceinline__ void load_wb(const ProjArgs &a, int c0, float (&wb)[C
       wb[e][h] = h < a.H ? __bfloat162float(a.w_b[(c0 + e) * a.H + h]) : 0.0f;
 }
 
-// Rows are taken in groups of kRowsPerWarp by the warps in turn: group g goes
-// to warp g mod (number of warps), so a warp keeps kRowsPerWarp rows of loads
-// in flight.
+// Rows are taken in groups of RPW by the warps in turn: group g goes to warp
+// g mod (number of warps). A warp loads its next group while it works on the
+// current one.
 __device__ __forceinline__ int64_t first_group() {
   return blockIdx.x * (int64_t)(blockDim.x >> 5) + (threadIdx.x >> 5);
 }
 __device__ __forceinline__ int64_t group_stride() { return (int64_t)gridDim.x * (blockDim.x >> 5); }
 
+template <int CPL, int RPW>
+__device__ __forceinline__ void load_group(const __nv_bfloat16 *m, int64_t rows, int cols,
+                                           int64_t r0, int c0, uint32_t (&w)[RPW][CPL / 2]) {
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) {
+    if (r0 + r < rows) {
+      load_raw<CPL>(m + (r0 + r) * cols + c0, w[r]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < CPL / 2; ++e) w[r][e] = 0u;
+    }
+  }
+}
+
 // x = LayerNorm(z) * gamma + beta (bf16), stats = (mean, rstd), and
 // bias[h][row] = sum_c x[c] w_b[c][h] from the rounded x the GEMM also reads.
+// One warp per row, four rows at a time: the row sums of the four rows, then
+// the 4 x HM bias dot products, are each one recursive-halving warp sum.
 template <int CPL, int HM>
-__global__ void __launch_bounds__(256, CPL <= 4 ? 4 : 2) ln_fwd_kernel(ProjArgs a) {
+__global__ void __launch_bounds__(256, CPL <= 4 ? 3 : 2) ln_fwd_kernel(ProjArgs a) {
+  constexpr int R = kRowsPerWarp;
   const int lane = threadIdx.x & 31;
   const int c0 = lane * CPL;
+  const float inv_cz = 1.0f / a.cz;
   float wb[CPL][HM];
   load_wb<CPL, HM>(a, c0, wb);
   float g[CPL], bt[CPL];
@@ -127,39 +178,63 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 4 : 2) ln_fwd_kernel(ProjArgs 
     g[e] = a.gamma[c0 + e];
     bt[e] = a.beta[c0 + e];
   }
-  const int64_t groups = (a.rows + kRowsPerWarp - 1) / kRowsPerWarp;
-  for (int64_t grp = first_group(); grp < groups; grp += group_stride()) {
-    const int64_t r0 = grp * kRowsPerWarp;
-    float v[kRowsPerWarp][CPL];
+  const int64_t groups = (a.rows + R - 1) / R;
+  int64_t grp = first_group();
+  uint32_t raw[R][CPL / 2];
+  if (grp < groups) load_group<CPL, R>(a.z, a.rows, a.cz, grp * R, c0, raw);
+  for (; grp < groups; grp += group_stride()) {
+    const int64_t r0 = grp * R;
+    float v[R][CPL];
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r)
-      if (r0 + r < a.rows) load_row<CPL>(a.z + (r0 + r) * a.cz + c0, v[r]);
+    for (int r = 0; r < R; ++r) unpack<CPL>(raw[r], v[r]);
+    if (grp + group_stride() < groups)
+      load_group<CPL, R>(a.z, a.rows, a.cz, (grp + group_stride()) * R, c0, raw);
+    float t[R], mean[R], rstd[R];
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-      const int64_t row = r0 + r;
-      if (row >= a.rows) break;                    // warp-uniform
-      float s = 0.0f;
+    for (int r = 0; r < R; ++r) {
+      t[r] = 0.0f;
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) s += v[r][e];
-      const float mean = warp_sum(s) / a.cz;
-      float q = 0.0f;
+      for (int e = 0; e < CPL; ++e) t[r] += v[r][e];
+    }
+    float tot = reduce_scatter<R>(t, lane);
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) q += (v[r][e] - mean) * (v[r][e] - mean);
-      const float rstd = rsqrtf(warp_sum(q) / a.cz + a.eps);
+    for (int r = 0; r < R; ++r) mean[r] = __shfl_sync(0xffffffffu, tot, r << (5 - ilog2(R))) * inv_cz;
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) v[r][e] = bf16_round((v[r][e] - mean) * rstd * g[e] + bt[e]);
-      store_row<CPL>(a.x + row * a.cz + c0, v[r]);
-      if (lane == 0) reinterpret_cast<float2 *>(a.stats)[row] = make_float2(mean, rstd);
+    for (int r = 0; r < R; ++r) {
+      t[r] = 0.0f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) t[r] += (v[r][e] - mean[r]) * (v[r][e] - mean[r]);
+    }
+    tot = reduce_scatter<R>(t, lane);
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      rstd[r] = rsqrtf(__shfl_sync(0xffffffffu, tot, r << (5 - ilog2(R))) * inv_cz + a.eps);
+    float sm = 0.0f, sr = 0.0f;                    // lane r < R writes row r's statistics
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) v[r][e] = bf16_round((v[r][e] - mean[r]) * rstd[r] * g[e] + bt[e]);
+      if (r0 + r < a.rows) store_row<CPL>(a.x + (r0 + r) * a.cz + c0, v[r]);
+      if (lane == r) sm = mean[r], sr = rstd[r];
+    }
+    if (lane < R && r0 + lane < a.rows)
+      reinterpret_cast<float2 *>(a.stats)[r0 + lane] = make_float2(sm, sr);
+    float d[R * HM];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
 #pragma unroll
       for (int h = 0; h < HM; ++h) {
-        if (h >= a.H) break;
-        float d = 0.0f;
+        float acc = 0.0f;
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) d += v[r][e] * wb[e][h];
-        d = warp_sum(d);
-        if (lane == 0) a.bias[bias_base(a, row) + h * a.rows_per] = __float2bfloat16_rn(d);
+        for (int e = 0; e < CPL; ++e) acc += v[r][e] * wb[e][h];
+        d[r * HM + h] = acc;
       }
-    }
+    // lane l holds the total of (row, head) number l >> (5 - log2(R HM))
+    constexpr int kShift = 5 - ilog2(R * HM);
+    const float bsum = reduce_scatter<R * HM>(d, lane);
+    const int idx = lane >> kShift, r = idx / HM, h = idx % HM;
+    if ((lane & ((1 << kShift) - 1)) == 0 && h < a.H && r0 + r < a.rows)
+      a.bias[bias_base(a, r0 + r) + h * a.rows_per] = __float2bfloat16_rn(bsum);
   }
 }
 
@@ -167,12 +242,14 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 4 : 2) ln_fwd_kernel(ProjArgs 
 // sum_h dbias[h][row] w_b[c][h]; partial sums of dgamma, dbeta and
 // dw_b[c][h] = sum_rows x[c] dbias[h][row] (x as the forward stored it), one
 // set per block: each warp accumulates its rows, then the block's warps are
-// added in warp order.
-template <int CPL, int HM>
+// added in warp order. RPW rows at a time, the next group's inputs loaded
+// while the current one is worked on.
+template <int CPL, int HM, int RPW>
 __global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs a) {
   __shared__ float acc[256 * (2 + kMaxHeads)];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = lane * CPL;
+  const float inv_cz = 1.0f / a.cz;
   float wb[CPL][HM];
   load_wb<CPL, HM>(a, c0, wb);
   float g[CPL], dg[CPL], db[CPL], dwb[CPL][HM];
@@ -183,49 +260,80 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs 
 #pragma unroll
     for (int h = 0; h < HM; ++h) dwb[e][h] = 0.0f;
   }
-  const int64_t groups = (a.rows + kRowsPerWarp - 1) / kRowsPerWarp;
-  for (int64_t grp = first_group(); grp < groups; grp += group_stride()) {
-    const int64_t r0 = grp * kRowsPerWarp;
-    float z[kRowsPerWarp][CPL], dx[kRowsPerWarp][CPL];
+  const int64_t groups = (a.rows + RPW - 1) / RPW;
+  int64_t grp = first_group();
+  uint32_t zr[RPW][CPL / 2], xr[RPW][CPL / 2];
+  float dx[RPW][CPL], dbh[RPW][HM];
+  float2 st[RPW];
+  auto load = [&](int64_t r0) {
+    load_group<CPL, RPW>(a.z, a.rows, a.cz, r0, c0, zr);
+    load_group<CPL, RPW>(a.x, a.rows, a.cz, r0, c0, xr);
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r)
-      if (r0 + r < a.rows) {
-        load_row<CPL>(a.z + (r0 + r) * a.cz + c0, z[r]);
-        load_row_f32<CPL>(a.dx + (r0 + r) * a.cz + c0, dx[r]);
-      }
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
+    for (int r = 0; r < RPW; ++r) {
       const int64_t row = r0 + r;
-      if (row >= a.rows) break;                    // warp-uniform
-      float x[CPL];
-      load_row<CPL>(a.x + row * a.cz + c0, x);
-      const float2 st = reinterpret_cast<const float2 *>(a.stats)[row];
-      const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
+      if (row < a.rows) {
+        load_row_f32<CPL>(a.dx + row * a.cz + c0, dx[r]);
+        st[r] = reinterpret_cast<const float2 *>(a.stats)[row];
+        const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
 #pragma unroll
-      for (int h = 0; h < HM; ++h) {
-        if (h >= a.H) break;
-        const float dbh = __bfloat162float(dbias[h * a.rows_per]);
+        for (int h = 0; h < HM; ++h)
+          dbh[r][h] = h < a.H ? __bfloat162float(dbias[h * a.rows_per]) : 0.0f;
+      } else {
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-          dx[r][e] += dbh * wb[e][h];
-          dwb[e][h] += x[e] * dbh;
-        }
+        for (int e = 0; e < CPL; ++e) dx[r][e] = 0.0f;
+        st[r] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int h = 0; h < HM; ++h) dbh[r][h] = 0.0f;
       }
-      float s1 = 0.0f, s2 = 0.0f;
+    }
+  };
+  if (grp < groups) load(grp * RPW);
+  for (; grp < groups; grp += group_stride()) {
+    const int64_t r0 = grp * RPW;
+    float xh[RPW][CPL], u[RPW][CPL], s[2 * RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      float z[CPL], x[CPL];
+      unpack<CPL>(zr[r], z);
+      unpack<CPL>(xr[r], x);
 #pragma unroll
       for (int e = 0; e < CPL; ++e) {
-        const float xh = (z[r][e] - st.x) * st.y;
-        z[r][e] = xh;
-        dg[e] += dx[r][e] * xh;
-        db[e] += dx[r][e];
-        const float gx = dx[r][e] * g[e];
-        s1 += gx;
-        s2 += gx * xh;
-      }
-      const float m1 = warp_sum(s1) / a.cz, m2 = warp_sum(s2) / a.cz;
+        float d = dx[r][e];
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) z[r][e] = st.y * (dx[r][e] * g[e] - m1 - z[r][e] * m2);
-      store_row<CPL>(a.dz + row * a.cz + c0, z[r]);
+        for (int h = 0; h < HM; ++h) {
+          d += dbh[r][h] * wb[e][h];
+          dwb[e][h] += x[e] * dbh[r][h];
+        }
+        xh[r][e] = (z[e] - st[r].x) * st[r].y;
+        u[r][e] = d;
+      }
+    }
+    float rstd[RPW];
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) rstd[r] = st[r].y;
+    if (grp + group_stride() < groups) load((grp + group_stride()) * RPW);
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      s[r] = s[RPW + r] = 0.0f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) {
+        dg[e] += u[r][e] * xh[r][e];
+        db[e] += u[r][e];
+        u[r][e] *= g[e];                           // dL/dxhat
+        s[r] += u[r][e];
+        s[RPW + r] += u[r][e] * xh[r][e];
+      }
+    }
+    constexpr int kShift = 5 - ilog2(2 * RPW);
+    const float tot = reduce_scatter<2 * RPW>(s, lane);
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float m1 = __shfl_sync(0xffffffffu, tot, r << kShift) * inv_cz;
+      const float m2 = __shfl_sync(0xffffffffu, tot, (RPW + r) << kShift) * inv_cz;
+      float dz[CPL];
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) dz[e] = rstd[r] * (u[r][e] - m1 - xh[r][e] * m2);
+      if (r0 + r < a.rows) store_row<CPL>(a.dz + (r0 + r) * a.cz + c0, dz);
     }
   }
   // block partials [dgamma cz | dbeta cz | dw_b cz*H], warps added in order
@@ -348,10 +456,10 @@ cudaError_t launch_ln_bwd_h(const ProjArgs &a, cudaStream_t stream) {
   const int blocks = kProjBlocks;
   if (a.cz % 64) return cudaErrorInvalidValue;
   switch (a.cz / 32) {
-    case 2: ln_bwd_kernel<2, HM><<<blocks, 256, 0, stream>>>(a); break;
-    case 4: ln_bwd_kernel<4, HM><<<blocks, 256, 0, stream>>>(a); break;
-    case 6: ln_bwd_kernel<6, HM><<<blocks, 256, 0, stream>>>(a); break;
-    case 8: ln_bwd_kernel<8, HM><<<blocks, 256, 0, stream>>>(a); break;
+    case 2: ln_bwd_kernel<2, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
+    case 4: ln_bwd_kernel<4, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
+    case 6: ln_bwd_kernel<6, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
+    case 8: ln_bwd_kernel<8, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
