@@ -9,15 +9,19 @@
 // attention (LayerNorm output times the projection weights, and their
 // gradients, the weight gradients as split-K batches of fp32 partial sums).
 //
-// One CTA computes one 128x256 tile of one batch (fp32 in tensor memory):
-//   warp 0      TMA producer: 64-wide K slices of X and Y (48 KB), 2-stage ring
+// Persistent: one CTA per SM walks the 128x256 output tiles (n fastest, then
+// m, then the batch), so the tiles in flight at any moment are neighbours that
+// share operands in L2. Two accumulators in tensor memory (2 x 256 columns):
+// the epilogue of one tile overlaps the main loop of the next.
+//   warp 0      TMA producer: 64-wide K slices of X and Y (48 KB), 3-stage ring
+//               running across tiles
 //   warp 1      tensor-memory allocator and MMA issuer (N = 256 products)
-//   warps 2..5  epilogue: tensor memory -> bf16 or fp32 -> the idle stage
-//               buffers -> TMA stores (bf16: 64-column boxes, each routed to one
-//               of up to four output tensors by its column; fp32: 32-column
-//               boxes)
-// 96 KB of shared memory and 256 tensor-memory columns, so two CTAs share an
-// SM and one's epilogue overlaps the other's main loop.
+//   warps 2..9  epilogue, two per accumulator lane quarter (each half of the
+//               columns): tensor memory -> bf16 or fp32 (32-column loads, the
+//               next one in flight while the current one is converted) -> a
+//               2-box staging ring per warp -> TMA stores (bf16: 64-column
+//               boxes, each routed to one of up to four output tensors by its
+//               column; fp32: 32-column boxes)
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,28 +35,30 @@ namespace {
 
 constexpr int kTM = 128, kTK = 64;
 constexpr int kTN = 256;                               // output tile 128 x kTN
-constexpr int kStages = 2;
-constexpr int kMinBlocks = 2;                          // CTAs per SM the budget is sized for
-constexpr int kThreads = 192;
-constexpr uint32_t kTmemCols = kTN;
+constexpr int kStages = 3;
+constexpr int kEpiWarps = 8;                           // two per accumulator lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr uint32_t kTmemCols = 2 * kTN;                // two accumulators
 constexpr uint32_t kXBytes = kTM * kTK * 2;            // 16 KB X slice
 constexpr uint32_t kYBytes = kTN * kTK * 2;            // Y slice
 constexpr uint32_t kStageBytes = kXBytes + kYBytes;
-constexpr uint32_t kOffCtl = kStages * kStageBytes;
 constexpr uint32_t kAtomBytes = 64 * kTK * 2;          // one 64-wide MN atom column: 8 KB
-constexpr uint32_t kWarpStage = 16 * 1024;             // epilogue staging per warp
-static_assert(32 * kTN * 2 <= kWarpStage, "a warp's bf16 rows must fit its staging");
-static_assert(4 * kWarpStage <= kStages * kStageBytes, "staging reuses the operand stages");
+constexpr uint32_t kBoxBytes = 32 * 128;               // staged output box: 32 rows x 128 B
+constexpr int kRing = 2;                               // staged boxes per epilogue warp
+constexpr uint32_t kOffStaging = kStages * kStageBytes;
+constexpr uint32_t kOffCtl = kOffStaging + kEpiWarps * kRing * kBoxBytes;
 
-struct __align__(8) MulSmem {
+struct __align__(8) GemmSmem {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t acc_full;
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
   uint64_t teardown;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
-constexpr uint32_t kSmemBytes = kOffCtl + sizeof(MulSmem) + 1024;   // +1024 for alignment
+constexpr uint32_t kSmemBytes = kOffCtl + sizeof(GemmSmem) + 1024;  // +1024 for alignment
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
                                          volatile uint32_t *abort_flag, int32_t *status) {
@@ -112,30 +118,114 @@ __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
             : make_sdesc(base + ks * 32, 16, 1024, kSwizzle128B);
 }
 
+// Tile t of the walk: n fastest, then m, then the batch index.
+struct Tile {
+  int m0, n0, c;
+};
+__device__ __forceinline__ Tile tile_of(int t, int mt, int nt) {
+  return {((t / nt) % mt) * kTM, (t % nt) * kTN, t / (nt * mt)};
+}
+
+// K range of batch index c: split-K takes K columns [kbeg, kend) of operands
+// that have no batch dimension of their own (their batch coordinate is 0);
+// otherwise c is every tensor's batch coordinate.
+struct KRange {
+  int kbeg, nk, cin;
+};
+__device__ __forceinline__ KRange k_range(const GemmArgs &a, int c) {
+  const int kbeg = a.k_split ? c * a.k_split : 0;
+  const int kend = a.k_split ? min(a.K, kbeg + a.k_split) : a.K;
+  return {kbeg, (kend - kbeg + kTK - 1) / kTK, a.k_split ? 0 : c};
+}
+
+// One 32-column chunk of a warp's 32 accumulator rows -> its staging box; a
+// finished box goes out by TMA. bf16: two chunks fill a 64-column box; fp32:
+// one chunk is a box. Every box commits one bulk group (empty when the box
+// lies past the last output), so the ring's bulk_wait_read count is exact.
+template <bool F32>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, const Tile &tl,
+                                               int q4, int lane, uint8_t *ring, uint32_t &nbox,
+                                               const GemmOuts &outs, const GemmArgs &a) {
+  const bool first_half = F32 || (cb & 1) == 0;
+  uint8_t *box = ring + (nbox % kRing) * kBoxBytes;
+  if (first_half && nbox >= (uint32_t)kRing) {
+    if (lane == 0) bulk_wait_read<kRing - 1>();      // the store from this slot has read it
+    __syncwarp();
+  }
+  if (F32) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      *reinterpret_cast<uint4 *>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+          make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else {
+    float f[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+    const int col0 = tl.n0 + cb * 32;
+    if (a.col_bias && col0 + 32 > a.col_bias_from) {
+      if (col0 >= a.col_bias_from && col0 + 32 <= a.Nn) {
+        // the whole chunk takes the bias: the same 32 floats for every lane
+        const float4 *pb = reinterpret_cast<const float4 *>(a.col_bias + (col0 - a.col_bias_from));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 b = __ldg(pb + q);
+          f[4 * q] += b.x, f[4 * q + 1] += b.y, f[4 * q + 2] += b.z, f[4 * q + 3] += b.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = col0 + e;
+          if (col >= a.col_bias_from && col < a.Nn) f[e] += a.col_bias[col - a.col_bias_from];
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int chunk = (cb & 1) * 4 + q;             // 16-byte chunk of the 128-byte row
+      *reinterpret_cast<uint4 *>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
+          make_uint4(pack_bf16(f[8 * q], f[8 * q + 1]), pack_bf16(f[8 * q + 2], f[8 * q + 3]),
+                     pack_bf16(f[8 * q + 4], f[8 * q + 5]), pack_bf16(f[8 * q + 6], f[8 * q + 7]));
+    }
+  }
+  if (F32 || (cb & 1)) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      if (F32) {
+        tma_store_3d(&outs.map[0], box, tl.n0 + cb * 32, tl.m0 + q4 * 32, tl.c);
+      } else {
+        const int n = tl.n0 + (cb >> 1) * 64;          // first column of the box
+        const int o = n / a.cols_per_out;               // the output tensor it belongs to
+        if (o < a.nouts) tma_store_3d(&outs.map[o], box, n - o * a.cols_per_out, tl.m0 + q4 * 32, tl.c);
+      }
+      bulk_commit_group();
+    }
+    ++nbox;
+  }
+}
+
 template <bool XMN, bool YMN, bool F32>
-__global__ void __launch_bounds__(kThreads, kMinBlocks)
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ GemmMaps ys,
                const __grid_constant__ GemmOuts outs, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  MulSmem &ctl = *reinterpret_cast<MulSmem *>(smem + kOffCtl);
+  GemmSmem &ctl = *reinterpret_cast<GemmSmem *>(smem + kOffCtl);
   volatile uint32_t *abort_flag = &ctl.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kTM, n0 = blockIdx.y * kTN, c = blockIdx.z;
-  // split-K: batch index c takes K columns [kbeg, kend) of operands that have no
-  // batch dimension of their own; otherwise c is every tensor's batch coordinate
-  const int kbeg = a.k_split ? c * a.k_split : 0;
-  const int kend = a.k_split ? min(a.K, kbeg + a.k_split) : a.K;
-  const int cin = a.k_split ? 0 : c;
-  const int nk = (kend - kbeg + kTK - 1) / kTK;
+  const int mt = (a.M + kTM - 1) / kTM, nt = (a.Nn + kTN - 1) / kTN;
+  const int tiles = mt * nt * a.batch;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
-    mbar_init(&ctl.acc_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl.acc_full[b], 1);
+      mbar_init(&ctl.acc_empty[b], kEpiWarps);       // one arrival per epilogue warp
+    }
     mbar_init(&ctl.teardown, 1);
     ctl.abort_flag = 0u;
     fence_barrier_init();
@@ -154,127 +244,114 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
     if (elect_one()) {
       tma_prefetch_desc(&xs.map[0]);
       tma_prefetch_desc(&ys.map[0]);
-      int armed[kStages];
-      for (int s = 0; s < kStages; ++s) armed[s] = -1;
+      uint32_t it = 0;                                // K slices issued, over all tiles
       bool ok = true;
-      for (int kt = 0; kt < nk; ++kt) {
-        const int st = kt % kStages;
-        if (kt >= kStages &&
-            !wait_bar(&ctl.empty[st], ((kt / kStages) - 1) & 1, abort_flag, a.status)) {
-          ok = false;
-          break;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const Tile tl = tile_of(t, mt, nt);
+        const KRange kr = k_range(a, tl.c);
+        for (int kt = 0; kt < kr.nk; ++kt, ++it) {
+          const int st = it % kStages;
+          if (it >= (uint32_t)kStages &&
+              !wait_bar(&ctl.empty[st], ((it / kStages) - 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t *dst = smem + st * kStageBytes;
+          mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
+          const int k = kr.kbeg + kt * kTK;
+          const int xi = k / a.k_per_x;                // the X tensor holding this K slice
+          load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], tl.m0, k - xi * a.k_per_x, kr.cin);
+          if (a.n_per_y)
+            load_y_slice<YMN>(dst + kXBytes, ys, a, &ctl.full[st], tl.n0, k, kr.cin);
+          else
+            load_slice<YMN, kTN>(dst + kXBytes, &ys.map[0], &ctl.full[st], tl.n0, k, kr.cin);
         }
-        uint8_t *dst = smem + st * kStageBytes;
-        mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
-        const int k = kbeg + kt * kTK;
-        const int xi = k / a.k_per_x;                  // the X tensor holding this K slice
-        load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], m0, k - xi * a.k_per_x, cin);
-        if (a.n_per_y)
-          load_y_slice<YMN>(dst + kXBytes, ys, a, &ctl.full[st], n0, k, cin);
-        else
-          load_slice<YMN, kTN>(dst + kXBytes, &ys.map[0], &ctl.full[st], n0, k, cin);
-        armed[st] = kt / kStages;
       }
-      if (!ok)
-        for (int s = 0; s < kStages; ++s)
-          if (armed[s] >= 0) mbar_wait(&ctl.full[s], armed[s] & 1);
+      if (!ok)      // let the copies already issued land before the CTA exits
+        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
+          mbar_wait(&ctl.full[j % kStages], (j / kStages) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer --
     if (elect_one()) {
       const uint32_t idesc = make_idesc_bf16(kTM, kTN, XMN, YMN);
+      uint32_t it = 0;
       bool ok = true;
-      for (int kt = 0; kt < nk && ok; ++kt) {
-        const int st = kt % kStages;
-        if (!wait_bar(&ctl.full[st], (kt / kStages) & 1, abort_flag, a.status)) {
+      int j = 0;                                      // tiles of this CTA
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
+        const int buf = j & 1;
+        if (j >= 2 &&
+            !wait_bar(&ctl.acc_empty[buf], ((j >> 1) - 1) & 1, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t xa = smem_u32(smem + st * kStageBytes);
-        const uint32_t ya = xa + kXBytes;
+        const uint32_t d = tmem + buf * kTN;
+        const KRange kr = k_range(a, tile_of(t, mt, nt).c);
+        for (int kt = 0; kt < kr.nk; ++kt, ++it) {
+          const int st = it % kStages;
+          if (!wait_bar(&ctl.full[st], (it / kStages) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + st * kStageBytes);
+          const uint32_t ya = xa + kXBytes;
 #pragma unroll
-        for (int ks = 0; ks < kTK / 16; ++ks)
-          mma_ss(tmem, slice_desc<XMN>(xa, ks), slice_desc<YMN>(ya, ks), idesc,
-                 (kt > 0 || ks > 0) ? 1u : 0u);
-        mma_commit(&ctl.empty[st]);
+          for (int ks = 0; ks < kTK / 16; ++ks)
+            mma_ss(d, slice_desc<XMN>(xa, ks), slice_desc<YMN>(ya, ks), idesc,
+                   (kt > 0 || ks > 0) ? 1u : 0u);
+          mma_commit(&ctl.empty[st]);
+        }
+        if (ok) mma_commit(&ctl.acc_full[buf]);
       }
-      mma_commit(&ctl.acc_full);
       // No tensor-memory operation may be in flight when the CTA tears down.
       mma_commit(&ctl.teardown);
       mbar_wait(&ctl.teardown, 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue --
-    const int q4 = warp & 3;
-    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-    bool ok = true;
-    if (!mbar_try_wait(&ctl.acc_full, 0)) ok = wait_bar(&ctl.acc_full, 0, abort_flag, a.status);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    // Warp w reads accumulator lanes 32 (w % 4) .. + 31 (its rank in the
+    // warpgroup); the first four epilogue warps take columns 0..127 of the tile,
+    // the other four columns 128..255. Chunks past the output's last column
+    // (rounded up to a whole box) are skipped.
+    const int e = warp - 2, q4 = warp & 3, half = e >> 2;
+    uint8_t *ring = smem + kOffStaging + e * kRing * kBoxBytes;
+    uint32_t nbox = 0;
+    int j = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
+      const int buf = j & 1;
+      bool ok = mbar_try_wait(&ctl.acc_full[buf], (j >> 1) & 1) ||
+                wait_bar(&ctl.acc_full[buf], (j >> 1) & 1, abort_flag, a.status);
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      // The operand stages are idle once the accumulator is complete: each warp
-      // stages its 32 rows there (boxes of 32 rows x 128 bytes, 128-byte
-      // swizzle) and stores them with TMA, which clips rows and columns past the
-      // output's extent.
-      // 16 KB per warp: the four 64-column bf16 boxes of its rows, or a ring of
-      // four 32-column fp32 boxes whose slot is reused once its store has read it
-      uint8_t *stage = smem + q4 * kWarpStage;
+      const Tile tl = tile_of(t, mt, nt);
+      const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kTN;
+      const int cols = a.Nn - tl.n0;                   // output columns in this tile
+      const int live = F32 ? (cols + 31) / 32 : 2 * ((cols + 63) / 64);
+      const int cb0 = half * (kTN / 64), cb1 = min(cb0 + kTN / 64, live);
+      if (cb0 < cb1) {
+        uint32_t va[32], vb[32];
+        tmem_ld32_issue(ta + cb0 * 32, va);
+        tmem_wait_ld32(va);
 #pragma unroll 1
-      for (int cb = 0; cb < kTN / 32; ++cb) {
-        uint32_t v[32];
-        tmem_ld32(tl + cb * 32, v);
-        if (F32) {
-          // 32 fp32 columns = one 128-byte row of a box
-          uint8_t *box = stage + (cb & 3) * (32 * 128);
-          if (cb >= 4) {
-            if (lane == 0) bulk_wait_read<3>();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<uint4 *>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) =
-                make_uint4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&outs.map[0], box, n0 + cb * 32, m0 + q4 * 32, c);
-            bulk_commit_group();
-          }
-        } else {
-          uint8_t *box = stage + (cb >> 1) * (32 * 128);
-          if (a.col_bias) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int col = n0 + cb * 32 + e;
-              if (col >= a.col_bias_from && col < a.Nn)
-                v[e] = __float_as_uint(__uint_as_float(v[e]) + a.col_bias[col - a.col_bias_from]);
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int chunk = (cb & 1) * 4 + q;       // 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4 *>(box + lane * 128 + ((chunk ^ (lane & 7)) << 4)) =
-                make_uint4(pack_bf16(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
-                           pack_bf16(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
-                           pack_bf16(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
-                           pack_bf16(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
-          }
-          if (cb & 1) {
-            fence_proxy_async_smem();
-            __syncwarp();
-            const int n = n0 + (cb >> 1) * 64;        // first column of the box
-            const int o = n / a.cols_per_out;          // the output tensor it belongs to
-            if (lane == 0 && o < a.nouts) {
-              tma_store_3d(&outs.map[o], box, n - o * a.cols_per_out, m0 + q4 * 32, c);
-              bulk_commit_group();
-            }
-          }
+        for (int cb = cb0; cb < cb1; cb += 2) {
+          const bool has_b = cb + 1 < cb1, has_a = cb + 2 < cb1;
+          if (has_b) tmem_ld32_issue(ta + (cb + 1) * 32, vb);
+          epilogue_chunk<F32>(va, cb, tl, q4, lane, ring, nbox, outs, a);
+          if (has_b) tmem_wait_ld32(vb);
+          if (has_a) tmem_ld32_issue(ta + (cb + 2) * 32, va);
+          if (has_b) epilogue_chunk<F32>(vb, cb + 1, tl, q4, lane, ring, nbox, outs, a);
+          if (has_a) tmem_wait_ld32(va);
         }
       }
-      if (lane == 0) bulk_wait_all();
+      // every load of this accumulator is done: hand it back to the MMA warp
+      tc_fence_before();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.acc_empty[buf]);
     }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -292,7 +369,14 @@ cudaError_t launch(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
   cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((args.M + kTM - 1) / kTM, (args.Nn + kTN - 1) / kTN, args.batch);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  const int64_t tiles = (int64_t)((args.M + kTM - 1) / kTM) * ((args.Nn + kTN - 1) / kTN) *
+                        args.batch;
+  if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  const int grid = (int)(tiles < sms ? tiles : sms);
   gemm_tc_kernel<XMN, YMN, F32><<<grid, kThreads, kSmemBytes, stream>>>(x, y, d, args);
   return cudaGetLastError();
 }

@@ -363,6 +363,31 @@ __device__ __forceinline__ void tmem_ld8x2_issue(uint32_t ta, uint32_t tb, uint3
       : "memory");
 }
 
+// 32 columns left in flight: the registers must not be read before
+// tmem_wait_ld32 on the same array, which ties them to the wait.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : TRI_R8(0), TRI_R8(8), TRI_R8(16), TRI_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+
+#define TRI_U8(b) "+r"(r[b + 0]), "+r"(r[b + 1]), "+r"(r[b + 2]), "+r"(r[b + 3]), \
+    "+r"(r[b + 4]), "+r"(r[b + 5]), "+r"(r[b + 6]), "+r"(r[b + 7])
+
+// Waits for every tensor-memory load of this thread; r (the array loaded last)
+// is an in-out operand, so no use of it moves above the wait.
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : TRI_U8(0), TRI_U8(8), TRI_U8(16), TRI_U8(24)
+               :
+               : "memory");
+}
+
+#undef TRI_U8
+
 #define TRI_UA8(b) "+r"(a[b + 0]), "+r"(a[b + 1]), "+r"(a[b + 2]), "+r"(a[b + 3]), \
     "+r"(a[b + 4]), "+r"(a[b + 5]), "+r"(a[b + 6]), "+r"(a[b + 7])
 #define TRI_UB8(b) "+r"(b_[b + 0]), "+r"(b_[b + 1]), "+r"(b_[b + 2]), "+r"(b_[b + 3]), \
