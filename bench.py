@@ -677,15 +677,97 @@ def run_block(args, rank, world, local):
             "clocks": clk, "gpu_launches": sum(launches.values()) * args.steps}
 
 
+PROJ_METRIC = ("LayerNorm + projection stages fwd+bwd GB/s (algorithmic HBM bytes) at N=768, "
+               "cz=128, H=4, c=32 bf16")
+
+
+def run_proj(args, rank, world, local):
+    """One step: the four projection calls around the attention (input side
+    forward and backward, output side forward and backward) at N=768, cz=128,
+    H=4, c=32, without the attention itself. HBM-bound work: the value is the
+    algorithmic bytes of the four stages over the step time."""
+    import triangle_attention_b200 as ta
+    N, cz, H, c = 768, 128, 4, 32
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = tri_inputs.make_block_inputs(N, cz, H, c, None, seed=11 + rank)
+    g = {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in d.items()}
+    stream = torch.cuda.current_stream()
+    ws = ta.workspace(ta.proj_workspace_size(ta.proj_problem(g["z"], H, c)), dev)
+    outs = ta.proj_in_fwd(g["z"], g["gamma"], g["beta"], g["w_qkvg"], g["b_g"], g["w_b"], ws=ws)
+    ig = ta.proj_in_bwd(g["z"], g["gamma"], g["w_qkvg"], g["w_b"], outs[0], outs[1], g["dq"],
+                        g["dk"], g["dv"], g["dg"], g["dbias"], ws=ws)
+    o = g["dq"]                                   # stands in for the attention output
+    y = ta.proj_out_fwd(o, g["w_o"], g["b_o"], ws=ws)
+    og = ta.proj_out_bwd(o, g["w_o"], g["dy"], ws=ws)
+    stages = {
+        "proj_in_fwd": lambda: ta.proj_in_fwd(g["z"], g["gamma"], g["beta"], g["w_qkvg"],
+                                              g["b_g"], g["w_b"], outs=outs, ws=ws),
+        "proj_in_bwd": lambda: ta.proj_in_bwd(g["z"], g["gamma"], g["w_qkvg"], g["w_b"], outs[0],
+                                              outs[1], g["dq"], g["dk"], g["dv"], g["dg"],
+                                              g["dbias"], grads=ig, ws=ws),
+        "proj_out_fwd": lambda: ta.proj_out_fwd(o, g["w_o"], g["b_o"], y=y, ws=ws),
+        "proj_out_bwd": lambda: ta.proj_out_bwd(o, g["w_o"], g["dy"], grads=og, ws=ws),
+    }
+    names = list(stages)
+    for _ in range(args.warmup):
+        for n in names:
+            stages[n]()
+    torch.cuda.synchronize()
+    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
+    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark()
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in names]
+          for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        for j, n in enumerate(names):
+            ev[i][j][0].record(stream)
+            stages[n]()
+            ev[i][j][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if ta.read_status(ws):
+        raise RuntimeError("device status set in the timed region")
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+    stage_ms = {n: float(np.median([ev[i][j][0].elapsed_time(ev[i][j][1])
+                                    for i in range(args.steps)])) for j, n in enumerate(names)}
+    by = block_bytes(N, cz, H, c)
+    peaks = load_peaks()
+    gbs = {n: by[n] / (stage_ms[n] * 1e-3) / 1e9 for n in names}
+    top = max(names, key=lambda n: stage_ms[n])
+    return {"metric": PROJ_METRIC, "value": world * sum(by.values()) / (ms * 1e-3) / 1e9,
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded, tri_inputs.make_block_inputs)",
+            "config": {"workload": "proj_n768_cz128", "N": N, "cz": cz, "H": H, "c": c,
+                       "l2": "inputs larger than L2 (z 151 MB, q/k/v/g 151 MB each)",
+                       "parallelism": "independent replica per GPU"},
+            "stage_ms": stage_ms, "stage_gbs": gbs,
+            "roofline": {"bound": "hbm", "kernel": top, "achieved": gbs[top],
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs[top] / peaks["hbm_gbs"], "traffic": None,
+                         "note": "algorithmic bytes of the whole stage over its event time"},
+            "clocks": clk, "gpu_launches": 17 * args.steps}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[1])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["attention", "trimul", "block"], default="attention",
-                    help="attention (the default line), the triangle multiplication, or the "
-                         "whole block around the attention")
+    ap.add_argument("--op", choices=["attention", "trimul", "block", "proj"],
+                    default="attention",
+                    help="attention (the default line), the triangle multiplication, the "
+                         "whole block around the attention, or its projection stages alone")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget-s", type=float, default=150.0,
@@ -711,6 +793,8 @@ def main():
             line = run_trimul(args, rank, world, local)
         elif args.op == "block":
             line = run_block(args, rank, world, local)
+        elif args.op == "proj":
+            line = run_proj(args, rank, world, local)
         else:
             line = run_ours(args, rank, world, local, w)
         if rank == 0:

@@ -35,7 +35,7 @@ namespace {
 
 constexpr int kTM = 128, kTK = 64;
 constexpr int kTN = 256;                               // output tile 128 x kTN
-constexpr int kStages = 3;
+constexpr int kMaxStages = 4;
 constexpr int kEpiWarps = 8;                           // two per accumulator lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 2 * kTN;                // two accumulators
@@ -44,21 +44,33 @@ constexpr uint32_t kYBytes = kTN * kTK * 2;            // Y slice
 constexpr uint32_t kStageBytes = kXBytes + kYBytes;
 constexpr uint32_t kAtomBytes = 64 * kTK * 2;          // one 64-wide MN atom column: 8 KB
 constexpr uint32_t kBoxBytes = 32 * 128;               // staged output box: 32 rows x 128 B
-constexpr int kRing = 2;                               // staged boxes per epilogue warp
-constexpr uint32_t kOffStaging = kStages * kStageBytes;
-constexpr uint32_t kOffCtl = kOffStaging + kEpiWarps * kRing * kBoxBytes;
+
+// Two shapes of the pipeline. Long K (8 or more slices per tile): 4 operand
+// stages, the latency of the loads is what limits the main loop, and one
+// staged box per epilogue warp is enough because the epilogue hides behind it.
+// Short K (the projections): 3 stages and 2 boxes per warp, the epilogue is
+// the longer part of a tile.
+template <int STAGES, int RING>
+struct Pipe {
+  static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
+  static constexpr uint32_t kOffCtl = kOffStaging + kEpiWarps * RING * kBoxBytes;
+};
 
 struct __align__(8) GemmSmem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t teardown;
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
-constexpr uint32_t kSmemBytes = kOffCtl + sizeof(GemmSmem) + 1024;  // +1024 for alignment
-static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+template <int STAGES, int RING>
+constexpr uint32_t smem_bytes() {
+  return Pipe<STAGES, RING>::kOffCtl + sizeof(GemmSmem) + 1024;   // +1024 for alignment
+}
+static_assert(smem_bytes<4, 1>() <= 227 * 1024 && smem_bytes<3, 2>() <= 227 * 1024,
+              "shared memory budget");
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
                                          volatile uint32_t *abort_flag, int32_t *status) {
@@ -142,14 +154,14 @@ __device__ __forceinline__ KRange k_range(const GemmArgs &a, int c) {
 // finished box goes out by TMA. bf16: two chunks fill a 64-column box; fp32:
 // one chunk is a box. Every box commits one bulk group (empty when the box
 // lies past the last output), so the ring's bulk_wait_read count is exact.
-template <bool F32>
+template <bool F32, int RING>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, const Tile &tl,
                                                int q4, int lane, uint8_t *ring, uint32_t &nbox,
                                                const GemmOuts &outs, const GemmArgs &a) {
   const bool first_half = F32 || (cb & 1) == 0;
-  uint8_t *box = ring + (nbox % kRing) * kBoxBytes;
-  if (first_half && nbox >= (uint32_t)kRing) {
-    if (lane == 0) bulk_wait_read<kRing - 1>();      // the store from this slot has read it
+  uint8_t *box = ring + (nbox % RING) * kBoxBytes;
+  if (first_half && nbox >= (uint32_t)RING) {
+    if (lane == 0) bulk_wait_read<RING - 1>();       // the store from this slot has read it
     __syncwarp();
   }
   if (F32) {
@@ -204,21 +216,21 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, 
   }
 }
 
-template <bool XMN, bool YMN, bool F32>
+template <bool XMN, bool YMN, bool F32, int STAGES, int RING>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ GemmMaps ys,
                const __grid_constant__ GemmOuts outs, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  GemmSmem &ctl = *reinterpret_cast<GemmSmem *>(smem + kOffCtl);
+  GemmSmem &ctl = *reinterpret_cast<GemmSmem *>(smem + Pipe<STAGES, RING>::kOffCtl);
   volatile uint32_t *abort_flag = &ctl.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = (a.M + kTM - 1) / kTM, nt = (a.Nn + kTN - 1) / kTN;
   const int tiles = mt * nt * a.batch;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
@@ -250,9 +262,9 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
         const Tile tl = tile_of(t, mt, nt);
         const KRange kr = k_range(a, tl.c);
         for (int kt = 0; kt < kr.nk; ++kt, ++it) {
-          const int st = it % kStages;
-          if (it >= (uint32_t)kStages &&
-              !wait_bar(&ctl.empty[st], ((it / kStages) - 1) & 1, abort_flag, a.status)) {
+          const int st = it % STAGES;
+          if (it >= (uint32_t)STAGES &&
+              !wait_bar(&ctl.empty[st], ((it / STAGES) - 1) & 1, abort_flag, a.status)) {
             ok = false;
             break;
           }
@@ -268,8 +280,8 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
         }
       }
       if (!ok)      // let the copies already issued land before the CTA exits
-        for (uint32_t j = (it > (uint32_t)kStages ? it - kStages : 0u); j < it; ++j)
-          mbar_wait(&ctl.full[j % kStages], (j / kStages) & 1);
+        for (uint32_t j = (it > (uint32_t)STAGES ? it - STAGES : 0u); j < it; ++j)
+          mbar_wait(&ctl.full[j % STAGES], (j / STAGES) & 1);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer --
@@ -289,8 +301,8 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
         const uint32_t d = tmem + buf * kTN;
         const KRange kr = k_range(a, tile_of(t, mt, nt).c);
         for (int kt = 0; kt < kr.nk; ++kt, ++it) {
-          const int st = it % kStages;
-          if (!wait_bar(&ctl.full[st], (it / kStages) & 1, abort_flag, a.status)) {
+          const int st = it % STAGES;
+          if (!wait_bar(&ctl.full[st], (it / STAGES) & 1, abort_flag, a.status)) {
             ok = false;
             break;
           }
@@ -316,7 +328,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
     // the other four columns 128..255. Chunks past the output's last column
     // (rounded up to a whole box) are skipped.
     const int e = warp - 2, q4 = warp & 3, half = e >> 2;
-    uint8_t *ring = smem + kOffStaging + e * kRing * kBoxBytes;
+    uint8_t *ring = smem + Pipe<STAGES, RING>::kOffStaging + e * RING * kBoxBytes;
     uint32_t nbox = 0;
     int j = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
@@ -338,10 +350,10 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
         for (int cb = cb0; cb < cb1; cb += 2) {
           const bool has_b = cb + 1 < cb1, has_a = cb + 2 < cb1;
           if (has_b) tmem_ld32_issue(ta + (cb + 1) * 32, vb);
-          epilogue_chunk<F32>(va, cb, tl, q4, lane, ring, nbox, outs, a);
+          epilogue_chunk<F32, RING>(va, cb, tl, q4, lane, ring, nbox, outs, a);
           if (has_b) tmem_wait_ld32(vb);
           if (has_a) tmem_ld32_issue(ta + (cb + 2) * 32, va);
-          if (has_b) epilogue_chunk<F32>(vb, cb + 1, tl, q4, lane, ring, nbox, outs, a);
+          if (has_b) epilogue_chunk<F32, RING>(vb, cb + 1, tl, q4, lane, ring, nbox, outs, a);
           if (has_a) tmem_wait_ld32(va);
         }
       }
@@ -363,13 +375,22 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
   }
 }
 
+template <bool XMN, bool YMN, bool F32, int STAGES, int RING>
+cudaError_t launch_pipe(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
+                        const GemmArgs &args, int grid, cudaStream_t stream) {
+  constexpr uint32_t bytes = smem_bytes<STAGES, RING>();
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32, STAGES, RING>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<XMN, YMN, F32, STAGES, RING><<<grid, kThreads, bytes, stream>>>(x, y, d, args);
+  return cudaGetLastError();
+}
+
 template <bool XMN, bool YMN, bool F32>
 cudaError_t launch(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
                    const GemmArgs &args, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
+  cudaError_t e;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
@@ -377,8 +398,10 @@ cudaError_t launch(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
                         args.batch;
   if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  gemm_tc_kernel<XMN, YMN, F32><<<grid, kThreads, kSmemBytes, stream>>>(x, y, d, args);
-  return cudaGetLastError();
+  const int k_tile = args.k_split ? args.k_split : args.K;   // K of one tile
+  if ((k_tile + kTK - 1) / kTK >= 8)
+    return launch_pipe<XMN, YMN, F32, 4, 1>(x, y, d, args, grid, stream);
+  return launch_pipe<XMN, YMN, F32, 3, 2>(x, y, d, args, grid, stream);
 }
 
 }  // namespace
