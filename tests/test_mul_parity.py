@@ -47,7 +47,7 @@ def test_host_rejections():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("C,N", [(4, 64), (3, 136), (2, 200), (8, 256), (1, 8)])
+@pytest.mark.parametrize("C,N", [(4, 64), (3, 136), (2, 200), (8, 256), (1, 8), (1, 512), (2, 520)])
 @pytest.mark.parametrize("direction", [ta.OUTGOING, ta.INCOMING])
 def test_mul_matches_oracle(C, N, direction):
     a, b, dt = stacks(C, N, seed=N + C + direction)

@@ -33,25 +33,32 @@
 namespace tri {
 namespace {
 
-constexpr int kTM = 128, kTK = 64;
-constexpr int kTN = 256;                               // output tile 128 x kTN
+constexpr int kTM = 128, kTK = 64;                     // rows of one accumulator; K slice
+constexpr int kTN = 256;                               // output tile (128 or 256) x kTN
 constexpr int kMaxStages = 4;
 constexpr int kEpiWarps = 8;                           // two per accumulator lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr uint32_t kTmemCols = 2 * kTN;                // two accumulators
-constexpr uint32_t kXBytes = kTM * kTK * 2;            // 16 KB X slice
+constexpr uint32_t kTmemCols = 2 * kTN;                // two 128 x 256 accumulators
 constexpr uint32_t kYBytes = kTN * kTK * 2;            // Y slice
-constexpr uint32_t kStageBytes = kXBytes + kYBytes;
 constexpr uint32_t kAtomBytes = 64 * kTK * 2;          // one 64-wide MN atom column: 8 KB
 constexpr uint32_t kBoxBytes = 32 * 128;               // staged output box: 32 rows x 128 B
 
-// Two shapes of the pipeline. Long K (8 or more slices per tile): 4 operand
-// stages, the latency of the loads is what limits the main loop, and one
-// staged box per epilogue warp is enough because the epilogue hides behind it.
-// Short K (the projections): 3 stages and 2 boxes per warp, the epilogue is
-// the longer part of a tile.
-template <int STAGES, int RING>
+// Shapes of the pipeline.
+//  HALVES = 1: 128 x 256 tiles, the two accumulators hold consecutive tiles, so
+//    one tile's epilogue overlaps the next tile's main loop. Short K (the
+//    projections) takes 3 operand stages and two staged boxes per epilogue warp
+//    (the epilogue is the longer part of a tile); long K with few rows (the
+//    weight gradients) takes 4 stages and one box.
+//  HALVES = 2: 256 x 256 tiles for long K and many rows (the triangle
+//    multiplication): the two accumulators are the two 128-row halves of one
+//    tile, so a K slice of Y feeds twice the MMA work and the operand traffic
+//    per FLOP falls by a quarter; the epilogue no longer overlaps the main loop.
+template <int STAGES, int RING, int HALVES>
 struct Pipe {
+  static constexpr int kTileM = kTM * HALVES;
+  static constexpr int kBufs = HALVES == 1 ? 2 : 1;     // accumulator sets in TMEM
+  static constexpr uint32_t kXBytes = kTileM * kTK * 2;
+  static constexpr uint32_t kStageBytes = kXBytes + kYBytes;
   static constexpr uint32_t kOffStaging = STAGES * kStageBytes;
   static constexpr uint32_t kOffCtl = kOffStaging + kEpiWarps * RING * kBoxBytes;
 };
@@ -65,11 +72,12 @@ struct __align__(8) GemmSmem {
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
-template <int STAGES, int RING>
+template <int STAGES, int RING, int HALVES>
 constexpr uint32_t smem_bytes() {
-  return Pipe<STAGES, RING>::kOffCtl + sizeof(GemmSmem) + 1024;   // +1024 for alignment
+  return Pipe<STAGES, RING, HALVES>::kOffCtl + sizeof(GemmSmem) + 1024;   // +1024: alignment
 }
-static_assert(smem_bytes<4, 1>() <= 227 * 1024 && smem_bytes<3, 2>() <= 227 * 1024,
+static_assert(smem_bytes<4, 1, 1>() <= 227 * 1024 && smem_bytes<3, 2, 1>() <= 227 * 1024 &&
+              smem_bytes<3, 1, 2>() <= 227 * 1024,
               "shared memory budget");
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity,
@@ -134,8 +142,8 @@ __device__ __forceinline__ uint64_t slice_desc(uint32_t base, int ks) {
 struct Tile {
   int m0, n0, c;
 };
-__device__ __forceinline__ Tile tile_of(int t, int mt, int nt) {
-  return {((t / nt) % mt) * kTM, (t % nt) * kTN, t / (nt * mt)};
+__device__ __forceinline__ Tile tile_of(int t, int mt, int nt, int tile_m) {
+  return {((t / nt) % mt) * tile_m, (t % nt) * kTN, t / (nt * mt)};
 }
 
 // K range of batch index c: split-K takes K columns [kbeg, kend) of operands
@@ -156,7 +164,7 @@ __device__ __forceinline__ KRange k_range(const GemmArgs &a, int c) {
 // lies past the last output), so the ring's bulk_wait_read count is exact.
 template <bool F32, int RING>
 __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, const Tile &tl,
-                                               int q4, int lane, uint8_t *ring, uint32_t &nbox,
+                                               int row0, int lane, uint8_t *ring, uint32_t &nbox,
                                                const GemmOuts &outs, const GemmArgs &a) {
   const bool first_half = F32 || (cb & 1) == 0;
   uint8_t *box = ring + (nbox % RING) * kBoxBytes;
@@ -204,11 +212,11 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, 
     __syncwarp();
     if (lane == 0) {
       if (F32) {
-        tma_store_3d(&outs.map[0], box, tl.n0 + cb * 32, tl.m0 + q4 * 32, tl.c);
+        tma_store_3d(&outs.map[0], box, tl.n0 + cb * 32, row0, tl.c);
       } else {
         const int n = tl.n0 + (cb >> 1) * 64;          // first column of the box
         const int o = n / a.cols_per_out;               // the output tensor it belongs to
-        if (o < a.nouts) tma_store_3d(&outs.map[o], box, n - o * a.cols_per_out, tl.m0 + q4 * 32, tl.c);
+        if (o < a.nouts) tma_store_3d(&outs.map[o], box, n - o * a.cols_per_out, row0, tl.c);
       }
       bulk_commit_group();
     }
@@ -216,17 +224,18 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&v)[32], int cb, 
   }
 }
 
-template <bool XMN, bool YMN, bool F32, int STAGES, int RING>
+template <bool XMN, bool YMN, bool F32, int STAGES, int RING, int HALVES>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ GemmMaps ys,
                const __grid_constant__ GemmOuts outs, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  GemmSmem &ctl = *reinterpret_cast<GemmSmem *>(smem + Pipe<STAGES, RING>::kOffCtl);
+  using P = Pipe<STAGES, RING, HALVES>;
+  GemmSmem &ctl = *reinterpret_cast<GemmSmem *>(smem + P::kOffCtl);
   volatile uint32_t *abort_flag = &ctl.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = (a.M + kTM - 1) / kTM, nt = (a.Nn + kTN - 1) / kTN;
+  const int mt = (a.M + P::kTileM - 1) / P::kTileM, nt = (a.Nn + kTN - 1) / kTN;
   const int tiles = mt * nt * a.batch;
 
   if (threadIdx.x == 0) {
@@ -234,7 +243,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
       mbar_init(&ctl.full[s], 1);
       mbar_init(&ctl.empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < P::kBufs; ++b) {
       mbar_init(&ctl.acc_full[b], 1);
       mbar_init(&ctl.acc_empty[b], kEpiWarps);       // one arrival per epilogue warp
     }
@@ -259,7 +268,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
       uint32_t it = 0;                                // K slices issued, over all tiles
       bool ok = true;
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const Tile tl = tile_of(t, mt, nt);
+        const Tile tl = tile_of(t, mt, nt, P::kTileM);
         const KRange kr = k_range(a, tl.c);
         for (int kt = 0; kt < kr.nk; ++kt, ++it) {
           const int st = it % STAGES;
@@ -268,15 +277,16 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
             ok = false;
             break;
           }
-          uint8_t *dst = smem + st * kStageBytes;
-          mbar_arrive_expect_tx(&ctl.full[st], kStageBytes);
+          uint8_t *dst = smem + st * P::kStageBytes;
+          mbar_arrive_expect_tx(&ctl.full[st], P::kStageBytes);
           const int k = kr.kbeg + kt * kTK;
           const int xi = k / a.k_per_x;                // the X tensor holding this K slice
-          load_slice<XMN, kTM>(dst, &xs.map[xi], &ctl.full[st], tl.m0, k - xi * a.k_per_x, kr.cin);
+          load_slice<XMN, P::kTileM>(dst, &xs.map[xi], &ctl.full[st], tl.m0,
+                                     k - xi * a.k_per_x, kr.cin);
           if (a.n_per_y)
-            load_y_slice<YMN>(dst + kXBytes, ys, a, &ctl.full[st], tl.n0, k, kr.cin);
+            load_y_slice<YMN>(dst + P::kXBytes, ys, a, &ctl.full[st], tl.n0, k, kr.cin);
           else
-            load_slice<YMN, kTN>(dst + kXBytes, &ys.map[0], &ctl.full[st], tl.n0, k, kr.cin);
+            load_slice<YMN, kTN>(dst + P::kXBytes, &ys.map[0], &ctl.full[st], tl.n0, k, kr.cin);
         }
       }
       if (!ok)      // let the copies already issued land before the CTA exits
@@ -291,15 +301,15 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
       bool ok = true;
       int j = 0;                                      // tiles of this CTA
       for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++j) {
-        const int buf = j & 1;
-        if (j >= 2 &&
-            !wait_bar(&ctl.acc_empty[buf], ((j >> 1) - 1) & 1, abort_flag, a.status)) {
+        const int buf = j % P::kBufs;
+        const int use = j / P::kBufs;                 // earlier uses of this accumulator set
+        if (use >= 1 &&
+            !wait_bar(&ctl.acc_empty[buf], (use - 1) & 1, abort_flag, a.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + buf * kTN;
-        const KRange kr = k_range(a, tile_of(t, mt, nt).c);
+        const KRange kr = k_range(a, tile_of(t, mt, nt, P::kTileM).c);
         for (int kt = 0; kt < kr.nk; ++kt, ++it) {
           const int st = it % STAGES;
           if (!wait_bar(&ctl.full[st], (it / STAGES) & 1, abort_flag, a.status)) {
@@ -307,12 +317,18 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
             break;
           }
           tc_fence_after();
-          const uint32_t xa = smem_u32(smem + st * kStageBytes);
-          const uint32_t ya = xa + kXBytes;
+          const uint32_t xa = smem_u32(smem + st * P::kStageBytes);
+          const uint32_t ya = xa + P::kXBytes;
 #pragma unroll
-          for (int ks = 0; ks < kTK / 16; ++ks)
-            mma_ss(d, slice_desc<XMN>(xa, ks), slice_desc<YMN>(ya, ks), idesc,
-                   (kt > 0 || ks > 0) ? 1u : 0u);
+          for (int h = 0; h < HALVES; ++h) {
+            // rows 128h.. of the X slice: 16 KB on in both layouts (K-major: the
+            // second 128-row box; MN-major: the third 64-wide atom column)
+            const uint32_t d = tmem + (buf * HALVES + h) * kTN;
+#pragma unroll
+            for (int ks = 0; ks < kTK / 16; ++ks)
+              mma_ss(d, slice_desc<XMN>(xa + h * kTM * kTK * 2, ks), slice_desc<YMN>(ya, ks),
+                     idesc, (kt > 0 || ks > 0) ? 1u : 0u);
+          }
           mma_commit(&ctl.empty[st]);
         }
         if (ok) mma_commit(&ctl.acc_full[buf]);
@@ -324,25 +340,30 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
   } else {
     // ------------------------------------------------------------ epilogue --
     // Warp w reads accumulator lanes 32 (w % 4) .. + 31 (its rank in the
-    // warpgroup); the first four epilogue warps take columns 0..127 of the tile,
-    // the other four columns 128..255. Chunks past the output's last column
-    // (rounded up to a whole box) are skipped.
-    const int e = warp - 2, q4 = warp & 3, half = e >> 2;
-    uint8_t *ring = smem + Pipe<STAGES, RING>::kOffStaging + e * RING * kBoxBytes;
+    // warpgroup). HALVES = 1: the first four epilogue warps take columns 0..127
+    // of the tile, the other four columns 128..255. HALVES = 2: the first four
+    // take the upper 128-row half, the other four the lower half, all columns.
+    // Chunks past the output's last column (rounded up to a whole box) are
+    // skipped.
+    const int e = warp - 2, q4 = warp & 3, grp = e >> 2;
+    uint8_t *ring = smem + P::kOffStaging + e * RING * kBoxBytes;
     uint32_t nbox = 0;
     int j = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++j) {
-      const int buf = j & 1;
-      bool ok = mbar_try_wait(&ctl.acc_full[buf], (j >> 1) & 1) ||
-                wait_bar(&ctl.acc_full[buf], (j >> 1) & 1, abort_flag, a.status);
+      const int buf = j % P::kBufs, par = (j / P::kBufs) & 1;
+      bool ok = mbar_try_wait(&ctl.acc_full[buf], par) ||
+                wait_bar(&ctl.acc_full[buf], par, abort_flag, a.status);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const Tile tl = tile_of(t, mt, nt);
-      const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + buf * kTN;
+      const Tile tl = tile_of(t, mt, nt, P::kTileM);
+      const int acc = HALVES == 1 ? buf : grp;          // accumulator this warp drains
+      const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + acc * kTN;
+      const int row0 = tl.m0 + (HALVES == 1 ? 0 : grp * kTM) + q4 * 32;
       const int cols = a.Nn - tl.n0;                   // output columns in this tile
       const int live = F32 ? (cols + 31) / 32 : 2 * ((cols + 63) / 64);
-      const int cb0 = half * (kTN / 64), cb1 = min(cb0 + kTN / 64, live);
-      if (cb0 < cb1) {
+      const int cb0 = HALVES == 1 ? grp * (kTN / 64) : 0;
+      const int cb1 = min(cb0 + (HALVES == 1 ? kTN / 64 : kTN / 32), live);
+      if (cb0 < cb1 && row0 < a.M) {
         uint32_t va[32], vb[32];
         tmem_ld32_issue(ta + cb0 * 32, va);
         tmem_wait_ld32(va);
@@ -350,10 +371,10 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
         for (int cb = cb0; cb < cb1; cb += 2) {
           const bool has_b = cb + 1 < cb1, has_a = cb + 2 < cb1;
           if (has_b) tmem_ld32_issue(ta + (cb + 1) * 32, vb);
-          epilogue_chunk<F32, RING>(va, cb, tl, q4, lane, ring, nbox, outs, a);
+          epilogue_chunk<F32, RING>(va, cb, tl, row0, lane, ring, nbox, outs, a);
           if (has_b) tmem_wait_ld32(vb);
           if (has_a) tmem_ld32_issue(ta + (cb + 2) * 32, va);
-          if (has_b) epilogue_chunk<F32, RING>(vb, cb + 1, tl, q4, lane, ring, nbox, outs, a);
+          if (has_b) epilogue_chunk<F32, RING>(vb, cb + 1, tl, row0, lane, ring, nbox, outs, a);
           if (has_a) tmem_wait_ld32(va);
         }
       }
@@ -375,14 +396,20 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps xs, const __grid_constant__ Gemm
   }
 }
 
-template <bool XMN, bool YMN, bool F32, int STAGES, int RING>
+template <bool XMN, bool YMN, bool F32, int STAGES, int RING, int HALVES>
 cudaError_t launch_pipe(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
-                        const GemmArgs &args, int grid, cudaStream_t stream) {
-  constexpr uint32_t bytes = smem_bytes<STAGES, RING>();
-  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32, STAGES, RING>,
+                        const GemmArgs &args, int sms, cudaStream_t stream) {
+  constexpr uint32_t bytes = smem_bytes<STAGES, RING, HALVES>();
+  constexpr int tile_m = Pipe<STAGES, RING, HALVES>::kTileM;
+  const int64_t tiles = (int64_t)((args.M + tile_m - 1) / tile_m) * ((args.Nn + kTN - 1) / kTN) *
+                        args.batch;
+  if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<XMN, YMN, F32, STAGES, RING, HALVES>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  gemm_tc_kernel<XMN, YMN, F32, STAGES, RING><<<grid, kThreads, bytes, stream>>>(x, y, d, args);
+  gemm_tc_kernel<XMN, YMN, F32, STAGES, RING, HALVES><<<grid, kThreads, bytes, stream>>>(
+      x, y, d, args);
   return cudaGetLastError();
 }
 
@@ -394,14 +421,10 @@ cudaError_t launch(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return e;
-  const int64_t tiles = (int64_t)((args.M + kTM - 1) / kTM) * ((args.Nn + kTN - 1) / kTN) *
-                        args.batch;
-  if (tiles >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  const int grid = (int)(tiles < sms ? tiles : sms);
   const int k_tile = args.k_split ? args.k_split : args.K;   // K of one tile
-  if ((k_tile + kTK - 1) / kTK >= 8)
-    return launch_pipe<XMN, YMN, F32, 4, 1>(x, y, d, args, grid, stream);
-  return launch_pipe<XMN, YMN, F32, 3, 2>(x, y, d, args, grid, stream);
+  if ((k_tile + kTK - 1) / kTK < 8) return launch_pipe<XMN, YMN, F32, 3, 2, 1>(x, y, d, args, sms, stream);
+  if (args.M <= kTM) return launch_pipe<XMN, YMN, F32, 4, 1, 1>(x, y, d, args, sms, stream);
+  return launch_pipe<XMN, YMN, F32, 3, 1, 2>(x, y, d, args, sms, stream);
 }
 
 }  // namespace
