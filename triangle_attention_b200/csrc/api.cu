@@ -905,6 +905,7 @@ tri_attn_status tri_proj_in_bwd(const tri_proj_problem *prob, const void *z, con
   a.dbias = static_cast<const __nv_bfloat16 *>(dbias);
   a.dz = static_cast<__nv_bfloat16 *>(dz);
   a.part = ws.part;
+  a.status = ws.status;
   cudaError_t e = tri::launch_ln_bwd(a, stream);
   const int64_t warps = tri::proj_partials(), pw = cz * (2 + prob->H);
   if (e == cudaSuccess) e = tri::launch_ordered_sum(ws.part, warps, pw, cz, dgamma, cz, cz, stream);

@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "common.cuh"
 #include "ptx.cuh"
 #include "proj.cuh"
 
@@ -238,18 +239,81 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 3 : 2) ln_fwd_kernel(ProjArgs 
   }
 }
 
+// Backward staging: chunks of kChunkRows rows of z, x (bf16) and dx (fp32)
+// come into shared memory by 1-D bulk copies, kBwdStages chunks in flight per
+// block, so the warps never wait on single-row loads.
+constexpr int kChunkRows = 32;                  // 4 rows per warp of a 256-thread block
+constexpr int kBwdStages = 3;
+constexpr uint32_t kAccBytes = 256 * (2 + kMaxHeads) * 4;
+
+__host__ __device__ constexpr uint32_t bwd_stage_bytes(int cz) { return kChunkRows * cz * 8; }
+__host__ __device__ constexpr uint32_t bwd_smem_bytes(int cz) {
+  return kAccBytes + 128 + kBwdStages * bwd_stage_bytes(cz);
+}
+
+// Bounded wait on a staging barrier; false once it ran out or the block gave up.
+__device__ __forceinline__ bool stage_wait(uint64_t *bar, uint32_t parity,
+                                           volatile uint32_t *abort_flag, int32_t *status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t polls = 1; polls < kWaitMaxPolls; ++polls) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((polls & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) break;
+    }
+  }
+  *abort_flag = 1u;
+  report_status(status, kStatusTimeout);
+  return false;
+}
+
 // dz from dx (the projections' gradient w.r.t. x, fp32) plus the bias term
 // sum_h dbias[h][row] w_b[c][h]; partial sums of dgamma, dbeta and
 // dw_b[c][h] = sum_rows x[c] dbias[h][row] (x as the forward stored it), one
 // set per block: each warp accumulates its rows, then the block's warps are
-// added in warp order. RPW rows at a time, the next group's inputs loaded
-// while the current one is worked on.
-template <int CPL, int HM, int RPW>
-__global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs a) {
-  __shared__ float acc[256 * (2 + kMaxHeads)];
+// added in warp order. Block b takes the chunks b, b + gridDim.x, ...; warp w
+// the rows 4w .. 4w + 3 of each.
+template <int CPL, int HM>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(ProjArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  float *acc = reinterpret_cast<float *>(smem);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + kAccBytes);
+  uint64_t *empty = full + kBwdStages;
+  volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(empty + kBwdStages);
+  uint8_t *stages = smem + kAccBytes + 128;
+  const uint32_t stage_bytes = bwd_stage_bytes(a.cz);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int c0 = lane * CPL;
   const float inv_cz = 1.0f / a.cz;
+  const int64_t nchunks = (a.rows + kChunkRows - 1) / kChunkRows;
+  const bool producer = threadIdx.x == 0;
+  if (producer) {
+    for (int st = 0; st < kBwdStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], blockDim.x >> 5);
+    }
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  // chunk `chunk` into stage st: z | x | dx of its rows
+  auto issue = [&](int64_t chunk, int st) {
+    const int64_t r0 = chunk * kChunkRows;
+    const int64_t nr = a.rows - r0 < kChunkRows ? a.rows - r0 : (int64_t)kChunkRows;
+    const uint32_t b16 = (uint32_t)(nr * a.cz * 2);
+    uint8_t *dst = stages + st * stage_bytes;
+    mbar_arrive_expect_tx(&full[st], 4 * b16);
+    bulk_load(dst, a.z + r0 * a.cz, b16, &full[st]);
+    bulk_load(dst + kChunkRows * a.cz * 2, a.x + r0 * a.cz, b16, &full[st]);
+    bulk_load(dst + kChunkRows * a.cz * 4, a.dx + r0 * a.cz, 2 * b16, &full[st]);
+  };
+  int64_t issued = 0;                           // chunks of this block issued so far
+  if (producer)
+    for (int64_t ch = blockIdx.x; issued < kBwdStages - 1 && ch < nchunks; ch += gridDim.x)
+      issue(ch, (int)(issued++));
+
   float wb[CPL][HM];
   load_wb<CPL, HM>(a, c0, wb);
   float g[CPL], dg[CPL], db[CPL], dwb[CPL][HM];
@@ -260,82 +324,72 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs 
 #pragma unroll
     for (int h = 0; h < HM; ++h) dwb[e][h] = 0.0f;
   }
-  const int64_t groups = (a.rows + RPW - 1) / RPW;
-  int64_t grp = first_group();
-  uint32_t zr[RPW][CPL / 2], xr[RPW][CPL / 2];
-  float dx[RPW][CPL], dbh[RPW][HM];
-  float2 st[RPW];
-  auto load = [&](int64_t r0) {
-    load_group<CPL, RPW>(a.z, a.rows, a.cz, r0, c0, zr);
-    load_group<CPL, RPW>(a.x, a.rows, a.cz, r0, c0, xr);
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const int64_t row = r0 + r;
-      if (row < a.rows) {
-        load_row_f32<CPL>(a.dx + row * a.cz + c0, dx[r]);
-        st[r] = reinterpret_cast<const float2 *>(a.stats)[row];
-        const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
-#pragma unroll
-        for (int h = 0; h < HM; ++h)
-          dbh[r][h] = h < a.H ? __bfloat162float(dbias[h * a.rows_per]) : 0.0f;
-      } else {
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) dx[r][e] = 0.0f;
-        st[r] = make_float2(0.0f, 0.0f);
-#pragma unroll
-        for (int h = 0; h < HM; ++h) dbh[r][h] = 0.0f;
+  int64_t i = 0;                                // chunks of this block consumed so far
+  for (int64_t chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x, ++i) {
+    const int st = (int)(i % kBwdStages);
+    if (producer) {
+      const int64_t next = chunk + (int64_t)(kBwdStages - 1) * gridDim.x;
+      if (next < nchunks) {
+        const int ns = (int)(issued % kBwdStages);
+        // that stage last held chunk number issued - kBwdStages of this block
+        const bool ok = issued < kBwdStages ||
+                        stage_wait(&empty[ns], ((issued - kBwdStages) / kBwdStages) & 1,
+                                   abort_flag, a.status);
+        if (ok) issue(next, ns), ++issued;
       }
     }
-  };
-  if (grp < groups) load(grp * RPW);
-  for (; grp < groups; grp += group_stride()) {
-    const int64_t r0 = grp * RPW;
-    float xh[RPW][CPL], u[RPW][CPL], s[2 * RPW];
+    __syncwarp();
+    if (!__all_sync(0xffffffffu,
+                    stage_wait(&full[st], (i / kBwdStages) & 1, abort_flag, a.status)))
+      break;
+    const uint8_t *sz = stages + st * stage_bytes;
+    const uint8_t *sx = sz + kChunkRows * a.cz * 2;
+    const float *sdx = reinterpret_cast<const float *>(sz + kChunkRows * a.cz * 4);
+    const int64_t r0 = chunk * kChunkRows + warp * 4;
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      float z[CPL], x[CPL];
-      unpack<CPL>(zr[r], z);
-      unpack<CPL>(xr[r], x);
+    for (int r = 0; r < 4; ++r) {
+      const int64_t row = r0 + r;
+      if (row >= a.rows) break;                 // warp-uniform
+      const int lr = warp * 4 + r;              // row within the chunk
+      float z[CPL], x[CPL], u[CPL], xh[CPL];
+      load_row<CPL>(reinterpret_cast<const __nv_bfloat16 *>(sz) + lr * a.cz + c0, z);
+      load_row<CPL>(reinterpret_cast<const __nv_bfloat16 *>(sx) + lr * a.cz + c0, x);
+      load_row_f32<CPL>(sdx + lr * a.cz + c0, u);
+      const float2 stt = reinterpret_cast<const float2 *>(a.stats)[row];
+      const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
+      float dbh[HM];
+#pragma unroll
+      for (int h = 0; h < HM; ++h) dbh[h] = h < a.H ? __bfloat162float(dbias[h * a.rows_per]) : 0.0f;
+      float s[2] = {0.0f, 0.0f};
 #pragma unroll
       for (int e = 0; e < CPL; ++e) {
-        float d = dx[r][e];
 #pragma unroll
         for (int h = 0; h < HM; ++h) {
-          d += dbh[r][h] * wb[e][h];
-          dwb[e][h] += x[e] * dbh[r][h];
+          u[e] += dbh[h] * wb[e][h];
+          dwb[e][h] += x[e] * dbh[h];
         }
-        xh[r][e] = (z[e] - st[r].x) * st[r].y;
-        u[r][e] = d;
+        xh[e] = (z[e] - stt.x) * stt.y;
+        dg[e] += u[e] * xh[e];
+        db[e] += u[e];
+        u[e] *= g[e];                           // dL/dxhat
+        s[0] += u[e];
+        s[1] += u[e] * xh[e];
       }
+      const float tot = reduce_scatter<2>(s, lane);
+      const float m1 = __shfl_sync(0xffffffffu, tot, 0) * inv_cz;
+      const float m2 = __shfl_sync(0xffffffffu, tot, 16) * inv_cz;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) u[e] = stt.y * (u[e] - m1 - xh[e] * m2);
+      store_row<CPL>(a.dz + row * a.cz + c0, u);
     }
-    float rstd[RPW];
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) rstd[r] = st[r].y;
-    if (grp + group_stride() < groups) load((grp + group_stride()) * RPW);
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      s[r] = s[RPW + r] = 0.0f;
-#pragma unroll
-      for (int e = 0; e < CPL; ++e) {
-        dg[e] += u[r][e] * xh[r][e];
-        db[e] += u[r][e];
-        u[r][e] *= g[e];                           // dL/dxhat
-        s[r] += u[r][e];
-        s[RPW + r] += u[r][e] * xh[r][e];
-      }
-    }
-    constexpr int kShift = 5 - ilog2(2 * RPW);
-    const float tot = reduce_scatter<2 * RPW>(s, lane);
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float m1 = __shfl_sync(0xffffffffu, tot, r << kShift) * inv_cz;
-      const float m2 = __shfl_sync(0xffffffffu, tot, (RPW + r) << kShift) * inv_cz;
-      float dz[CPL];
-#pragma unroll
-      for (int e = 0; e < CPL; ++e) dz[e] = rstd[r] * (u[r][e] - m1 - xh[r][e] * m2);
-      if (r0 + r < a.rows) store_row<CPL>(a.dz + (r0 + r) * a.cz + c0, dz);
-    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
   }
+  __syncthreads();
+  // copies issued but never consumed (only after a timeout) must land before exit
+  if (producer)
+    for (int64_t j = i; j < issued; ++j)
+      mbar_wait(&full[j % kBwdStages], (j / kBwdStages) & 1);
   // block partials [dgamma cz | dbeta cz | dw_b cz*H], warps added in order
   const int len = a.cz * (2 + a.H);
   for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
@@ -356,7 +410,7 @@ __global__ void __launch_bounds__(256, CPL <= 4 ? 2 : 1) ln_bwd_kernel(ProjArgs 
     __syncthreads();
   }
   float *part = a.part + blockIdx.x * (int64_t)len;
-  for (int i = threadIdx.x; i < len; i += blockDim.x) part[i] = acc[i];
+  for (int j = threadIdx.x; j < len; j += blockDim.x) part[j] = acc[j];
 }
 
 // Per-warp partial column sums of a [rows][cols] bf16 matrix (cols = 32*CPL),
@@ -451,18 +505,26 @@ cudaError_t launch_ln_fwd(const ProjArgs &a, cudaStream_t stream) {
   return a.H <= 4 ? launch_ln_fwd_h<4>(a, stream) : launch_ln_fwd_h<kMaxHeads>(a, stream);
 }
 
+template <int CPL, int HM>
+cudaError_t launch_ln_bwd_k(const ProjArgs &a, cudaStream_t stream) {
+  const uint32_t bytes = bwd_smem_bytes(a.cz);
+  cudaError_t e = cudaFuncSetAttribute(ln_bwd_kernel<CPL, HM>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  ln_bwd_kernel<CPL, HM><<<kProjBlocks, 256, bytes, stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int HM>
 cudaError_t launch_ln_bwd_h(const ProjArgs &a, cudaStream_t stream) {
-  const int blocks = kProjBlocks;
   if (a.cz % 64) return cudaErrorInvalidValue;
   switch (a.cz / 32) {
-    case 2: ln_bwd_kernel<2, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
-    case 4: ln_bwd_kernel<4, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
-    case 6: ln_bwd_kernel<6, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
-    case 8: ln_bwd_kernel<8, HM, 2><<<blocks, 256, 0, stream>>>(a); break;
+    case 2: return launch_ln_bwd_k<2, HM>(a, stream);
+    case 4: return launch_ln_bwd_k<4, HM>(a, stream);
+    case 6: return launch_ln_bwd_k<6, HM>(a, stream);
+    case 8: return launch_ln_bwd_k<8, HM>(a, stream);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_ln_bwd(const ProjArgs &a, cudaStream_t stream) {

@@ -27,6 +27,7 @@ struct ProjArgs {
   const __nv_bfloat16 *dbias;        // backward: [batch][H][rows_per]
   __nv_bfloat16 *dz;                 // backward: [rows][cz]
   float *part;                       // backward: [kProjBlocks][cz * (2 + H)] partial sums
+  int32_t *status;                   // backward: device status word (bounded waits)
 };
 
 int proj_partials();         // partial sums per row reduction (kProjBlocks)
