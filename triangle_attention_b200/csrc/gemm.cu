@@ -400,6 +400,7 @@ template <bool XMN, bool YMN, bool F32, int STAGES, int RING, int HALVES>
 cudaError_t launch_pipe(const GemmMaps &x, const GemmMaps &y, const GemmOuts &d,
                         const GemmArgs &args, int sms, cudaStream_t stream) {
   constexpr uint32_t bytes = smem_bytes<STAGES, RING, HALVES>();
+  static_assert(bytes <= 227 * 1024, "shared memory budget");
   constexpr int tile_m = Pipe<STAGES, RING, HALVES>::kTileM;
   const int64_t tiles = (int64_t)((args.M + tile_m - 1) / tile_m) * ((args.Nn + kTN - 1) / kTN) *
                         args.batch;

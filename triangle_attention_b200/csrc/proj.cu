@@ -100,7 +100,7 @@ __device__ __forceinline__ void load_row_f32(const float *p, float (&v)[CPL]) {
   }
 }
 
-constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
+__host__ __device__ constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n / 2); }
 
 // Warp sum of NV values at once (NV a power of two, at most 32) by recursive
 // halving: at lane offsets 16, 8, ... each lane keeps half of its values and
