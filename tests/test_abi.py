@@ -20,7 +20,7 @@ def declared_functions():
     for h in HEADERS:
         src = open(h).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-        for m in re.finditer(r"\b(tri_attn_\w+)\s*\(", src):
+        for m in re.finditer(r"\b(tri_(?:attn|mul|proj)_\w+)\s*\(", src):
             names.add(m.group(1))
     return sorted(names)
 
@@ -35,7 +35,9 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("tri_attn_fwd", "tri_attn_bwd", "tri_attn_fwd_workspace_size",
                      "tri_attn_bwd_workspace_size", "tri_attn_read_status",
-                     "tri_attn_status_string", "tri_attn_version"):
+                     "tri_attn_status_string", "tri_attn_version", "tri_mul_fwd", "tri_mul_bwd",
+                     "tri_proj_in_fwd", "tri_proj_in_bwd", "tri_proj_out_fwd",
+                     "tri_proj_out_bwd", "tri_proj_workspace_size"):
         assert required in names
 
 
