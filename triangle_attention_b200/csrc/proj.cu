@@ -339,6 +339,19 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(ProjArgs a) {
       }
     }
     __syncwarp();
+    // lane l fetches the statistics and dbias of row l of the chunk while the
+    // chunk lands; the rows' threads take them by shuffle
+    float2 lst = make_float2(0.0f, 0.0f);
+    float ldb[HM];
+    {
+      const int64_t lrow = chunk * kChunkRows + lane;
+      const bool in = lrow < a.rows;
+      if (in) lst = reinterpret_cast<const float2 *>(a.stats)[lrow];
+      const __nv_bfloat16 *dbias = a.dbias + (in ? bias_base(a, lrow) : 0);
+#pragma unroll
+      for (int h = 0; h < HM; ++h)
+        ldb[h] = (in && h < a.H) ? __bfloat162float(dbias[h * a.rows_per]) : 0.0f;
+    }
     if (!__all_sync(0xffffffffu,
                     stage_wait(&full[st], (i / kBwdStages) & 1, abort_flag, a.status)))
       break;
@@ -355,11 +368,11 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(ProjArgs a) {
       load_row<CPL>(reinterpret_cast<const __nv_bfloat16 *>(sz) + lr * a.cz + c0, z);
       load_row<CPL>(reinterpret_cast<const __nv_bfloat16 *>(sx) + lr * a.cz + c0, x);
       load_row_f32<CPL>(sdx + lr * a.cz + c0, u);
-      const float2 stt = reinterpret_cast<const float2 *>(a.stats)[row];
-      const __nv_bfloat16 *dbias = a.dbias + bias_base(a, row);
+      const float2 stt = make_float2(__shfl_sync(0xffffffffu, lst.x, lr),
+                                     __shfl_sync(0xffffffffu, lst.y, lr));
       float dbh[HM];
 #pragma unroll
-      for (int h = 0; h < HM; ++h) dbh[h] = h < a.H ? __bfloat162float(dbias[h * a.rows_per]) : 0.0f;
+      for (int h = 0; h < HM; ++h) dbh[h] = __shfl_sync(0xffffffffu, ldb[h], lr);
       float s[2] = {0.0f, 0.0f};
 #pragma unroll
       for (int e = 0; e < CPL; ++e) {
