@@ -15,6 +15,12 @@ independent problem (weak scaling); ranks share only a barrier and a max of
 the elapsed time. `--impl reference` times the fp64 CPU oracle on this host's
 cores instead (rank 0 only), on bounded samples of attention rows.
 
+Other lines (`--op`): `trimul` times the triangle multiplicative update
+contraction (N=768, C=128, both directions, forward + backward), `proj` the
+LayerNorm and projection stages around the attention (N=768, cz=128), `block`
+the whole block LayerNorm -> projections -> attention -> output projection and
+its backward. The default line is the attention.
+
 Rank 0 prints one JSON line.
 """
 
