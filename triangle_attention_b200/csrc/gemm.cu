@@ -9,19 +9,21 @@
 // attention (LayerNorm output times the projection weights, and their
 // gradients, the weight gradients as split-K batches of fp32 partial sums).
 //
-// Persistent: one CTA per SM walks the 128x256 output tiles (n fastest, then
-// m, then the batch), so the tiles in flight at any moment are neighbours that
-// share operands in L2. Two accumulators in tensor memory (2 x 256 columns):
-// the epilogue of one tile overlaps the main loop of the next.
-//   warp 0      TMA producer: 64-wide K slices of X and Y (48 KB), 3-stage ring
+// Persistent: one CTA per SM walks the output tiles (n fastest, then m, then
+// the batch), so the tiles in flight at any moment are neighbours that share
+// operands in L2. Tensor memory holds two 128 x 256 fp32 accumulators (all 512
+// columns): either two consecutive 128 x 256 tiles, so the epilogue of one tile
+// overlaps the main loop of the next, or the two 128-row halves of one
+// 256 x 256 tile (the shapes are described at Pipe below).
+//   warp 0      TMA producer: 64-wide K slices of X and Y, a ring of stages
 //               running across tiles
 //   warp 1      tensor-memory allocator and MMA issuer (N = 256 products)
-//   warps 2..9  epilogue, two per accumulator lane quarter (each half of the
-//               columns): tensor memory -> bf16 or fp32 (32-column loads, the
-//               next one in flight while the current one is converted) -> a
-//               2-box staging ring per warp -> TMA stores (bf16: 64-column
-//               boxes, each routed to one of up to four output tensors by its
-//               column; fp32: 32-column boxes)
+//   warps 2..9  epilogue, two per accumulator lane quarter: tensor memory ->
+//               bf16 or fp32 (32-column loads, the next one in flight while the
+//               current one is converted) -> a staging ring of 4 KB boxes per
+//               warp -> TMA stores (bf16: 64-column boxes, each routed to one
+//               of up to four output tensors by its column; fp32: 32-column
+//               boxes)
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
