@@ -9,8 +9,9 @@
 // One warp per pair position (row of z [rows][cz]); lane l holds channels
 // l*CPL .. l*CPL + CPL - 1, so a warp reads and writes whole rows contiguously.
 // Reductions over rows (dgamma, dbeta, the bias weights, the gate bias) are
-// accumulated per warp over a fixed set of rows and summed over the warps in a
-// fixed order: repeated calls are bit-identical.
+// accumulated per warp over a fixed set of rows, added over a block's warps in
+// warp order into one partial per block, and the partials are summed in block
+// order by ordered_sum_kernel: repeated calls are bit-identical.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
