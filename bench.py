@@ -665,8 +665,8 @@ def run_block(args, rank, world, local):
             for n in by}
     top = max(by, key=lambda n: stage_ms[n])
     launches = {"proj_in_fwd": 2, "attention_fwd": ta.kernel_launches(aprob, False, False),
-                "proj_out_fwd": 1, "proj_out_bwd": 5,
-                "attention_bwd": ta.kernel_launches(aprob, True, False), "proj_in_bwd": 9}
+                "proj_out_fwd": 1, "proj_out_bwd": 4,
+                "attention_bwd": ta.kernel_launches(aprob, True, False), "proj_in_bwd": 6}
     return {"metric": BLOCK_METRIC, "value": whole_job_tflops(world, sum(fl.values()), ms),
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -761,7 +761,7 @@ def run_proj(args, rank, world, local):
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs[top] / peaks["hbm_gbs"], "traffic": None,
                          "note": "algorithmic bytes of the whole stage over its event time"},
-            "clocks": clk, "gpu_launches": 17 * args.steps}
+            "clocks": clk, "gpu_launches": 13 * args.steps}
 
 
 def main():

@@ -686,12 +686,14 @@ struct ProjWs {
 size_t carve_proj(const tri_proj_problem *p, void *base, ProjWs *ws) {
   const int64_t R = proj_total_rows(p), cz = p->cz, hc = (int64_t)p->H * p->c;
   const int64_t warps = tri::proj_partials();
-  int64_t part = warps * cz * (2 + p->H);
-  part = std::max(part, warps * std::max(hc, cz));
+  // input backward: LayerNorm partials then the db_g column-sum partials, or the
+  // dW_qkvg split-K partials; output backward: the dW_o split-K partials then the
+  // db_o column-sum partials
+  int64_t part = warps * (cz * (2 + p->H) + hc);
   if (R > 0) {
     const KSplit si = split_k(cz, 4 * hc, R), so = split_k(hc, cz, R);
     part = std::max(part, (int64_t)si.n * cz * 4 * hc);
-    part = std::max(part, (int64_t)so.n * hc * cz);
+    part = std::max(part, (int64_t)so.n * hc * cz + warps * cz);
   }
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -729,7 +731,8 @@ tri_attn_status zero_f32(float *p, size_t n, cudaStream_t s) {
 // stored [K][M], Y as ny tensors [K][Nn / ny] side by side along n: split-K
 // partials into ws->part, then one ordered sum into out [M][Nn].
 tri_attn_status weight_grad(const void *x, const void *const *y, int ny, int64_t M, int64_t Nn,
-                            int64_t K, float *out, const ProjWs &ws, cudaStream_t stream) {
+                            int64_t K, float *out, const ProjWs &ws, cudaStream_t stream,
+                            tri::SumSeg *defer = nullptr) {
   const KSplit sp = split_k(M, Nn, K);
   const int64_t per_y = Nn / ny;
   tri::GemmMaps xs, ys;
@@ -753,19 +756,23 @@ tri_attn_status weight_grad(const void *x, const void *const *y, int ny, int64_t
   args.status = ws.status;
   tri_attn_status st = cuda_status(tri::launch_gemm_tc(true, true, true, xs, ys, outs, args, stream));
   if (st != TRI_ATTN_OK) return st;
-  return cuda_status(
-      tri::launch_ordered_sum(ws.part, sp.n, M * Nn, M * Nn, out, M * Nn, M * Nn, stream));
+  const tri::SumSeg seg{ws.part, sp.n, M * Nn, M * Nn, out, M * Nn, M * Nn};
+  if (defer) {                 // the caller sums it together with other partials
+    *defer = seg;
+    return TRI_ATTN_OK;
+  }
+  return cuda_status(tri::launch_ordered_sums(&seg, 1, stream));
 }
 
-// Column sums of a bf16 [R][cols] matrix into out[cols], in a fixed order.
-tri_attn_status column_sums(const void *m, int64_t R, int64_t cols, float *out, const ProjWs &ws,
-                            cudaStream_t stream) {
-  const int warps = tri::proj_partials();
-  cudaError_t e = tri::launch_colsum(static_cast<const __nv_bfloat16 *>(m), R, (int)cols,
-                                     ws.part, stream);
-  if (e == cudaSuccess)
-    e = tri::launch_ordered_sum(ws.part, warps, cols, cols, out, cols, cols, stream);
-  return cuda_status(e);
+// Elements of the split-K partials of a weight gradient (where other partials
+// may follow in the workspace).
+int64_t weight_grad_partials(int64_t M, int64_t Nn, int64_t K) {
+  return (int64_t)split_k(M, Nn, K).n * M * Nn;
+}
+
+// Sum segment of per-block column-sum partials [blocks][cols] into out[cols].
+tri::SumSeg colsum_segment(const float *part, int64_t cols, float *out) {
+  return tri::SumSeg{part, tri::proj_partials(), cols, cols, out, cols, cols};
 }
 
 }  // namespace
@@ -907,15 +914,20 @@ tri_attn_status tri_proj_in_bwd(const tri_proj_problem *prob, const void *z, con
   a.part = ws.part;
   a.status = ws.status;
   cudaError_t e = tri::launch_ln_bwd(a, stream);
+  // the db_g column-sum partials follow the LayerNorm partials; one launch sums both
   const int64_t warps = tri::proj_partials(), pw = cz * (2 + prob->H);
-  if (e == cudaSuccess) e = tri::launch_ordered_sum(ws.part, warps, pw, cz, dgamma, cz, cz, stream);
+  float *cpart = ws.part + warps * pw;
   if (e == cudaSuccess)
-    e = tri::launch_ordered_sum(ws.part + cz, warps, pw, cz, dbeta, cz, cz, stream);
-  if (e == cudaSuccess)
-    e = tri::launch_ordered_sum(ws.part + 2 * cz, warps, pw, cz * prob->H, dw_b, cz * prob->H,
-                                cz * prob->H, stream);
+    e = tri::launch_colsum(static_cast<const __nv_bfloat16 *>(dg), R, (int)hc, cpart, stream);
+  if (e == cudaSuccess) {
+    const tri::SumSeg segs[4] = {
+        {ws.part, warps, pw, cz, dgamma, cz, cz},
+        {ws.part + cz, warps, pw, cz, dbeta, cz, cz},
+        {ws.part + 2 * cz, warps, pw, cz * prob->H, dw_b, cz * prob->H, cz * prob->H},
+        colsum_segment(cpart, hc, db_g)};
+    e = tri::launch_ordered_sums(segs, 4, stream);
+  }
   if ((st = cuda_status(e)) != TRI_ATTN_OK) return st;
-  if ((st = column_sums(dg, R, hc, db_g, ws, stream)) != TRI_ATTN_OK) return st;
   // dw_qkvg = x^T [dq dk dv dg]
   const void *grads[4] = {dq, dk, dv, dg};
   return weight_grad(x, grads, 4, cz, 4 * hc, R, dw_qkvg, ws, stream);
@@ -994,8 +1006,16 @@ tri_attn_status tri_proj_out_bwd(const tri_proj_problem *prob, const void *o, co
     st = cuda_status(tri::launch_gemm_tc(false, false, false, xs, ys, outs, args, stream));
     if (st != TRI_ATTN_OK) return st;
   }
-  if ((st = weight_grad(o, &dy, 1, hc, cz, R, dw_o, ws, stream)) != TRI_ATTN_OK) return st;
-  return column_sums(dy, R, cz, db_o, ws, stream);
+  // dW_o split-K partials, then the db_o column-sum partials after them; one sum launch
+  tri::SumSeg segs[2];
+  if ((st = weight_grad(o, &dy, 1, hc, cz, R, dw_o, ws, stream, &segs[0])) != TRI_ATTN_OK)
+    return st;
+  float *cpart = ws.part + weight_grad_partials(hc, cz, R);
+  cudaError_t e = tri::launch_colsum(static_cast<const __nv_bfloat16 *>(dy), R, (int)cz, cpart,
+                                     stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  segs[1] = colsum_segment(cpart, cz, db_o);
+  return cuda_status(tri::launch_ordered_sums(segs, 2, stream));
 }
 
 }  // extern "C"

@@ -460,39 +460,40 @@ __global__ void __launch_bounds__(256) colsum_kernel(const __nv_bfloat16 *m, int
   for (int i = threadIdx.x; i < cols; i += blockDim.x) part[blockIdx.x * (int64_t)cols + i] = acc[i];
 }
 
-// out[i] = sum over k < n of part[k * part_stride + i], element i landing at
-// out + (i / width) * out_stride + i % width. A block of 32 warps takes 32
-// consecutive elements (one per lane); warp w adds the k of its fixed share
-// [w n / 32, (w + 1) n / 32) in order, then the 32 warp sums are added in warp
-// order, so the result does not depend on scheduling.
-__global__ void __launch_bounds__(1024) ordered_sum_kernel(const float *part, int64_t n,
-                                                           int64_t part_stride, int64_t len,
-                                                           float *out, int64_t width,
-                                                           int64_t out_stride) {
+// Each segment: out[i] = sum over k < n of part[k * part_stride + i], element i
+// landing at out + (i / width) * out_stride + i % width. A block of 32 warps
+// takes 32 consecutive elements of one segment (one per lane); warp w adds the
+// k of its fixed share [w n / 32, (w + 1) n / 32) in order, then the 32 warp
+// sums are added in warp order, so the result does not depend on scheduling.
+// Several segments share one launch (blocks first_block[s] .. of segment s).
+__global__ void __launch_bounds__(1024) ordered_sum_kernel(const __grid_constant__ SumSegs ss) {
   __shared__ float ws[32][33];
+  int si = 0;
+  while (si + 1 < ss.nseg && (int64_t)blockIdx.x >= ss.first_block[si + 1]) ++si;
+  const SumSeg &g = ss.seg[si];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t i = blockIdx.x * 32ll + lane;
-  const int64_t k0 = warp * n / 32, k1 = (warp + 1) * n / 32;
+  const int64_t i = ((int64_t)blockIdx.x - ss.first_block[si]) * 32 + lane;
+  const int64_t k0 = warp * g.n / 32, k1 = (warp + 1) * g.n / 32;
   float s = 0.0f;
-  if (i < len) {
-    const float *p = part + i;
+  if (i < g.len) {
+    const float *p = g.part + i;
     int64_t k = k0;
     for (; k + 4 <= k1; k += 4) {
-      const float v0 = p[k * part_stride], v1 = p[(k + 1) * part_stride];
-      const float v2 = p[(k + 2) * part_stride], v3 = p[(k + 3) * part_stride];
+      const float v0 = p[k * g.part_stride], v1 = p[(k + 1) * g.part_stride];
+      const float v2 = p[(k + 2) * g.part_stride], v3 = p[(k + 3) * g.part_stride];
       s += v0;
       s += v1;
       s += v2;
       s += v3;
     }
-    for (; k < k1; ++k) s += p[k * part_stride];
+    for (; k < k1; ++k) s += p[k * g.part_stride];
   }
   ws[warp][lane] = s;
   __syncthreads();
-  if (warp == 0 && i < len) {
+  if (warp == 0 && i < g.len) {
     float t = 0.0f;
     for (int w = 0; w < 32; ++w) t += ws[w][lane];
-    out[(i / width) * out_stride + i % width] = t;
+    g.out[(i / g.width) * g.out_stride + i % g.width] = t;
   }
 }
 
@@ -560,14 +561,27 @@ cudaError_t launch_colsum(const __nv_bfloat16 *m, int64_t rows, int cols, float 
   return cudaGetLastError();
 }
 
+cudaError_t launch_ordered_sums(const SumSeg *segs, int nseg, cudaStream_t stream) {
+  if (nseg < 1 || nseg > kMaxSumSegs) return cudaErrorInvalidValue;
+  SumSegs ss{};
+  ss.nseg = nseg;
+  int64_t blocks = 0;
+  for (int s = 0; s < nseg; ++s) {
+    ss.seg[s] = segs[s];
+    ss.first_block[s] = blocks;
+    blocks += (segs[s].len + 31) / 32;
+  }
+  if (blocks == 0) return cudaSuccess;
+  if (blocks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  ordered_sum_kernel<<<(unsigned)blocks, 1024, 0, stream>>>(ss);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_ordered_sum(const float *part, int64_t n, int64_t part_stride, int64_t len,
                                float *out, int64_t width, int64_t out_stride,
                                cudaStream_t stream) {
-  if (len == 0) return cudaSuccess;
-  const int64_t blocks = (len + 31) / 32;
-  ordered_sum_kernel<<<(unsigned)blocks, 1024, 0, stream>>>(part, n, part_stride, len, out,
-                                                           width, out_stride);
-  return cudaGetLastError();
+  const SumSeg seg{part, n, part_stride, len, out, width, out_stride};
+  return launch_ordered_sums(&seg, 1, stream);
 }
 
 }  // namespace tri

@@ -36,10 +36,24 @@ cudaError_t launch_ln_bwd(const ProjArgs &a, cudaStream_t stream);
 // per-block partial column sums of m [rows][cols] into part [kProjBlocks][cols]
 cudaError_t launch_colsum(const __nv_bfloat16 *m, int64_t rows, int cols, float *part,
                           cudaStream_t stream);
-// out[(i / width) * out_stride + i % width] = sum_{k < n} part[k * part_stride + i],
-// in k order, for i < len
+// One fixed-order sum over partials: out[(i / width) * out_stride + i % width] =
+// sum_{k < n} part[k * part_stride + i], in k order, for i < len.
+struct SumSeg {
+  const float *part;
+  int64_t n, part_stride, len;
+  float *out;
+  int64_t width, out_stride;
+};
+constexpr int kMaxSumSegs = 4;
+struct SumSegs {
+  SumSeg seg[kMaxSumSegs];
+  int nseg;
+  int64_t first_block[kMaxSumSegs];
+};
 cudaError_t launch_ordered_sum(const float *part, int64_t n, int64_t part_stride, int64_t len,
                                float *out, int64_t width, int64_t out_stride,
                                cudaStream_t stream);
+// up to kMaxSumSegs sums in one launch
+cudaError_t launch_ordered_sums(const SumSeg *segs, int nseg, cudaStream_t stream);
 
 }  // namespace tri
