@@ -1,5 +1,5 @@
 // Inline-PTX building blocks for sm_100a: mbarriers with bounded waits, TMA
-// tile loads (never with cluster multicast), tcgen05 tensor-memory allocation,
+// tile loads (each copy lands in this CTA only), tcgen05 tensor-memory allocation,
 // MMA issue/commit and tensor-memory loads/stores, shared-memory matrix and
 // instruction descriptors.
 #pragma once
