@@ -332,10 +332,12 @@ tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const vo
  * Ownership, errors, determinism: as for the attention. Every pointer is a
  * caller-owned, 16-byte aligned device pointer (x and stats too: the forward
  * writes them, the backward reads them). The workspace (tri_proj_workspace_size
- * bytes, one size for all four calls) holds the status word and the fp32
- * partial sums; parameter gradients are summed over the rows in a fixed order
- * (per-warp or per-split partials, then one ordered sum), so repeated calls are
- * bit-identical.
+ * bytes, one size for all four calls, device, 16-byte aligned) holds the status
+ * word that tri_attn_read_status() reads, the input backward's dx in fp32
+ * ([batch*rows][cz]) and the fp32 partial sums; parameter gradients are summed
+ * over the rows in a fixed order (per-block or per-split partials, then one
+ * ordered sum), so repeated calls are bit-identical. Device-side bounded waits
+ * that run out set TRI_ATTN_ERR_TIMEOUT in the status word; nothing traps.
  */
 typedef struct {
     int64_t rows;   /* pair positions per batch element (N*N) */
