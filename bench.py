@@ -87,73 +87,87 @@ def config_dict(w) -> dict:
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+    """SM clock and clock-event reasons sampled DURING the timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    A thread polls NVML (read-only queries) every `period_s` seconds, so even a
+    timed region of a few tens of milliseconds gets many samples; nvidia-smi's
+    own polling (100 ms at best) would see none. Falls back to `nvidia-smi -lms`
+    when NVML is not importable."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    REASON_BITS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40,
+                   "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
 
-    def start(self, wait_s: float = 20.0):
-        """Start sampling and wait for the first sample, so that nvidia-smi's own
-        start-up (which can stall other driver clients) ends before timing."""
-        import threading
-        self.lines = []
+    def __init__(self, device: int, period_s: float = 0.002):
+        self.device = device
+        self.period = period_s
+        self.samples = []
+        self.begin = 0
+        self.handle = None
+        self.thread = None
+        self.source = "nvml"
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            visible = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+                       if v.strip()]
+            idx = int(visible[self.device]) if self.device < len(visible) and \
+                visible[self.device].isdigit() else self.device
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def start(self):
+        import threading
+        try:
+            import pynvml
+            self.handle = self._nvml_handle()
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                  pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+            self.source = "unavailable"
             return
-        first = threading.Event()
+        self.running = True
 
-        def reader():
-            for line in self.proc.stdout:
-                self.lines.append(line)
-                first.set()
-            first.set()
+        def poll():
+            import pynvml
+            while self.running:
+                try:
+                    mhz = pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    self.samples.append((float(mhz), int(rs)))
+                except Exception:
+                    pass
+                time.sleep(self.period)
 
-        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread = threading.Thread(target=poll, daemon=True)
         self.thread.start()
-        first.wait(wait_s)
+        t_end = time.time() + 2.0
+        while not self.samples and time.time() < t_end:
+            time.sleep(0.001)
 
     def mark(self):
         """Index of the first sample taken inside the timed region."""
-        self.begin = len(self.lines)
+        self.begin = len(self.samples)
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        end = len(self.lines)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=10)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
-        out = "".join(self.lines[getattr(self, "begin", 0):max(end, getattr(self, "begin", 0) + 1)])
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable"],
+                    "samples": 0, "source": self.source}
+        end = len(self.samples)
+        self.running = False
+        self.thread.join(timeout=2)
+        window = self.samples[self.begin:end] or self.samples[-1:]
+        sm = [m for m, _ in window]
+        reasons = sorted(name for name, bit in self.REASON_BITS.items()
+                         if any(r & bit for _, r in window))
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(window),
+                "source": f"NVML poll every {self.period * 1e3:.0f} ms inside the timed region"}
 
 
 # ------------------------------------------------------------- distributed --
@@ -227,24 +241,49 @@ def oracle_rows_step(d, rows) -> float:
     return time.perf_counter() - t0
 
 
-def cpu_baseline(d, w, budget_s: float = 15.0) -> dict:
-    """The oracle as it stands, on this host's cores, on a bounded sample of
-    attention rows of the same workload (whole rows: every head, query, key)."""
-    d = oracle_inputs(d)
+def oracle_rows_per_step(d, w, cores: int, step_s: float = 1.0) -> int:
+    """Attention rows in one oracle step: a whole number of rounds of the host's
+    threads (the oracle spreads (row, head) pairs over them), about step_s long.
+    Both CPU legs (cpu_baseline and --impl reference) take steps of this size, so
+    they time the same thing and report the same throughput."""
+    t_row = oracle_rows_step(d, [0]) + 1e-9     # calibration, also warms the library
+    unit = max(1, -(-cores // w.H))             # rows that give every thread one pair
+    rounds = max(1, round(step_s / (t_row * unit)))
+    return int(min(w.N, unit * rounds))
+
+
+def oracle_sample(d, w, steps: int, warmup: int, seed: int, budget_s: float = 0.0) -> dict:
+    """fp64 oracle forward + backward on random samples of whole attention rows
+    (every head, query and key) of the workload, `steps` steps (or, with a
+    budget, steps until `budget_s` seconds of oracle time are spent);
+    throughput per row."""
     cores = oracle_threads()
-    rows_per_call = max(2, 2 * ((cores + w.H - 1) // w.H))
-    rng = np.random.default_rng(1)
-    done, secs = 0, 0.0
-    while secs < budget_s and done < w.N:
-        rows = rng.choice(w.N, size=min(rows_per_call, w.N), replace=False)
-        secs += oracle_rows_step(d, rows)
-        done += len(rows)
+    rows_per_step = oracle_rows_per_step(d, w, cores)
+    rng = np.random.default_rng(seed)
+    for _ in range(warmup):
+        oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
+    secs, done = 0.0, 0
+    while done < steps or secs < budget_s:
+        secs += oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
+        done += 1
+    steps = done
     f_fwd, f_bwd = flops(w.N, w.H, w.c)
     unit_flops = (f_fwd + f_bwd) / w.N          # one attention row, all heads
-    return {"value": unit_flops * done / secs / 1e12, "unit": UNIT, "cores": cores,
-            "kind": "oracle",
-            "sample": f"{done} of {w.N} attention rows (all heads), fp64 forward+backward, "
-                      f"{secs:.1f} s"}
+    value = unit_flops * rows_per_step * steps / secs / 1e12
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{steps} steps of {rows_per_step} of {w.N} attention rows (all heads), "
+                      f"fp64 forward+backward, {secs:.1f} s",
+            "ms_per_step": secs / steps * 1e3}
+
+
+def cpu_baseline(d, w, budget_s: float = 15.0) -> dict:
+    """The oracle as it stands, on this host's cores, on a bounded sample of
+    attention rows of the same workload: steps of about a second until the
+    budget is spent (the same step shape as the reference arm)."""
+    d = oracle_inputs(d)
+    res = oracle_sample(d, w, steps=1, warmup=1, seed=2, budget_s=budget_s)
+    res.pop("ms_per_step")
+    return res
 
 
 def run_reference(args, rank, world, w):
@@ -252,29 +291,15 @@ def run_reference(args, rank, world, w):
     if rank != 0:
         return None
     d = oracle_inputs(tri_inputs.workload_inputs(w.name))
-    cores = oracle_threads()
-    t_row = oracle_rows_step(d, [0]) + 1e-9     # calibration, also warms the library
-    budget_s = args.ref_budget_s
-    per_step = budget_s / max(1, args.steps + args.warmup)
-    rows_per_step = int(max(1, min(w.N, round(per_step / t_row))))
-    rng = np.random.default_rng(2)
-    for _ in range(args.warmup):
-        oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
-    secs = 0.0
-    for _ in range(args.steps):
-        secs += oracle_rows_step(d, rng.choice(w.N, rows_per_step, replace=False))
-    f_fwd, f_bwd = flops(w.N, w.H, w.c)
-    unit_flops = (f_fwd + f_bwd) / w.N
-    value = unit_flops * rows_per_step * args.steps / secs / 1e12
-    sample = (f"{rows_per_step} of {w.N} attention rows (all heads) per step, fp64 "
-              f"forward+backward")
+    res = oracle_sample(d, w, steps=args.steps, warmup=args.warmup, seed=2)
+    value = res["value"]
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
+            "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(w),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": res["cores"],
+                             "kind": "oracle", "sample": res["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -333,8 +358,7 @@ def run_ours(args, rank, world, local, w):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
 
-    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
-    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -505,8 +529,7 @@ def run_trimul(args, rank, world, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
-    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -633,8 +656,7 @@ def run_block(args, rank, world, local):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
-    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -720,8 +742,7 @@ def run_proj(args, rank, world, local):
         for n in names:
             stages[n]()
     torch.cuda.synchronize()
-    visible = [s for s in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if s.strip()]
-    clocks = ClockSampler(visible[local].strip() if local < len(visible) else local)
+    clocks = ClockSampler(local)
     clocks.start()
     barrier(world)
     torch.cuda.synchronize()
@@ -776,8 +797,6 @@ def main():
                          "whole block around the attention, or its projection stages alone")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-budget-s", type=float, default=150.0,
-                    help="host seconds the reference arm spends over all its steps")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")

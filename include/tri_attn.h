@@ -108,6 +108,13 @@ int tri_attn_version(void);
 const char *tri_attn_status_string(tri_attn_status status);
 
 /*
+ * Description of the CUDA error behind the last call on this host thread that
+ * returned TRI_ATTN_ERR_CUDA ("no error" if there was none); a static string
+ * owned by the CUDA runtime, never NULL. Host-only, enqueues nothing.
+ */
+const char *tri_attn_last_cuda_error(void);
+
+/*
  * Workspace the forward needs, in bytes (a status word, plus a transposed copy
  * of the bias for the ENDING variant). Writes *bytes; fails only on an invalid
  * problem.
@@ -214,14 +221,19 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
  * rejected with TRI_ATTN_ERR_WORKSPACE before anything is enqueued (starting
  * node: any size up to the N limit; ending node: H*N*N*2 bytes must also fit).
  *
- * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture. The call
- * itself never calls cudaMalloc, cudaFree or any allocating routine.
+ * The first call in a CUDA context looks up the array's device address with
+ * that context's device current and keeps it, keyed by the context's unique
+ * id; a later call in another context (a new primary context after
+ * cudaDeviceReset, or one the caller made current) looks it up again. Make the
+ * first call of each context before any stream capture. The call itself never
+ * calls cudaMalloc, cudaFree or any allocating routine.
  *
  * All calls share the one array and leave their scratch in it; every call
  * rewrites what it reads. Calls whose work overlaps on the GPU (other streams,
  * other host threads) race on the array and corrupt each other's results:
- * serialise them. A device-side failure shows as NaN in lse.
+ * serialise them. The status word lives inside the private array, so
+ * tri_attn_read_status() cannot reach it: for this entry point NaN in lse is
+ * the only sign of a device-side failure (a bounded wait that ran out).
  */
 tri_attn_status tri_attn_fwd_noalloc(const tri_attn_problem *prob, const void *q, const void *k,
                                      const void *v, const void *bias, const void *gate,

@@ -106,6 +106,8 @@ def lib():
         L.tri_attn_version.restype = ctypes.c_int
         L.tri_attn_status_string.argtypes = [ctypes.c_int]
         L.tri_attn_status_string.restype = ctypes.c_char_p
+        L.tri_attn_last_cuda_error.argtypes = []
+        L.tri_attn_last_cuda_error.restype = ctypes.c_char_p
         L.tri_attn_fwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
         L.tri_attn_bwd_workspace_size.argtypes = [PP, ctypes.POINTER(sz)]
         PO = ctypes.POINTER(LaunchOpts)
@@ -172,6 +174,8 @@ def _stream(stream=None):
 
 def _check(code: int, where: str):
     if code != 0:
+        if code == 4:   # TRI_ATTN_ERR_CUDA: name the CUDA error behind it
+            where = f"{where} [{lib().tri_attn_last_cuda_error().decode()}]"
         raise TriAttnError(code, where)
 
 

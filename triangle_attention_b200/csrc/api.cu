@@ -267,8 +267,13 @@ tri_attn_status mul_product(const tri_mul_problem *p, const void *x, bool x_mn, 
   return gemm_bf16(x, x_mn, y, y_mn, out, p->N, p->N, p->N, p->C, status, stream);
 }
 
+// The CUDA error behind the last TRI_ATTN_ERR_CUDA of this host thread.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
 tri_attn_status cuda_status(cudaError_t e) {
-  return e == cudaSuccess ? TRI_ATTN_OK : TRI_ATTN_ERR_CUDA;
+  if (e == cudaSuccess) return TRI_ATTN_OK;
+  g_last_cuda_error = e;
+  return TRI_ATTN_ERR_CUDA;
 }
 
 // Record the caller's timing event before (start) or after (stop) the main kernel.
@@ -308,6 +313,10 @@ cudaError_t mark(const tri_attn_launch_opts *opts, bool start, cudaStream_t stre
 extern "C" {
 
 int tri_attn_version(void) { return (1 << 16) | 0; }
+
+const char *tri_attn_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char *tri_attn_status_string(tri_attn_status s) {
   switch (s) {
