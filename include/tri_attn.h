@@ -172,13 +172,33 @@ tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const 
  */
 typedef struct {
     uint32_t struct_size;
-    uint32_t flags;           /* reserved, must be 0 */
+    uint32_t flags;           /* TRI_ATTN_OPT_* bits (backward only), else 0 */
     void *main_start;
     void *main_stop;
     void *out_residual;
 } tri_attn_launch_opts;
 
 #define TRI_ATTN_LAUNCH_OPTS_V1_SIZE ((uint32_t)(2 * sizeof(uint32_t) + 2 * sizeof(void *)))
+
+/*
+ * flags bit of tri_attn_bwd_ex: sum the per-tile contributions of dq, dk and dv
+ * inside the main kernel instead of in a second kernel. The bf16 backward
+ * splits every attention row into 128 x 128 query-key tiles, and each row's
+ * dq (dk, dv) is a sum over the key (query) tiles of that row ("TurboPairFormer
+ * accelera fino a 1,73x l'addestramento di OpenFold3 nei test", section "Dove
+ * si impiega il tempo"). By default every tile writes its bf16 contribution to
+ * the workspace and a reduction kernel adds them up in tile order. With this
+ * bit the tiles of one (row group, head) pair run as co-resident CTAs that pass
+ * their contributions through a ring of a few rows in the workspace (resident
+ * in L2) to one owner CTA per output tile, which adds them in tile order in
+ * fp32 and writes the result: no partial tensors, no reduction kernel, and the
+ * results are as deterministic as the default path's (they differ from it only
+ * in rounding). Applies when ceil(N / 128) <= 12 and one pair's
+ * ceil(N / 128)^2 CTAs fit on the device's SMs; otherwise the call takes the
+ * default path. tri_attn_bwd_workspace_size covers both paths. The forward and
+ * the fp32 backward reject the bit (TRI_ATTN_ERR_INVALID_ARG).
+ */
+#define TRI_ATTN_OPT_ONCHIP_SUMS 0x1u
 
 /* tri_attn_fwd with options (opts may be NULL: same as tri_attn_fwd). */
 tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
@@ -196,9 +216,11 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                 tri_attn_stream_t stream, const tri_attn_launch_opts *opts);
 
 /*
- * Number of kernel launches one call of the forward (backward = 0) or the
- * backward (backward = 1) enqueues for this problem and mask kind
- * (has_mask != 0 for a non-NULL mask). Writes *launches; host-only.
+ * Number of kernel launches one call of the forward (backward = 0), the
+ * backward (backward = 1) or the backward with TRI_ATTN_OPT_ONCHIP_SUMS
+ * (backward = 2) enqueues for this problem and mask kind (has_mask != 0 for a
+ * non-NULL mask), on the current device. Writes *launches; host-only. Any
+ * other value of backward: TRI_ATTN_ERR_INVALID_ARG.
  */
 tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backward,
                                          int has_mask, int32_t *launches);

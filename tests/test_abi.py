@@ -122,6 +122,45 @@ def test_host_side_rejections_before_any_launch(lib):
     assert lib.tri_attn_bwd(ctypes.byref(zero), *bargs, fake, 1 << 20, z) == 0
 
 
+def test_onchip_sum_option_on_the_host(lib):
+    """TRI_ATTN_OPT_ONCHIP_SUMS: accepted by the bf16 backward only; the launch
+    count and the workspace size cover that path. No CUDA call is made."""
+    fake = ctypes.c_void_p(4096)
+    z = None
+    prob = P(N=768)
+    args = [fake] * 5 + [z] + [fake, fake]
+    bargs = [fake] * 5 + [z] + [fake] * 8
+    opts = ta.launch_opts(onchip_sums=True)
+    assert opts.flags == ta.OPT_ONCHIP_SUMS == 1
+    # the forward takes no flags, and no flag but bit 0 exists
+    assert lib.tri_attn_fwd_ex(ctypes.byref(prob), *args, fake, 1 << 40, z,
+                               ctypes.byref(opts)) == 1
+    bad = ta.launch_opts()
+    bad.flags = 2
+    assert lib.tri_attn_bwd_ex(ctypes.byref(prob), *bargs, fake, 1 << 40, z,
+                               ctypes.byref(bad)) == 1
+    # the fp32 backward rejects the bit
+    f32 = P(N=32, dtype=ta.F32)
+    assert lib.tri_attn_bwd_ex(ctypes.byref(f32), *bargs, fake, 1 << 40, z,
+                               ctypes.byref(opts)) == 1
+    # too small a workspace is still caught first
+    assert lib.tri_attn_bwd_ex(ctypes.byref(prob), *bargs, fake, 16, z, ctypes.byref(opts)) == 3
+    # launches: mask bits, preprocessing, one main launch for all 4 heads of
+    # N=768 on 148 SMs (36 CTAs per head); the default path has 4
+    n = ctypes.c_int32(0)
+    assert lib.tri_attn_kernel_launches(ctypes.byref(prob), 2, 0, ctypes.byref(n)) == 0
+    assert n.value == 3
+    assert lib.tri_attn_kernel_launches(ctypes.byref(prob), 1, 0, ctypes.byref(n)) == 0
+    assert n.value == 4
+    assert lib.tri_attn_kernel_launches(ctypes.byref(prob), 3, 0, ctypes.byref(n)) == 1
+    # the workspace holds the exchange ring of that path too: 8 slots x 4 pairs x
+    # 3 kinds x 36 blocks of 128 x 32 bf16, plus dU and the (lse, D) pairs
+    rc, nb = ws_size(lib, prob, "bwd")
+    assert rc == 0
+    pair = 768 * 768 * 4 * 32
+    assert nb >= 2 * pair + 8 * 768 * 768 * 4 + 8 * 4 * 3 * 36 * 128 * 32 * 2
+
+
 def test_read_status_rejects_null(lib):
     v = ctypes.c_int32(0)
     assert lib.tri_attn_read_status(None, ctypes.byref(v), None) == 1

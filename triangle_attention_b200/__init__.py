@@ -50,17 +50,23 @@ class LaunchOpts(ctypes.Structure):
                 ("out_residual", ctypes.c_void_p)]
 
 
-def launch_opts(main_start=None, main_stop=None, residual=None) -> LaunchOpts:
-    """Options: torch.cuda.Event objects recorded around the main kernel, and
-    the bf16 rounding residual of `out` (a tensor shaped like out) that the
-    forward writes and the backward uses for D and dgate."""
+OPT_ONCHIP_SUMS = 0x1
+
+
+def launch_opts(main_start=None, main_stop=None, residual=None,
+                onchip_sums: bool = False) -> LaunchOpts:
+    """Options: torch.cuda.Event objects recorded around the main kernel, the
+    bf16 rounding residual of `out` (a tensor shaped like out) that the
+    forward writes and the backward uses for D and dgate, and (backward only)
+    the on-chip summation of the tile contributions (TRI_ATTN_OPT_ONCHIP_SUMS)."""
     def handle(ev):
         if ev is None:
             return None
         if not ev.cuda_event:            # torch creates the event lazily
             ev.record()
         return ctypes.c_void_p(ev.cuda_event)
-    return LaunchOpts(ctypes.sizeof(LaunchOpts), 0, handle(main_start), handle(main_stop),
+    return LaunchOpts(ctypes.sizeof(LaunchOpts), OPT_ONCHIP_SUMS if onchip_sums else 0,
+                      handle(main_start), handle(main_stop),
                       None if residual is None else ctypes.c_void_p(residual.data_ptr()))
 
 
@@ -193,10 +199,13 @@ def bwd_workspace_size(prob: Problem) -> int:
     return n.value
 
 
-def kernel_launches(prob: Problem, backward: bool, has_mask: bool) -> int:
-    """Kernel launches one forward (backward=False) or backward call enqueues."""
+def kernel_launches(prob: Problem, backward: bool, has_mask: bool,
+                    onchip_sums: bool = False) -> int:
+    """Kernel launches one forward (backward=False) or backward call enqueues
+    (onchip_sums: the backward with OPT_ONCHIP_SUMS)."""
     n = ctypes.c_int32(0)
-    _check(lib().tri_attn_kernel_launches(ctypes.byref(prob), int(backward), int(has_mask),
+    code = (2 if onchip_sums else 1) if backward else 0
+    _check(lib().tri_attn_kernel_launches(ctypes.byref(prob), code, int(has_mask),
                                           ctypes.byref(n)), "tri_attn_kernel_launches")
     return n.value
 

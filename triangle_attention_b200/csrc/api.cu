@@ -106,19 +106,40 @@ size_t carve_fwd(const tri_attn_problem *p, void *ws, bool per_row_mask, FwdWs *
   return c.off;
 }
 
+// SMs of the current device (the B200's 148 when no device answers, as on a
+// build host): the on-chip-sum backward sizes its grid, and so its workspace, by it.
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
 struct BwdWs {
   FwdWs fw;
   void *du;
   float *D;
   // fp32 path: partial sums per tile, reduced by a second kernel
   float *part_dq, *part_dk, *part_dv;
-  // bf16 path: bf16 contributions per tile, reduced by a second kernel
+  // bf16 path without on-chip sums: bf16 contributions per tile, reduced by a
+  // second kernel
   __nv_bfloat16 *bpart_q, *bpart_k, *bpart_v;
   float *part_db;
   int ntile, ngroups;
+  // bf16 path with on-chip sums (tc): lse/D pairs, exchange ring and flags
+  bool tc;
+  int ghl;                      // (group, head) pairs per launch
+  float *LD;
+  __nv_bfloat16 *ring;
+  int32_t *flags;               // exported | consumed_q | consumed_kv
+  int64_t nflags;
 };
 
-size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, BwdWs *out) {
+size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool onchip,
+                 BwdWs *out) {
   Carver c(ws);
   BwdWs w{};
   w.fw.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
@@ -128,14 +149,25 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, BwdWs *
     const int64_t rows = per_row_mask ? p->N : 1;
     w.fw.mask_bits =
         static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
-    if (p->variant == TRI_ATTN_ENDING)
-      w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
-    tri::bwd_bf16_plan((int)p->N, p->H, &w.ntile, &w.ngroups);
-    w.du = c.take(2 * pair);
-    w.D = static_cast<float *>(c.take(4 * nn * p->H));
-    w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
-    w.bpart_k = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
-    w.bpart_v = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+    w.tc = onchip && tri::bwd_tc_plan((int)p->N, p->H, sm_count(), &w.ntile, &w.ngroups, &w.ghl);
+    if (w.tc) {
+      const int64_t gh = (int64_t)w.ngroups * p->H, nb = w.ntile;
+      w.du = c.take(2 * pair);
+      w.LD = static_cast<float *>(c.take(8 * nn * p->H));
+      w.ring = static_cast<__nv_bfloat16 *>(
+          c.take((size_t)tri::bwd_tc_ring_slots() * w.ghl * 3 * nb * nb * 128 * 32 * 2));
+      w.nflags = gh * nb * nb + 2 * gh * nb * tri::bwd_tc_consumed_flags_per_tile();
+      w.flags = static_cast<int32_t *>(c.take(4 * (size_t)w.nflags));
+    } else {
+      if (p->variant == TRI_ATTN_ENDING)
+        w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
+      tri::bwd_bf16_plan((int)p->N, p->H, &w.ntile, &w.ngroups);
+      w.du = c.take(2 * pair);
+      w.D = static_cast<float *>(c.take(4 * nn * p->H));
+      w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+      w.bpart_k = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+      w.bpart_v = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+    }
   } else {
     tri::f32_bwd_plan(make_frame(p, nullptr, nullptr), &w.ntile, &w.ngroups);
     w.du = c.take(4 * pair);
@@ -284,11 +316,12 @@ void *opt_residual(const tri_attn_launch_opts *opts) {
   return opts->out_residual;
 }
 
-// Options are well formed: a known size, no flags, an aligned residual that
-// only the bf16 path takes.
-tri_attn_status check_opts(const tri_attn_problem *prob, const tri_attn_launch_opts *opts) {
+// Options are well formed: a known size, no flags beyond `allowed`, an aligned
+// residual that only the bf16 path takes.
+tri_attn_status check_opts(const tri_attn_problem *prob, const tri_attn_launch_opts *opts,
+                           uint32_t allowed) {
   if (!opts) return TRI_ATTN_OK;
-  if (opts->struct_size < TRI_ATTN_LAUNCH_OPTS_V1_SIZE || opts->flags != 0)
+  if (opts->struct_size < TRI_ATTN_LAUNCH_OPTS_V1_SIZE || (opts->flags & ~allowed) != 0)
     return TRI_ATTN_ERR_INVALID_ARG;
   const void *res = opt_residual(opts);
   if (res && !aligned16(res)) return TRI_ATTN_ERR_INVALID_ARG;
@@ -343,7 +376,9 @@ tri_attn_status tri_attn_bwd_workspace_size(const tri_attn_problem *prob, size_t
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
   if (!bytes) return TRI_ATTN_ERR_INVALID_ARG;
-  *bytes = carve_bwd(prob, nullptr, true, nullptr);
+  // large enough for either backward path (TRI_ATTN_OPT_ONCHIP_SUMS or not)
+  *bytes = std::max(carve_bwd(prob, nullptr, true, false, nullptr),
+                    carve_bwd(prob, nullptr, true, true, nullptr));
   return TRI_ATTN_OK;
 }
 
@@ -354,7 +389,7 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
                                 const tri_attn_launch_opts *opts) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  st = check_opts(prob, opts);
+  st = check_opts(prob, opts, 0u);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
@@ -431,14 +466,17 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                 tri_attn_stream_t stream_, const tri_attn_launch_opts *opts) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  st = check_opts(prob, opts);
+  st = check_opts(prob, opts, TRI_ATTN_OPT_ONCHIP_SUMS);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
     return TRI_ATTN_ERR_WORKSPACE;
   const bool per_row = mask && prob->mask_row_stride == prob->N;
+  const bool onchip = opts && (opts->flags & TRI_ATTN_OPT_ONCHIP_SUMS) != 0;
+  if (onchip && prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_INVALID_ARG;
   BwdWs w;
-  if (workspace_bytes < carve_bwd(prob, workspace, per_row, &w)) return TRI_ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < carve_bwd(prob, workspace, per_row, onchip, &w))
+    return TRI_ATTN_ERR_WORKSPACE;
   if (prob->N == 0) return TRI_ATTN_OK;
   TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
   TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse); TRI_CHECK_PTR(dout);
@@ -473,8 +511,67 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   const int64_t words = mask_words_per_row(prob);
   const int64_t rows = mask_rows(prob, mask != nullptr);
   const bool x_inner = prob->variant == TRI_ATTN_STARTING;
-  const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.fw.biasT : bias;
   const int64_t N = prob->N, H = prob->H;
+  const float scale = 1.0f / sqrtf((float)prob->c);
+
+  if (w.tc) {
+    tri::BwdMaps maps;
+    if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner) ||
+        !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner) ||
+        !encode_pair(&maps.v, v, N, H, f.sR, f.sX, x_inner) ||
+        !encode_pair(&maps.du, w.du, N, H, N * H * 32, H * 32, true))
+      return TRI_ATTN_ERR_CUDA;
+    tri::BwdTcArgs a{};
+    a.N = f.N;
+    a.H = f.H;
+    a.x_inner = x_inner ? 1 : 0;
+    a.nb = w.ntile;
+    a.ngroups = w.ngroups;
+    a.rows_per_group = (f.N + w.ngroups - 1) / w.ngroups;
+    a.scale = scale;
+    a.sR = f.sR;
+    a.sX = f.sX;
+    a.bX = f.bX;
+    a.bY = f.bY;
+    a.bias = static_cast<const __nv_bfloat16 *>(bias);
+    a.LD = reinterpret_cast<const float4 *>(w.LD);
+    a.mask_bits = w.fw.mask_bits;
+    a.mask_bits_stride = rows > 1 ? words : 0;
+    a.dq = static_cast<__nv_bfloat16 *>(dq);
+    a.dk = static_cast<__nv_bfloat16 *>(dk);
+    a.dv = static_cast<__nv_bfloat16 *>(dv);
+    a.dbias = static_cast<__nv_bfloat16 *>(dbias);
+    a.part_db = w.part_db;
+    a.ring = w.ring;
+    const int64_t gh_total = (int64_t)w.ngroups * H, nb = w.ntile;
+    a.exported = w.flags;
+    a.consumed_q = w.flags + gh_total * nb * nb;
+    a.consumed_kv = a.consumed_q + gh_total * nb * tri::bwd_tc_consumed_flags_per_tile();
+    a.status = w.fw.status;
+    // mask bits, status reset and the exchange flags zeroed in one launch
+    cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, w.flags,
+                                          w.nflags, stream);
+    if (e == cudaSuccess)
+      e = tri::launch_bwd_pre_bf16(f, static_cast<const __nv_bfloat16 *>(gate),
+                                   static_cast<const __nv_bfloat16 *>(out),
+                                   static_cast<const __nv_bfloat16 *>(opt_residual(opts)),
+                                   static_cast<const __nv_bfloat16 *>(dout),
+                                   static_cast<__nv_bfloat16 *>(w.du), nullptr,
+                                   static_cast<__nv_bfloat16 *>(dgate), lse, w.LD, stream);
+    if (e == cudaSuccess) e = mark(opts, true, stream);
+    for (int64_t gh0 = 0; e == cudaSuccess && gh0 < gh_total; gh0 += w.ghl) {
+      a.gh0 = (int)gh0;
+      a.ghl = (int)std::min<int64_t>(w.ghl, gh_total - gh0);
+      e = tri::launch_bwd_tc(maps, a, stream);
+    }
+    if (e == cudaSuccess) e = mark(opts, false, stream);
+    if (e == cudaSuccess && w.ngroups > 1)
+      e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, w.ngroups,
+                                                 static_cast<__nv_bfloat16 *>(dbias), stream);
+    return cuda_status(e);
+  }
+
+  const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.fw.biasT : bias;
   tri::BwdMaps maps;
   if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner) ||
       !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner) ||
@@ -487,7 +584,7 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   a.H = f.H;
   a.x_inner = x_inner ? 1 : 0;
   a.nb = w.ntile;
-  a.scale = 1.0f / sqrtf((float)prob->c);
+  a.scale = scale;
   a.sR = f.sR;
   a.sX = f.sX;
   a.lse = lse;
@@ -516,7 +613,7 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                  static_cast<const __nv_bfloat16 *>(opt_residual(opts)),
                                  static_cast<const __nv_bfloat16 *>(dout),
                                  static_cast<__nv_bfloat16 *>(w.du), w.D,
-                                 static_cast<__nv_bfloat16 *>(dgate), stream);
+                                 static_cast<__nv_bfloat16 *>(dgate), nullptr, nullptr, stream);
   if (e == cudaSuccess) e = mark(opts, true, stream);
   if (e == cudaSuccess) e = tri::launch_bwd_bf16(maps, a, stream);
   if (e == cudaSuccess) e = mark(opts, false, stream);
@@ -545,8 +642,9 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
                                          int has_mask, int32_t *launches) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  if (!launches) return TRI_ATTN_ERR_INVALID_ARG;
+  if (!launches || backward < 0 || backward > 2) return TRI_ATTN_ERR_INVALID_ARG;
   (void)has_mask;
+  const bool onchip = backward == 2;
   int32_t n = 0;
   if (prob->N > 0) {
     if (prob->dtype == TRI_ATTN_F32) {
@@ -554,7 +652,7 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
         n = 1;
       } else {
         BwdWs w;
-        carve_bwd(prob, nullptr, false, &w);
+        carve_bwd(prob, nullptr, false, false, &w);
         n = 5 + (w.ngroups > 1 ? 1 : 0);  // pre, main, three reductions, dbias reduction
       }
     } else {
@@ -563,9 +661,16 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
         n = 2 + ending;  // mask bits, [bias transpose], main
       } else {
         BwdWs w;
-        carve_bwd(prob, nullptr, false, &w);
-        // mask bits, [transpose], pre, main, partial reduction, [dbias reduction]
-        n = 4 + ending + (w.ngroups > 1 ? 1 : 0);
+        carve_bwd(prob, nullptr, false, onchip, &w);
+        if (w.tc) {
+          // mask bits, pre, one main launch per group of (group, head) pairs,
+          // [dbias reduction]
+          const int64_t gh = (int64_t)w.ngroups * prob->H;
+          n = 2 + (int32_t)((gh + w.ghl - 1) / w.ghl) + (w.ngroups > 1 ? 1 : 0);
+        } else {
+          // mask bits, [transpose], pre, main, partial reduction, [dbias reduction]
+          n = 4 + ending + (w.ngroups > 1 ? 1 : 0);
+        }
       }
     }
   }

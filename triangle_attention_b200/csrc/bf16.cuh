@@ -71,6 +71,41 @@ struct BwdArgs {
 void bwd_bf16_plan(int N, int H, int *nxb, int *ngroups);
 cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream_t stream);
 
+// ------------------------------------------- backward with on-chip sums --
+// The backward whose cross-tile sums of dq, dk and dv run inside the kernel
+// (bwd_tc.cu). One CTA per (query tile X, key tile Y, local group-head pair z);
+// the CTAs of one pair exchange their gradient blocks through `ring` and the
+// integer flags, so all CTAs of a launch must be resident at once.
+struct BwdTcArgs {
+  int N, H;
+  int x_inner;
+  int nb;                            // tiles per axis, ceil(N / 128) (at most 12)
+  int ngroups, rows_per_group;       // attention rows split into groups
+  int gh0, ghl;                      // first (group, head) pair of this launch, pairs in it
+  float scale;
+  int64_t sR, sX;                    // pair strides of the variant frame (outputs)
+  int64_t bX, bY;                    // bias and dbias strides of the variant frame
+  const __nv_bfloat16 *bias;         // the caller's bias (variant frame through bX, bY)
+  const float4 *LD;                  // [N][H][N/2]: (-lse*log2e) and (-D) of query pairs
+  const uint32_t *mask_bits;
+  int64_t mask_bits_stride;
+  __nv_bfloat16 *dq, *dk, *dv;       // results (variant frame strides)
+  __nv_bfloat16 *dbias;              // ngroups == 1
+  float *part_db;                    // [ngroups][H, N, N] (ngroups > 1)
+  __nv_bfloat16 *ring;               // [slots][ghl][3][nb][nb][4][128][8] gradient blocks
+  int32_t *exported;                 // [ngroups*H][nb][nb] rows exported per CTA
+  int32_t *consumed_q, *consumed_kv; // [ngroups*H][nb][slots][2] rows summed, per owner warp
+  int32_t *status;
+};
+
+int bwd_tc_ring_slots();
+// Consumed flags per output tile (ring slots x owner warps).
+int bwd_tc_consumed_flags_per_tile();
+// Tiling of the on-chip-sum backward for `sms` SMs; false when it does not
+// apply (more than 12 tiles per axis, odd N, or more CTAs per pair than SMs).
+bool bwd_tc_plan(int N, int H, int sms, int *nb, int *ngroups, int *gh_per_launch);
+cudaError_t launch_bwd_tc(const BwdMaps &maps, const BwdTcArgs &args, cudaStream_t stream);
+
 // ------------------------------------------------------------ preparation --
 // Packs the key mask of every attention row into bits (0 beyond N), resets the
 // status word and zeroes `nzero` int32 words at `zero` (counters; may be 0).
@@ -89,10 +124,13 @@ cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part
 // du (compact variant frame, bf16) = dout * sigmoid(g); D = sum_c dout * out;
 // dgate (storage layout) = dout * out * (1 - sigmoid(g)); out + out_res in
 // place of out when out_res (the forward's rounding residual) is given.
+// With lse and LD given (the on-chip-sum backward), D goes into LD instead:
+// LD[(r*H + h)*(N/2) + x/2] = (-lse*log2e of x, x+1; -D of x, x+1), with an
+// exponent of -inf for a query whose lse is -inf (all keys masked).
 cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
                                 const __nv_bfloat16 *out, const __nv_bfloat16 *out_res,
                                 const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
-                                cudaStream_t stream);
+                                const float *lse, float *LD, cudaStream_t stream);
 
 }  // namespace tri

@@ -69,7 +69,9 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
                                     const __nv_bfloat16 *__restrict__ out_res,
                                     const __nv_bfloat16 *__restrict__ dout,
                                     __nv_bfloat16 *__restrict__ du, float *__restrict__ D,
-                                    __nv_bfloat16 *__restrict__ dgate, int ending) {
+                                    __nv_bfloat16 *__restrict__ dgate,
+                                    const float *__restrict__ lse, float *__restrict__ LD,
+                                    int ending) {
   const int64_t total = (int64_t)f.N * f.N * f.H * 4;
   const unsigned group = 0xfu << (threadIdx.x & 28);   // the 4 lanes of one (a, b, h)
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
@@ -110,7 +112,18 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
     // fixed combination order: (q0 + q1) + (q2 + q3)
     d += __shfl_xor_sync(group, d, 1);
     d += __shfl_xor_sync(group, d, 2);
-    if (q == 0) D[(r * f.H + h) * f.N + x] = d;
+    if (q == 0) {
+      const int64_t rx = (r * f.H + h) * f.N + x;
+      if (LD) {
+        // (-lse*log2e of the query pair, -D of the pair) in one 16-byte group
+        const float l = lse[rx];
+        float *p = LD + ((r * f.H + h) * (f.N / 2) + (x >> 1)) * 4 + (x & 1);
+        p[0] = l == -INFINITY ? -INFINITY : -l * 1.4426950408889634f;
+        p[2] = -d;
+      } else {
+        D[rx] = d;
+      }
+    }
   }
 }
 
@@ -199,12 +212,12 @@ cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
                                 const __nv_bfloat16 *out, const __nv_bfloat16 *out_res,
                                 const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
-                                cudaStream_t stream) {
+                                const float *lse, float *LD, cudaStream_t stream) {
   const int64_t total = (int64_t)f.N * f.N * f.H * 4;
   if (total == 0) return cudaSuccess;
   const int ending = f.variant == 1 ? 1 : 0;
   bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, out_res, dout,
-                                                                  du, D, dgate, ending);
+                                                                  du, D, dgate, lse, LD, ending);
   return cudaGetLastError();
 }
 

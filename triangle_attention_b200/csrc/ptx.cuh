@@ -176,6 +176,24 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t *p, int v) {
   return old;
 }
 
+// Acquire load / release store of a flag at GPU scope: writes made before the
+// release (and, by cumulativity, writes the releasing thread observed through a
+// CTA barrier) are visible to a thread whose acquire load reads the value.
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t *p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t *p, int32_t v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's generic-proxy view of global memory with later
+// async-proxy (bulk copy) accesses of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 32-byte streaming store (eight 32-bit words, 32-byte aligned address).
 __device__ __forceinline__ void st_global_cs_v8(void *p, const uint32_t (&v)[8]) {
   asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
@@ -336,6 +354,20 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (
       : TRI_RA8(0), TRI_RA8(8), TRI_RA8(16), TRI_RA8(24), TRI_RB8(0), TRI_RB8(8), TRI_RB8(16),
         TRI_RB8(24)
       : "r"(ta), "r"(tb)
+      : "memory");
+}
+
+// Three 8-column loads with a single wait.
+__device__ __forceinline__ void tmem_ld8x3(uint32_t ta, uint32_t tb, uint32_t tc,
+                                           uint32_t (&a)[8], uint32_t (&b_)[8],
+                                           uint32_t (&c_)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%24];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%25];\n"
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16,%17,%18,%19,%20,%21,%22,%23}, [%26];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : TRI_RA8(0), TRI_RB8(0), TRI_RC8(0)
+      : "r"(ta), "r"(tb), "r"(tc)
       : "memory");
 }
 
