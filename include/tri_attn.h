@@ -271,6 +271,18 @@ tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_stat
                                      tri_attn_stream_t stream);
 
 /*
+ * The same device status word returned as the call's own status: synchronises
+ * the stream and returns what the last call that used this workspace recorded
+ * on the device (TRI_ATTN_OK, TRI_ATTN_ERR_TIMEOUT for a bounded wait that ran
+ * out, TRI_ATTN_ERR_BOUNDS for a tile the kernel refused). Returns
+ * TRI_ATTN_ERR_INVALID_ARG for a NULL workspace and TRI_ATTN_ERR_CUDA if the
+ * synchronisation or the copy fails. The workspace is caller-owned device
+ * memory laid out by tri_attn_fwd / tri_attn_bwd (the word sits at offset 0).
+ * The pages define no status channel; this is the boundary's query call.
+ */
+tri_attn_status tri_attn_get_status(const void *workspace, tri_attn_stream_t stream);
+
+/*
  * Diagnostic of the failure path (no counterpart on the pages): enqueues one
  * small kernel whose warp waits on a barrier that nothing ever completes,
  * using the same bounded wait (about 2 s) as the forward and backward kernels.

@@ -164,6 +164,7 @@ def test_onchip_sum_option_on_the_host(lib):
 def test_read_status_rejects_null(lib):
     v = ctypes.c_int32(0)
     assert lib.tri_attn_read_status(None, ctypes.byref(v), None) == 1
+    assert lib.tri_attn_get_status(None, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -66,3 +66,4 @@ def test_status_word_is_clean_after_calls():
            STARTING, ws=ws_b)
     assert ta.read_status(ws_f) == 0
     assert ta.read_status(ws_b) == 0
+    assert ta.get_status(ws_f) == 0 and ta.get_status(ws_b) == 0

@@ -27,6 +27,8 @@ def test_unsatisfied_wait_reports_timeout_and_context_survives():
     ws = ta.workspace(256, torch.device("cuda:0"))
     assert ta.check_wait_timeout(ws) == TIMEOUT
     assert ta.STATUS[TIMEOUT] == "device wait timed out"
+    # the same word through the query call of the boundary
+    assert ta.get_status(ws) == TIMEOUT
     # the same context runs a normal forward and backward afterwards
     g = to_device(make_inputs(136, H=2, c=32, dtype="bf16", seed=3), "cuda:0")
     prob = ta.problem(g["q"], g["mask"], STARTING)
@@ -35,4 +37,5 @@ def test_unsatisfied_wait_reports_timeout_and_context_survives():
     ta.bwd(g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], out, lse, g["dout"],
            STARTING, ws=ws_b)
     assert ta.read_status(ws_b) == 0
+    assert ta.get_status(ws_b) == 0
     assert torch.isfinite(lse).all()

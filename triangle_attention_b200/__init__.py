@@ -124,6 +124,7 @@ def lib():
         L.tri_attn_kernel_launches.argtypes = [PP, ctypes.c_int, ctypes.c_int,
                                                ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
+        L.tri_attn_get_status.argtypes = [P, P]
         L.tri_attn_check_wait_timeout.argtypes = [P, sz, P]
         MP = ctypes.POINTER(MulProblem)
         L.tri_mul_workspace_size.argtypes = [MP, ctypes.POINTER(sz)]
@@ -137,7 +138,7 @@ def lib():
         L.tri_proj_out_bwd.argtypes = [JP] + [P] * 6 + [P, sz, P]
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
-                  L.tri_attn_kernel_launches, L.tri_attn_read_status,
+                  L.tri_attn_kernel_launches, L.tri_attn_read_status, L.tri_attn_get_status,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
                   L.tri_mul_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
                   L.tri_proj_in_bwd, L.tri_proj_out_fwd, L.tri_proj_out_bwd):
@@ -273,6 +274,16 @@ def read_status(ws: torch.Tensor, stream=None) -> int:
     _check(lib().tri_attn_read_status(_p(ws), ctypes.byref(v), _stream(stream)),
            "tri_attn_read_status")
     return v.value
+
+
+def get_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronises the stream and returns the device status word of the last
+    call that used this workspace as a status code (0 = ok); raises only if the
+    query itself fails."""
+    code = lib().tri_attn_get_status(_p(ws), _stream(stream))
+    if code == 4:
+        _check(code, "tri_attn_get_status")
+    return code
 
 
 def check_wait_timeout(ws: torch.Tensor, stream=None) -> int:

@@ -690,6 +690,12 @@ tri_attn_status tri_attn_read_status(const void *workspace, int32_t *device_stat
   return TRI_ATTN_OK;
 }
 
+tri_attn_status tri_attn_get_status(const void *workspace, tri_attn_stream_t stream) {
+  int32_t v = 0;
+  const tri_attn_status st = tri_attn_read_status(workspace, &v, stream);
+  return st != TRI_ATTN_OK ? st : static_cast<tri_attn_status>(v);
+}
+
 tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
                                             tri_attn_stream_t stream) {
   if (!workspace || !aligned16(workspace) || workspace_bytes < 256)
