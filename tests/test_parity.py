@@ -1,6 +1,6 @@
 """Parity of the CUDA path with the fp64 oracle on identical seeded inputs.
 
-Full-tensor comparisons up to N=384 (every output element), sampled rows and
+Full-tensor comparisons up to N=640 (every output element), sampled rows and
 sampled dbias entries at N=768 and N=1536 (the oracle computes those one by
 one), ragged sizes that leave a partial 128-tile, per-row masks with a fully
 masked row, both variants, both dtypes."""
@@ -101,10 +101,30 @@ def test_bf16_small_and_tile_edges(N, H):
     full_check(d, STARTING, "bf16")
 
 
+def test_bf16_n512_full_two_row_groups():
+    """bf16, N=512, H=4 (4 tiles per axis): every output element. The backward
+    splits each head's 512 rows into two row groups here (16 tiles x 4 heads
+    fill 64 of the SMs twice), so the cross-group dbias sum and the multi-tile
+    contribution sums run at a size where all of them matter."""
+    d = make_inputs(512, H=4, c=32, dtype="bf16", seed=30, mask="random:51")
+    full_check(d, STARTING, "bf16")
+
+
+def test_bf16_n640_ending_full():
+    """bf16 ending node, N=640, H=2 (5 tiles per axis, two row groups per
+    head), trailing keys masked: every output element."""
+    d = make_inputs(640, H=2, c=32, dtype="bf16", seed=31, mask="trailing:40")
+    full_check(d, ENDING, "bf16")
+
+
 def test_bf16_n768_workload_sampled():
-    """bf16, N=768, H=4, c=32, no mask (the headline size): sampled rows of every
-    pair output and 64 sampled dbias entries (each summed over all 768 rows)."""
-    sampled_check(workload_inputs("n768_bf16"), STARTING, rows=[0, 257, 511, 767])
+    """bf16, N=768, H=4, c=32, no mask (the headline size): the attention rows on
+    both sides of every 128-row tile edge (the backward's row groups, the
+    forward's 8-row groups and the 128-query tiles all change there) plus a
+    middle row, every pair output of them, and 64 sampled dbias entries (each
+    summed over all 768 rows)."""
+    rows = [0, 127, 128, 255, 256, 257, 383, 384, 511, 512, 639, 640, 767]
+    sampled_check(workload_inputs("n768_bf16"), STARTING, rows=rows)
 
 
 def test_bf16_n1536_forward_sampled():
