@@ -225,6 +225,54 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
 tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backward,
                                          int has_mask, int32_t *launches);
 
+/*
+ * Row shards, for splitting one problem across GPUs (one process per GPU). The
+ * attention rows are independent problems that share only the pair bias, whose
+ * gradient dbias[h, x, y] sums over every row: the row-wise split of the pair
+ * representation across devices ("FastFold: Reducing AlphaFold Training Time
+ * from 11 Days to 67 Hours", methods, Dynamic Axial Parallelism) applied to this
+ * one operation. A shard is the rows [row_begin, row_begin + row_count) of the
+ * variant frame (the first residue index for the starting node, the second for
+ * the ending node); row_begin and row_count are multiples of 8 (else
+ * TRI_ATTN_ERR_INVALID_ARG); bf16 only (fp32: TRI_ATTN_ERR_UNSUPPORTED).
+ * Every pointer is the full [N, N, H, c] / [H, N, N] / [N, H, N] tensor as for
+ * tri_attn_fwd / tri_attn_bwd; a shard call reads what its rows need (all keys
+ * of its rows, and the whole bias) and writes only its rows of out, lse, dq, dk,
+ * dv and dgate. Workspace: the sizes tri_attn_fwd_workspace_size and
+ * tri_attn_bwd_workspace_size report. Results on a shard's rows are
+ * bit-identical to those of the whole-problem call.
+ */
+tri_attn_status tri_attn_fwd_rows(const tri_attn_problem *prob, int64_t row_begin,
+                                  int64_t row_count, const void *q, const void *k, const void *v,
+                                  const void *bias, const void *gate, const uint8_t *mask,
+                                  void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                  tri_attn_stream_t stream);
+
+/*
+ * Backward of a row shard. Instead of dbias it writes dbias_partial (device,
+ * caller-owned, fp32, [H, N, N] in the layout of dbias): the sum over the
+ * shard's rows, in a fixed order. The full dbias is the sum of every shard's
+ * partial; tri_attn_dbias_reduce adds gathered partials in rank order and rounds
+ * to bf16 once, so every rank obtains the same bits.
+ */
+tri_attn_status tri_attn_bwd_rows(const tri_attn_problem *prob, int64_t row_begin,
+                                  int64_t row_count, const void *q, const void *k, const void *v,
+                                  const void *bias, const void *gate, const uint8_t *mask,
+                                  const void *out, const float *lse, const void *dout, void *dq,
+                                  void *dk, void *dv, float *dbias_partial, void *dgate,
+                                  void *workspace, size_t workspace_bytes,
+                                  tri_attn_stream_t stream);
+
+/*
+ * dbias (bf16, [H, N, N]) = sum over i = 0 .. count-1, in that order, of the fp32
+ * partials[i] ([count][H][N][N], contiguous, 16-byte aligned; the all-gathered
+ * outputs of tri_attn_bwd_rows in rank order), rounded once. One kernel,
+ * asynchronous on `stream`. TRI_ATTN_ERR_INVALID_ARG for count < 1, a bad N or
+ * H, or NULL / misaligned pointers.
+ */
+tri_attn_status tri_attn_dbias_reduce(const float *partials, int32_t count, int64_t N, int32_t H,
+                                      void *dbias, tri_attn_stream_t stream);
+
 /* Size of the fixed scratch area behind tri_attn_fwd_noalloc, per GPU. */
 #define TRI_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 

@@ -125,6 +125,10 @@ def lib():
                                                ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.tri_attn_get_status.argtypes = [P, P]
+        i64 = ctypes.c_int64
+        L.tri_attn_fwd_rows.argtypes = [PP, i64, i64, P, P, P, P, P, P, P, P, P, sz, P]
+        L.tri_attn_bwd_rows.argtypes = [PP, i64, i64] + [P] * 15 + [sz, P]
+        L.tri_attn_dbias_reduce.argtypes = [P, ctypes.c_int32, i64, ctypes.c_int32, P, P]
         L.tri_attn_check_wait_timeout.argtypes = [P, sz, P]
         MP = ctypes.POINTER(MulProblem)
         L.tri_mul_workspace_size.argtypes = [MP, ctypes.POINTER(sz)]
@@ -139,6 +143,7 @@ def lib():
         for f in (L.tri_attn_fwd_workspace_size, L.tri_attn_bwd_workspace_size, L.tri_attn_fwd,
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
                   L.tri_attn_kernel_launches, L.tri_attn_read_status, L.tri_attn_get_status,
+                  L.tri_attn_fwd_rows, L.tri_attn_bwd_rows, L.tri_attn_dbias_reduce,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
                   L.tri_mul_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
                   L.tri_proj_in_bwd, L.tri_proj_out_fwd, L.tri_proj_out_bwd):
@@ -265,6 +270,96 @@ def bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, grad
                                  None if opts is None else ctypes.byref(opts)),
            "tri_attn_bwd")
     return dq, dk, dv, dbias, dgate
+
+
+# ------------------------------------------------------------ row shards --
+
+def shard_rows(N: int, world: int, rank: int) -> tuple:
+    """(row_begin, row_count) of rank `rank` when the N attention rows are split
+    into `world` contiguous shards of whole 8-row groups; the first
+    (N/8) mod world ranks take one group more."""
+    if world < 1 or not 0 <= rank < world or N % 8:
+        raise ValueError(f"cannot shard N={N} rows over {world} ranks (rank {rank})")
+    base, extra = divmod(N // 8, world)
+    begin = 8 * (rank * base + min(rank, extra))
+    return begin, 8 * (base + (1 if rank < extra else 0))
+
+
+def fwd_rows(q, k, v, bias, gate, mask, variant: int, row_begin: int, row_count: int,
+             out=None, lse=None, ws=None, stream=None):
+    """Forward of the attention rows [row_begin, row_begin + row_count) (bf16).
+    Inputs and outputs are the full tensors; only the shard's rows of out and
+    lse are written (the rest of freshly allocated outputs is undefined)."""
+    _contig(q, k, v, bias, gate, mask)
+    prob = problem(q, mask, variant)
+    N, H = q.shape[0], q.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((N, H, N), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(fwd_workspace_size(prob), q.device)
+    _check(lib().tri_attn_fwd_rows(ctypes.byref(prob), row_begin, row_count, _p(q), _p(k), _p(v),
+                                   _p(bias), _p(gate), _p(mask), _p(out), _p(lse), _p(ws),
+                                   ws.numel(), _stream(stream)), "tri_attn_fwd_rows")
+    return out, lse
+
+
+def bwd_rows(q, k, v, bias, gate, mask, out, lse, dout, variant: int, row_begin: int,
+             row_count: int, grads=None, ws=None, stream=None):
+    """Backward of a row shard. Returns (dq, dk, dv, dbias_partial, dgate): the
+    shard's rows of the pair gradients (full tensors, other rows untouched) and
+    the fp32 [H, N, N] sum of dbias over the shard's rows."""
+    _contig(q, k, v, bias, gate, mask, out, lse, dout)
+    prob = problem(q, mask, variant)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v),
+                 torch.empty(bias.shape, dtype=torch.float32, device=q.device),
+                 torch.empty_like(gate))
+    dq, dk, dv, dbp, dgate = grads
+    if ws is None:
+        ws = workspace(bwd_workspace_size(prob), q.device)
+    _check(lib().tri_attn_bwd_rows(ctypes.byref(prob), row_begin, row_count, _p(q), _p(k), _p(v),
+                                   _p(bias), _p(gate), _p(mask), _p(out), _p(lse), _p(dout),
+                                   _p(dq), _p(dk), _p(dv), _p(dbp), _p(dgate), _p(ws), ws.numel(),
+                                   _stream(stream)), "tri_attn_bwd_rows")
+    return dq, dk, dv, dbp, dgate
+
+
+def dbias_reduce(partials: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """bf16 dbias [H, N, N] = the fp32 partials [W, H, N, N] summed over W in
+    index order (rank order) and rounded once, on the GPU."""
+    _contig(partials)
+    W, H, N, _ = partials.shape
+    if out is None:
+        out = torch.empty((H, N, N), dtype=torch.bfloat16, device=partials.device)
+    _check(lib().tri_attn_dbias_reduce(_p(partials), W, N, H, _p(out), _stream(stream)),
+           "tri_attn_dbias_reduce")
+    return out
+
+
+def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
+    """[W, ...] stack of every rank's `partial`, in rank order (torch.distributed
+    all_gather; NCCL on GPUs, any backend's tensors work)."""
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    parts = [torch.empty_like(partial) for _ in range(world)]
+    dist.all_gather(parts, partial.contiguous(), group=group)
+    return torch.stack(parts)
+
+
+def sharded_bwd(q, k, v, bias, gate, mask, out, lse, dout, variant: int = STARTING, group=None,
+                ws=None, stream=None):
+    """Backward of one problem split by rows over the ranks of `group`: each
+    rank computes its shard's rows of dq, dk, dv and dgate, the dbias partials
+    are all-gathered and summed in rank order on the GPU, so every rank holds
+    the same full dbias. Returns (dq, dk, dv, dbias, dgate, (row_begin, row_count))."""
+    import torch.distributed as dist
+    rows = shard_rows(q.shape[0], dist.get_world_size(group), dist.get_rank(group))
+    dq, dk, dv, dbp, dgate = bwd_rows(q, k, v, bias, gate, mask, out, lse, dout, variant,
+                                      rows[0], rows[1], ws=ws, stream=stream)
+    dbias = dbias_reduce(gather_partials(dbp, group), stream=stream)
+    return dq, dk, dv, dbias, dgate, rows
 
 
 def read_status(ws: torch.Tensor, stream=None) -> int:

@@ -62,6 +62,8 @@ Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status
   f.mask = mask;
   f.mask_stride = mask ? p->mask_row_stride : 0;
   f.status = status;
+  f.row0 = 0;
+  f.row_end = (int)p->N;
   return f;
 }
 
@@ -161,7 +163,7 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
     } else {
       if (p->variant == TRI_ATTN_ENDING)
         w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
-      tri::bwd_bf16_plan((int)p->N, p->H, &w.ntile, &w.ngroups);
+      tri::bwd_bf16_plan((int)p->N, p->H, (int)p->N, &w.ntile, &w.ngroups);
       w.du = c.take(2 * pair);
       w.D = static_cast<float *>(c.take(4 * nn * p->H));
       w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
@@ -176,8 +178,16 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
     w.part_dk = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
     w.part_dv = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
   }
-  w.part_db = w.ngroups > 1 ? static_cast<float *>(c.take(4 * nn * p->H * (size_t)w.ngroups))
-                            : nullptr;
+  if (p->dtype == TRI_ATTN_BF16 && !w.tc) {
+    // per-group dbias sums: also taken by a row-shard call, whose groups split
+    // fewer rows but never number more than bwd_bf16_max_groups
+    w.part_db = static_cast<float *>(
+        c.take(4 * nn * p->H * (size_t)tri::bwd_bf16_max_groups((int)p->N, p->H)));
+  } else {
+    w.part_db = w.ngroups > 1
+                    ? static_cast<float *>(c.take(4 * nn * p->H * (size_t)w.ngroups))
+                    : nullptr;
+  }
   if (out) *out = w;
   return c.off;
 }
@@ -382,11 +392,14 @@ tri_attn_status tri_attn_bwd_workspace_size(const tri_attn_problem *prob, size_t
   return TRI_ATTN_OK;
 }
 
-tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
-                                const void *v, const void *bias, const void *gate,
-                                const uint8_t *mask, void *out, float *lse, void *workspace,
-                                size_t workspace_bytes, tri_attn_stream_t stream_,
-                                const tri_attn_launch_opts *opts) {
+namespace {
+
+// Forward over the attention rows [row0, row0 + row_count) (validated by the caller).
+tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void *k,
+                         const void *v, const void *bias, const void *gate, const uint8_t *mask,
+                         void *out, float *lse, void *workspace, size_t workspace_bytes,
+                         tri_attn_stream_t stream_, const tri_attn_launch_opts *opts,
+                         int64_t row0, int64_t row_count) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
   st = check_opts(prob, opts, 0u);
@@ -400,9 +413,13 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   if (prob->N == 0) return TRI_ATTN_OK;
   TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
   TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse);
-  const Frame f = make_frame(prob, mask, w.status);
+  Frame f = make_frame(prob, mask, w.status);
+  f.row0 = (int)row0;
+  f.row_end = (int)(row0 + row_count);
+  if (row_count == 0) return TRI_ATTN_OK;
 
   if (prob->dtype == TRI_ATTN_F32) {
+    if (row0 != 0 || row_count != prob->N) return TRI_ATTN_ERR_UNSUPPORTED;
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
     if (e == cudaSuccess) e = mark(opts, true, stream);
     if (e == cudaSuccess)
@@ -428,6 +445,8 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   tri::FwdArgs a;
   a.N = f.N;
   a.H = f.H;
+  a.row0 = f.row0;
+  a.row_end = f.row_end;
   a.x_inner = x_inner ? 1 : 0;
   a.scale = 1.0f / sqrtf((float)prob->c);
   a.sR = f.sR;
@@ -450,6 +469,17 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
   return cuda_status(e);
 }
 
+}  // namespace
+
+tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, void *out, float *lse, void *workspace,
+                                size_t workspace_bytes, tri_attn_stream_t stream,
+                                const tri_attn_launch_opts *opts) {
+  return fwd_impl(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes, stream,
+                  opts, 0, prob ? prob->N : 0);
+}
+
 tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
                              const void *v, const void *bias, const void *gate,
                              const uint8_t *mask, void *out, float *lse, void *workspace,
@@ -458,12 +488,17 @@ tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const 
                          stream, nullptr);
 }
 
-tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
-                                const void *v, const void *bias, const void *gate,
-                                const uint8_t *mask, const void *out, const float *lse,
-                                const void *dout, void *dq, void *dk, void *dv, void *dbias,
-                                void *dgate, void *workspace, size_t workspace_bytes,
-                                tri_attn_stream_t stream_, const tri_attn_launch_opts *opts) {
+namespace {
+
+// Backward over the attention rows [row0, row0 + row_count) (validated by the
+// caller). dbias_partial != NULL: the fp32 sum of dbias over these rows goes
+// there instead of the bf16 dbias.
+tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void *k,
+                         const void *v, const void *bias, const void *gate, const uint8_t *mask,
+                         const void *out, const float *lse, const void *dout, void *dq, void *dk,
+                         void *dv, void *dbias, float *dbias_partial, void *dgate,
+                         void *workspace, size_t workspace_bytes, tri_attn_stream_t stream_,
+                         const tri_attn_launch_opts *opts, int64_t row0, int64_t row_count) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
   st = check_opts(prob, opts, TRI_ATTN_OPT_ONCHIP_SUMS);
@@ -480,11 +515,20 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   if (prob->N == 0) return TRI_ATTN_OK;
   TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
   TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse); TRI_CHECK_PTR(dout);
-  TRI_CHECK_PTR(dq); TRI_CHECK_PTR(dk); TRI_CHECK_PTR(dv); TRI_CHECK_PTR(dbias);
-  TRI_CHECK_PTR(dgate);
-  const Frame f = make_frame(prob, mask, w.fw.status);
+  TRI_CHECK_PTR(dq); TRI_CHECK_PTR(dk); TRI_CHECK_PTR(dv); TRI_CHECK_PTR(dgate);
+  if (dbias_partial) {
+    TRI_CHECK_PTR(dbias_partial);
+  } else {
+    TRI_CHECK_PTR(dbias);
+  }
+  Frame f = make_frame(prob, mask, w.fw.status);
+  f.row0 = (int)row0;
+  f.row_end = (int)(row0 + row_count);
+  const bool shard = dbias_partial != nullptr || row0 != 0 || row_count != prob->N;
+  if (row_count == 0) return TRI_ATTN_OK;
 
   if (prob->dtype == TRI_ATTN_F32) {
+    if (shard) return TRI_ATTN_ERR_UNSUPPORTED;
     tri::F32BwdScratch s;
     s.du = static_cast<float *>(w.du);
     s.D = w.D;
@@ -514,7 +558,7 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   const int64_t N = prob->N, H = prob->H;
   const float scale = 1.0f / sqrtf((float)prob->c);
 
-  if (w.tc) {
+  if (w.tc && !shard) {
     tri::BwdMaps maps;
     if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner) ||
         !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner) ||
@@ -579,11 +623,16 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
       !encode_pair(&maps.du, w.du, N, H, N * H * 32, H * 32, true) ||
       !encode_bias(&maps.bias, bias_frame, N, H))
     return TRI_ATTN_ERR_CUDA;
+  // row groups of this call's rows (the whole problem unless a row shard)
+  int ntile = w.ntile, ngroups = w.ngroups;
+  tri::bwd_bf16_plan(f.N, f.H, (int)row_count, &ntile, &ngroups);
   tri::BwdArgs a;
   a.N = f.N;
   a.H = f.H;
+  a.row0 = f.row0;
+  a.row_end = f.row_end;
   a.x_inner = x_inner ? 1 : 0;
-  a.nb = w.ntile;
+  a.nb = ntile;
   a.scale = scale;
   a.sR = f.sR;
   a.sX = f.sX;
@@ -595,11 +644,12 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
   a.part_k = w.bpart_k;
   a.part_v = w.bpart_v;
   a.part_db = w.part_db;
-  a.dbias = static_cast<__nv_bfloat16 *>(dbias);
+  // one row group over every row writes dbias itself; otherwise per-group fp32 sums
+  a.dbias = (!dbias_partial && ngroups == 1) ? static_cast<__nv_bfloat16 *>(dbias) : nullptr;
   a.bX = f.bX;
   a.bY = f.bY;
-  a.ngroups = w.ngroups;
-  a.rows_per_group = (f.N + w.ngroups - 1) / w.ngroups;
+  a.ngroups = ngroups;
+  a.rows_per_group = (int)((row_count + ngroups - 1) / ngroups);
   a.status = w.fw.status;
 
   cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, nullptr,
@@ -622,10 +672,83 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                         static_cast<__nv_bfloat16 *>(dq),
                                         static_cast<__nv_bfloat16 *>(dk),
                                         static_cast<__nv_bfloat16 *>(dv), stream);
-  if (e == cudaSuccess && w.ngroups > 1)
-    e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, w.ngroups,
+  if (e == cudaSuccess && dbias_partial)
+    e = tri::launch_bias_reduce<float>(f, w.part_db, ngroups, dbias_partial, stream);
+  else if (e == cudaSuccess && ngroups > 1)
+    e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, ngroups,
                                                static_cast<__nv_bfloat16 *>(dbias), stream);
   return cuda_status(e);
+}
+
+}  // namespace
+
+tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
+                                const void *v, const void *bias, const void *gate,
+                                const uint8_t *mask, const void *out, const float *lse,
+                                const void *dout, void *dq, void *dk, void *dv, void *dbias,
+                                void *dgate, void *workspace, size_t workspace_bytes,
+                                tri_attn_stream_t stream, const tri_attn_launch_opts *opts) {
+  return bwd_impl(prob, q, k, v, bias, gate, mask, out, lse, dout, dq, dk, dv, dbias, nullptr,
+                  dgate, workspace, workspace_bytes, stream, opts, 0, prob ? prob->N : 0);
+}
+
+namespace {
+// A row shard is a whole number of 8-row groups inside [0, N).
+tri_attn_status check_rows(const tri_attn_problem *prob, int64_t row_begin, int64_t row_count) {
+  if (!prob || row_begin < 0 || row_count < 0 || row_begin + row_count > prob->N)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (row_begin % 8 != 0 || row_count % 8 != 0) return TRI_ATTN_ERR_INVALID_ARG;
+  return TRI_ATTN_OK;
+}
+}  // namespace
+
+tri_attn_status tri_attn_fwd_rows(const tri_attn_problem *prob, int64_t row_begin,
+                                  int64_t row_count, const void *q, const void *k, const void *v,
+                                  const void *bias, const void *gate, const uint8_t *mask,
+                                  void *out, float *lse, void *workspace, size_t workspace_bytes,
+                                  tri_attn_stream_t stream) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  st = check_rows(prob, row_begin, row_count);
+  if (st != TRI_ATTN_OK) return st;
+  return fwd_impl(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes, stream,
+                  nullptr, row_begin, row_count);
+}
+
+tri_attn_status tri_attn_bwd_rows(const tri_attn_problem *prob, int64_t row_begin,
+                                  int64_t row_count, const void *q, const void *k, const void *v,
+                                  const void *bias, const void *gate, const uint8_t *mask,
+                                  const void *out, const float *lse, const void *dout, void *dq,
+                                  void *dk, void *dv, float *dbias_partial, void *dgate,
+                                  void *workspace, size_t workspace_bytes,
+                                  tri_attn_stream_t stream) {
+  tri_attn_status st = check_problem(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  st = check_rows(prob, row_begin, row_count);
+  if (st != TRI_ATTN_OK) return st;
+  if (!dbias_partial && prob->N > 0) return TRI_ATTN_ERR_INVALID_ARG;
+  return bwd_impl(prob, q, k, v, bias, gate, mask, out, lse, dout, dq, dk, dv, nullptr,
+                  dbias_partial, dgate, workspace, workspace_bytes, stream, nullptr, row_begin,
+                  row_count);
+}
+
+tri_attn_status tri_attn_dbias_reduce(const float *partials, int32_t count, int64_t N, int32_t H,
+                                      void *dbias, tri_attn_stream_t stream) {
+  if (count < 1 || N < 0 || N > kMaxN || H < 1 || (N > 0 && (!partials || !dbias)))
+    return TRI_ATTN_ERR_INVALID_ARG;
+  if (!aligned16(partials) || !aligned16(dbias)) return TRI_ATTN_ERR_INVALID_ARG;
+  if (N == 0) return TRI_ATTN_OK;
+  // the partials and dbias share one [H][N][N] layout: an identity frame
+  Frame f{};
+  f.N = (int)N;
+  f.H = H;
+  f.bX = N;
+  f.bY = 1;
+  return cuda_status(tri::launch_bias_reduce<__nv_bfloat16>(
+      f, partials, count, static_cast<__nv_bfloat16 *>(dbias),
+      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tri_attn_status tri_attn_bwd(const tri_attn_problem *prob, const void *q, const void *k,

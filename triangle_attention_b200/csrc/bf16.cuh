@@ -25,6 +25,7 @@ struct FwdMaps {
 
 struct FwdArgs {
   int N, H;
+  int row0, row_end;                 // attention rows of this launch (multiples of 8)
   int x_inner;                       // dimension order of the pair maps (see above)
   float scale;                       // c^-1/2
   int64_t sR, sX;                    // pair strides of the variant frame (elements)
@@ -50,6 +51,7 @@ struct BwdMaps {
 
 struct BwdArgs {
   int N, H;
+  int row0, row_end;                 // attention rows of this launch
   int x_inner;
   int nb;                            // tiles per axis, ceil(N / 128)
   float scale;
@@ -61,14 +63,17 @@ struct BwdArgs {
   // bf16 tile contributions, [tile][row][H][2][N][16] (16-channel halves):
   // part_q over key tiles yb, part_k and part_v over query tiles xb
   __nv_bfloat16 *part_q, *part_k, *part_v;
-  float *part_db;                    // [ngroups][H, N, N] variant frame (ngroups > 1)
-  __nv_bfloat16 *dbias;              // final dbias (ngroups == 1)
+  float *part_db;                    // [ngroups][H, N, N] variant frame (used when dbias is null)
+  __nv_bfloat16 *dbias;              // final dbias (one row group covering every row), else null
   int64_t bX, bY;                    // dbias strides of the variant frame
   int ngroups, rows_per_group;
   int32_t *status;
 };
 
-void bwd_bf16_plan(int N, int H, int *nxb, int *ngroups);
+// Tiling of the backward over `rows` attention rows: tiles per axis and row groups
+// (never more than bwd_bf16_max_groups(N, H)).
+void bwd_bf16_plan(int N, int H, int rows, int *nxb, int *ngroups);
+int bwd_bf16_max_groups(int N, int H);
 cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream_t stream);
 
 // ------------------------------------------- backward with on-chip sums --

@@ -219,8 +219,8 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int N = a.N, H = a.H;
   const int xb = blockIdx.x, yb = blockIdx.y;
   const int h = blockIdx.z % H, g = blockIdx.z / H;
-  const int r0 = g * a.rows_per_group;
-  const int r1 = min(N, r0 + a.rows_per_group);
+  const int r0 = a.row0 + g * a.rows_per_group;
+  const int r1 = min(a.row_end, r0 + a.rows_per_group);
   const int T = max(0, r1 - r0);
 
   if (threadIdx.x == 0) {
@@ -539,7 +539,7 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const int y = y0 + e + u;
           const float val = u ? v.y : v.x;
           if (y < N) {
-            if (a.ngroups == 1)
+            if (a.dbias)
               a.dbias[hb + (int64_t)x * a.bX + (int64_t)y * a.bY] = __float2bfloat16_rn(val);
             else
               a.part_db[((int64_t)g * H + h) * N * N + (int64_t)x * N + y] = val;
@@ -560,15 +560,22 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
 }  // namespace
 
-void bwd_bf16_plan(int N, int H, int *nxb, int *ngroups) {
+int bwd_bf16_max_groups(int N, int H) {
   const int nb = (N + kBM - 1) / kBM;
-  *nxb = nb;
   const int64_t tiles = (int64_t)nb * nb * H;
   int64_t g = tiles > 0 ? 148 / tiles : 1;
   if (g < 1) g = 1;
   if (g > N) g = N > 0 ? N : 1;
-  const int rows = (int)((N + g - 1) / g);
-  *ngroups = rows > 0 ? (N + rows - 1) / rows : 1;
+  return (int)g;
+}
+
+void bwd_bf16_plan(int N, int H, int rows, int *nxb, int *ngroups) {
+  const int nb = (N + kBM - 1) / kBM;
+  *nxb = nb;
+  int64_t g = bwd_bf16_max_groups(N, H);
+  if (g > rows) g = rows > 0 ? rows : 1;
+  const int per = (int)((rows + g - 1) / g);
+  *ngroups = per > 0 ? (rows + per - 1) / per : 1;
 }
 
 cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream_t stream) {

@@ -23,6 +23,9 @@ struct Frame {
   const uint8_t *mask;
   int64_t mask_stride;
   int32_t *status;  // device status word, never null inside a launch
+  // attention rows [row0, row_end) of the variant frame that this call computes
+  // (0 and N unless the caller asked for a row shard)
+  int row0, row_end;
 };
 
 // Record a device-side failure (first writer wins; the value never goes back

@@ -158,8 +158,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = a.N;
   const int xb = blockIdx.x, h = blockIdx.y;
-  const int r0 = blockIdx.z * kRows;
-  const int nrows = min(kRows, N - r0);
+  const int r0 = a.row0 + blockIdx.z * kRows;
+  const int nrows = min(kRows, a.row_end - r0);
   const int nkb = (N + kBN - 1) / kBN;
   const int T = nkb * kRows;        // (key tile, row) steps, row fastest
 
@@ -483,7 +483,7 @@ cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream
   cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((args.N + kBM - 1) / kBM, args.H, (args.N + kRows - 1) / kRows);
+  dim3 grid((args.N + kBM - 1) / kBM, args.H, (args.row_end - args.row0 + kRows - 1) / kRows);
   fwd_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k, maps.v, maps.bias,
                                                            args);
   return cudaGetLastError();

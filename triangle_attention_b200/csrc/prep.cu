@@ -83,6 +83,7 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
     const int64_t aa = e / ((int64_t)f.H * f.N);
     const int64_t r = ending ? b : aa;
     const int64_t x = ending ? aa : b;
+    if (r < f.row0 || r >= f.row_end) continue;      // another call's row shard
     const int64_t so = w * 8;                                  // storage offset
     const int64_t co = (((r * f.N + x) * f.H) + h) * 32 + q * 8;   // compact variant frame
     const uint4 g4 = *reinterpret_cast<const uint4 *>(gate + so);
@@ -137,11 +138,15 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
                                            __nv_bfloat16 *__restrict__ dk,
                                            __nv_bfloat16 *__restrict__ dv) {
   const int64_t pair = (int64_t)f.N * f.N * f.H * 32;
-  const int64_t per = pair / 8;                 // 16-byte groups per tensor and tile
+  // 16-byte groups per attention row of one tensor and tile; rows are outermost,
+  // so this call's row shard is one contiguous range of groups
+  const int64_t per_row = (int64_t)f.N * f.H * 4;
+  const int64_t first = (int64_t)f.row0 * per_row;
+  const int64_t per = (int64_t)(f.row_end - f.row0) * per_row;
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < 3 * per;
        w += (int64_t)gridDim.x * blockDim.x) {
     const int which = (int)(w / per);
-    const int64_t gidx = w - which * per;
+    const int64_t gidx = first + (w - which * per);
     const __nv_bfloat16 *src = (which == 0 ? pq : which == 1 ? pk : pv) + gidx * 8;
     const float sc = which == 2 ? 1.0f : scale;
     float acc[8];
@@ -185,8 +190,8 @@ cudaError_t launch_partial_reduce_bf16(const Frame &f, const __nv_bfloat16 *part
                                        const __nv_bfloat16 *part_k, const __nv_bfloat16 *part_v,
                                        int nb, float scale, __nv_bfloat16 *dq, __nv_bfloat16 *dk,
                                        __nv_bfloat16 *dv, cudaStream_t stream) {
-  const int64_t work = 3 * ((int64_t)f.N * f.N * f.H * 32 / 8);
-  if (work == 0) return cudaSuccess;
+  const int64_t work = 3 * ((int64_t)(f.row_end - f.row0) * f.N * f.H * 4);
+  if (work <= 0) return cudaSuccess;
   partial_reduce_bf16_kernel<<<blocks_for(work, 256), 256, 0, stream>>>(f, part_q, part_k, part_v,
                                                                          nb, scale, dq, dk, dv);
   return cudaGetLastError();
