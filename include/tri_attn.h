@@ -39,11 +39,14 @@
  *                                                 N: a full [N, N] mask); NULL
  *                                                 means every key takes part.
  *
- * Types. dtype BF16: every tensor above except lse and mask is bfloat16;
- * contractions run on the tensor cores with fp32 accumulation, softmax and
+ * Types. dtype BF16: every tensor above except lse and mask is bfloat16. With
+ * c == 32 and N % 8 == 0 the contractions run on the tensor cores with fp32
+ * accumulation (P and dS rounded to bf16 before their products), softmax and
  * gate arithmetic in fp32; dbias is accumulated in fp32 over all rows and
- * rounded once. dtype F32: every tensor is float32 and all arithmetic is fp32
- * on the CUDA cores (no TF32).
+ * rounded once. Every other bf16 shape runs on the CUDA-core kernels: bf16
+ * loads widened to fp32, all arithmetic fp32, each result rounded to bf16
+ * once. dtype F32: every tensor is float32 and all arithmetic is fp32 on the
+ * CUDA cores (no TF32).
  *
  * Ownership and threading. Every pointer is a caller-owned device pointer,
  * 16-byte aligned, to contiguous memory. The library allocates no device
@@ -88,9 +91,13 @@ typedef enum { TRI_ATTN_F32 = 0, TRI_ATTN_BF16 = 1 } tri_attn_dtype;
 typedef enum { TRI_ATTN_STARTING = 0, TRI_ATTN_ENDING = 1 } tri_attn_variant;
 
 /*
- * Problem description. Limits: N >= 0; H >= 1; N * N * H * c < 2^31 * 64.
- * BF16 needs c == 32 and N % 8 == 0 (the bias rows are moved by TMA, whose row
- * pitch must be a multiple of 16 bytes). F32 needs 1 <= c <= 64.
+ * Problem description. Limits: N >= 0; H >= 1; 1 <= c <= 64
+ * (TRI_ATTN_ERR_UNSUPPORTED above); N * N * H * c < 2^31 * 64. BF16 problems
+ * with c == 32 and N % 8 == 0 take the tensor-core kernels (the bias rows are
+ * moved by TMA, whose row pitch must be a multiple of 16 bytes); the others,
+ * and all F32 problems, the CUDA-core kernels. The rounding-residual option,
+ * the on-chip-sum option and row shards need the tensor-core kernels
+ * (TRI_ATTN_ERR_UNSUPPORTED, or the default path for the on-chip-sum bit).
  */
 typedef struct {
     int64_t N;                /* residues: the pair tensors are N x N           */

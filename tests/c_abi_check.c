@@ -27,7 +27,7 @@ int main(void) {
     p.N = 64; p.H = 4; p.c = 32; p.dtype = TRI_ATTN_BF16; p.variant = TRI_ATTN_STARTING;
     CHECK(3, tri_attn_fwd_workspace_size(&p, &n) == TRI_ATTN_OK && n > 0);
     CHECK(4, tri_attn_bwd_workspace_size(&p, &n) == TRI_ATTN_OK && n > 0);
-    p.c = 16;                                          /* bf16 takes c = 32 only */
+    p.c = 65;                                          /* head dimensions up to 64 */
     CHECK(5, tri_attn_fwd_workspace_size(&p, &n) == TRI_ATTN_ERR_UNSUPPORTED);
     p.c = 32; p.variant = 7;
     CHECK(6, tri_attn_fwd_workspace_size(&p, &n) == TRI_ATTN_ERR_INVALID_ARG);

@@ -80,13 +80,26 @@ def test_workspace_sizes(lib):
 
 @pytest.mark.parametrize("prob,code", [
     (P(N=-1), 1), (P(H=0), 1), (P(c=0), 1), (P(dtype=7), 1), (P(variant=2), 1),
-    (P(stride=5), 1), (P(c=64), 2), (P(N=60), 2), (P(dtype=ta.F32, c=65), 2),
+    (P(stride=5), 1), (P(c=65), 2), (P(dtype=ta.F32, c=65), 2),
 ])
 def test_invalid_problems(lib, prob, code):
     rc, _ = ws_size(lib, prob)
     assert rc == code
     rc, _ = ws_size(lib, prob, "bwd")
     assert rc == code
+
+
+@pytest.mark.parametrize("prob", [P(c=16), P(c=64), P(N=60), P(N=7, c=48), P(N=1)])
+def test_bf16_shapes_of_the_cuda_core_kernels(lib, prob):
+    """bf16 head dimensions other than 32 and N not a multiple of 8 run on the
+    CUDA-core kernels: valid problems with a workspace of their own layout."""
+    rc, n = ws_size(lib, prob)
+    assert rc == 0 and n >= 4
+    rc, nb = ws_size(lib, prob, "bwd")
+    assert rc == 0 and nb > 0
+    launches = ctypes.c_int32(0)
+    assert lib.tri_attn_kernel_launches(ctypes.byref(prob), 0, 0, ctypes.byref(launches)) == 0
+    assert launches.value == 1
 
 
 def test_null_problem_and_null_size(lib):
@@ -114,7 +127,7 @@ def test_host_side_rejections_before_any_launch(lib):
     assert lib.tri_attn_fwd(ctypes.byref(prob), *mis, fake, 1 << 30, z) == 1
     # backward: invalid problem, then missing workspace
     bargs = [fake] * 5 + [z] + [fake] * 8
-    assert lib.tri_attn_bwd(ctypes.byref(P(c=7)), *bargs, fake, 1 << 40, z) == 2
+    assert lib.tri_attn_bwd(ctypes.byref(P(c=65)), *bargs, fake, 1 << 40, z) == 2
     assert lib.tri_attn_bwd(ctypes.byref(prob), *bargs, z, 0, z) == 3
     # N = 0 is a valid no-op
     zero = P(N=0)

@@ -101,6 +101,21 @@ def test_bf16_small_and_tile_edges(N, H):
     full_check(d, STARTING, "bf16")
 
 
+@pytest.mark.parametrize("N,c,variant,mask", [
+    (1, 32, STARTING, None), (7, 32, STARTING, "random:2"), (33, 16, ENDING, "random:5"),
+    (130, 64, STARTING, "trailing:10"), (64, 16, STARTING, None), (100, 48, ENDING, "row"),
+])
+def test_bf16_cuda_core_shapes(N, c, variant, mask):
+    """bf16 shapes the tensor-core kernels do not take (head dimensions other
+    than 32, N not a multiple of 8) run on the CUDA-core kernels with bf16
+    storage and fp32 arithmetic: every output element against the oracle."""
+    d = make_inputs(N, H=2, c=c, dtype="bf16", seed=N + c, bias_std=1.2,
+                    mask="none" if mask in (None, "row") else mask)
+    if mask == "row":
+        d["mask"] = full_mask(N, seed=N, keep_prob=0.8, fully_masked_rows=(3,))
+    full_check(d, variant, "bf16")
+
+
 def test_bf16_n512_full_two_row_groups():
     """bf16, N=512, H=4 (4 tiles per axis): every output element. The backward
     splits each head's 512 rows into two row groups here (16 tiles x 4 heads

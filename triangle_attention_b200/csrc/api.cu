@@ -36,9 +36,14 @@ tri_attn_status check_problem(const tri_attn_problem *p) {
   if (p->variant != TRI_ATTN_STARTING && p->variant != TRI_ATTN_ENDING)
     return TRI_ATTN_ERR_INVALID_ARG;
   if (p->mask_row_stride != 0 && p->mask_row_stride != p->N) return TRI_ATTN_ERR_INVALID_ARG;
-  if (p->dtype == TRI_ATTN_BF16 && (p->c != 32 || p->N % 8 != 0)) return TRI_ATTN_ERR_UNSUPPORTED;
-  if (p->dtype == TRI_ATTN_F32 && p->c > 64) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (p->c > 64) return TRI_ATTN_ERR_UNSUPPORTED;
   return TRI_ATTN_OK;
+}
+
+// bf16 problems the tensor-core kernels take (head dimension 32, N a multiple of
+// 8); every other problem runs on the CUDA-core kernels.
+bool tc_shape(const tri_attn_problem *p) {
+  return p->dtype == TRI_ATTN_BF16 && p->c == 32 && p->N % 8 == 0;
 }
 
 Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status) {
@@ -98,7 +103,7 @@ size_t carve_fwd(const tri_attn_problem *p, void *ws, bool per_row_mask, FwdWs *
   Carver c(ws);
   FwdWs w{};
   w.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
-  if (p->dtype == TRI_ATTN_BF16) {
+  if (tc_shape(p)) {
     const int64_t rows = per_row_mask ? p->N : 1;
     w.mask_bits = static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
     if (p->variant == TRI_ATTN_ENDING)
@@ -147,7 +152,7 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
   w.fw.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
   const size_t pair = (size_t)p->N * p->N * p->H * p->c;
   const size_t nn = (size_t)p->N * p->N;
-  if (p->dtype == TRI_ATTN_BF16) {
+  if (tc_shape(p)) {
     const int64_t rows = per_row_mask ? p->N : 1;
     w.fw.mask_bits =
         static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
@@ -178,7 +183,7 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
     w.part_dk = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
     w.part_dv = static_cast<float *>(c.take(4 * pair * (size_t)w.ntile));
   }
-  if (p->dtype == TRI_ATTN_BF16 && !w.tc) {
+  if (tc_shape(p) && !w.tc) {
     // per-group dbias sums: also taken by a row-shard call, whose groups split
     // fewer rows but never number more than bwd_bf16_max_groups
     w.part_db = static_cast<float *>(
@@ -335,7 +340,7 @@ tri_attn_status check_opts(const tri_attn_problem *prob, const tri_attn_launch_o
     return TRI_ATTN_ERR_INVALID_ARG;
   const void *res = opt_residual(opts);
   if (res && !aligned16(res)) return TRI_ATTN_ERR_INVALID_ARG;
-  if (res && prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (res && !tc_shape(prob)) return TRI_ATTN_ERR_UNSUPPORTED;
   return TRI_ATTN_OK;
 }
 
@@ -350,6 +355,33 @@ cudaError_t mark(const tri_attn_launch_opts *opts, bool start, cudaStream_t stre
   do {                                                     \
     if (!(p) || !aligned16(p)) return TRI_ATTN_ERR_INVALID_ARG; \
   } while (0)
+
+}  // namespace
+
+namespace {
+
+// The CUDA-core kernels with the caller's tensors of type T.
+template <typename T>
+cudaError_t core_fwd(const Frame &f, const void *q, const void *k, const void *v,
+                     const void *bias, const void *gate, void *out, float *lse,
+                     cudaStream_t stream) {
+  return tri::launch_f32_fwd<T>(f, static_cast<const T *>(q), static_cast<const T *>(k),
+                                static_cast<const T *>(v), static_cast<const T *>(bias),
+                                static_cast<const T *>(gate), static_cast<T *>(out), lse, stream);
+}
+
+template <typename T>
+cudaError_t core_bwd(const Frame &f, const void *q, const void *k, const void *v,
+                     const void *bias, const void *gate, const void *out, const float *lse,
+                     const void *dout, void *dq, void *dk, void *dv, void *dbias, void *dgate,
+                     const tri::F32BwdScratch &s, cudaStream_t stream) {
+  return tri::launch_f32_bwd<T>(f, static_cast<const T *>(q), static_cast<const T *>(k),
+                                static_cast<const T *>(v), static_cast<const T *>(bias),
+                                static_cast<const T *>(gate), static_cast<const T *>(out), lse,
+                                static_cast<const T *>(dout), static_cast<T *>(dq),
+                                static_cast<T *>(dk), static_cast<T *>(dv),
+                                static_cast<T *>(dbias), static_cast<T *>(dgate), s, stream);
+}
 
 }  // namespace
 
@@ -418,15 +450,15 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
   f.row_end = (int)(row0 + row_count);
   if (row_count == 0) return TRI_ATTN_OK;
 
-  if (prob->dtype == TRI_ATTN_F32) {
+  if (!tc_shape(prob)) {
+    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic)
     if (row0 != 0 || row_count != prob->N) return TRI_ATTN_ERR_UNSUPPORTED;
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
     if (e == cudaSuccess) e = mark(opts, true, stream);
     if (e == cudaSuccess)
-      e = tri::launch_f32_fwd(f, static_cast<const float *>(q), static_cast<const float *>(k),
-                              static_cast<const float *>(v), static_cast<const float *>(bias),
-                              static_cast<const float *>(gate), static_cast<float *>(out), lse,
-                              stream);
+      e = prob->dtype == TRI_ATTN_F32
+              ? core_fwd<float>(f, q, k, v, bias, gate, out, lse, stream)
+              : core_fwd<__nv_bfloat16>(f, q, k, v, bias, gate, out, lse, stream);
     if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
@@ -509,6 +541,7 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
   const bool per_row = mask && prob->mask_row_stride == prob->N;
   const bool onchip = opts && (opts->flags & TRI_ATTN_OPT_ONCHIP_SUMS) != 0;
   if (onchip && prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_INVALID_ARG;
+  // (bf16 shapes of the CUDA-core kernels take the default path)
   BwdWs w;
   if (workspace_bytes < carve_bwd(prob, workspace, per_row, onchip, &w))
     return TRI_ATTN_ERR_WORKSPACE;
@@ -527,7 +560,8 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
   const bool shard = dbias_partial != nullptr || row0 != 0 || row_count != prob->N;
   if (row_count == 0) return TRI_ATTN_OK;
 
-  if (prob->dtype == TRI_ATTN_F32) {
+  if (!tc_shape(prob)) {
+    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic)
     if (shard) return TRI_ATTN_ERR_UNSUPPORTED;
     tri::F32BwdScratch s;
     s.du = static_cast<float *>(w.du);
@@ -541,13 +575,11 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
     cudaError_t e = cudaMemsetAsync(w.fw.status, 0, sizeof(int32_t), stream);
     if (e == cudaSuccess) e = mark(opts, true, stream);
     if (e == cudaSuccess)
-      e = tri::launch_f32_bwd(
-          f, static_cast<const float *>(q), static_cast<const float *>(k),
-          static_cast<const float *>(v), static_cast<const float *>(bias),
-          static_cast<const float *>(gate), static_cast<const float *>(out), lse,
-          static_cast<const float *>(dout), static_cast<float *>(dq), static_cast<float *>(dk),
-          static_cast<float *>(dv), static_cast<float *>(dbias), static_cast<float *>(dgate), s,
-          stream);
+      e = prob->dtype == TRI_ATTN_F32
+              ? core_bwd<float>(f, q, k, v, bias, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
+                                s, stream)
+              : core_bwd<__nv_bfloat16>(f, q, k, v, bias, gate, out, lse, dout, dq, dk, dv,
+                                        dbias, dgate, s, stream);
     if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
@@ -709,7 +741,7 @@ tri_attn_status tri_attn_fwd_rows(const tri_attn_problem *prob, int64_t row_begi
                                   tri_attn_stream_t stream) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  if (prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!tc_shape(prob)) return TRI_ATTN_ERR_UNSUPPORTED;
   st = check_rows(prob, row_begin, row_count);
   if (st != TRI_ATTN_OK) return st;
   return fwd_impl(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes, stream,
@@ -725,7 +757,7 @@ tri_attn_status tri_attn_bwd_rows(const tri_attn_problem *prob, int64_t row_begi
                                   tri_attn_stream_t stream) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  if (prob->dtype != TRI_ATTN_BF16) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!tc_shape(prob)) return TRI_ATTN_ERR_UNSUPPORTED;
   st = check_rows(prob, row_begin, row_count);
   if (st != TRI_ATTN_OK) return st;
   if (!dbias_partial && prob->N > 0) return TRI_ATTN_ERR_INVALID_ARG;
@@ -770,7 +802,7 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
   const bool onchip = backward == 2;
   int32_t n = 0;
   if (prob->N > 0) {
-    if (prob->dtype == TRI_ATTN_F32) {
+    if (!tc_shape(prob)) {
       if (!backward) {
         n = 1;
       } else {

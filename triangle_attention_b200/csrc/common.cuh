@@ -41,10 +41,12 @@ __host__ __device__ inline int64_t pair_elems(const Frame &f) {
   return (int64_t)f.N * f.N * f.H * f.c;
 }
 
-// ------------------------------------------------------ fp32 CUDA-core path --
-cudaError_t launch_f32_fwd(const Frame &f, const float *q, const float *k, const float *v,
-                           const float *bias, const float *gate, float *out, float *lse,
-                           cudaStream_t stream);
+// ------------------------------------------------------- CUDA-core path --
+// T = float (the fp32 path) or __nv_bfloat16 (bf16 shapes the tensor-core
+// kernels do not take); arithmetic in fp32.
+template <typename T>
+cudaError_t launch_f32_fwd(const Frame &f, const T *q, const T *k, const T *v, const T *bias,
+                           const T *gate, T *out, float *lse, cudaStream_t stream);
 
 // Scratch of the fp32 backward, carved by the API layer.
 struct F32BwdScratch {
@@ -59,10 +61,10 @@ struct F32BwdScratch {
 
 int f32_bwd_tile();
 void f32_bwd_plan(const Frame &f, int *ntile, int *ngroups);
-cudaError_t launch_f32_bwd(const Frame &f, const float *q, const float *k, const float *v,
-                           const float *bias, const float *gate, const float *out,
-                           const float *lse, const float *dout, float *dq, float *dk,
-                           float *dv, float *dbias, float *dgate, const F32BwdScratch &s,
+template <typename T>
+cudaError_t launch_f32_bwd(const Frame &f, const T *q, const T *k, const T *v, const T *bias,
+                           const T *gate, const T *out, const float *lse, const T *dout, T *dq,
+                           T *dk, T *dv, T *dbias, T *dgate, const F32BwdScratch &s,
                            cudaStream_t stream);
 
 // ---------------------------------------------- fixed-order reductions (any) --

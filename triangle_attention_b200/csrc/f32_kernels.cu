@@ -1,5 +1,9 @@
-// fp32 path of gated triangle self-attention on the CUDA cores (FFMA, no TF32),
-// plus the fixed-order reductions that both dtypes use for their backward.
+// CUDA-core path of gated triangle self-attention (FFMA, no TF32): the fp32
+// path, and the bf16 path for the shapes the tensor-core kernels do not take
+// (head dimensions other than 32, N not a multiple of 8). The caller's tensors
+// are of type T (float or bf16): every load widens to fp32, all arithmetic is
+// fp32 and every result is rounded to T once. Also the fixed-order reductions
+// that both dtypes use for their backward.
 //
 // Forward: one thread per query, online softmax over key tiles staged in
 // shared memory, accurate expf/logf.
@@ -28,10 +32,19 @@ constexpr int kT = 32;        // backward block edge (queries and keys)
 constexpr int kBwdThreads = 256;
 constexpr int kEntries = kT * kT / kBwdThreads;  // probability entries per thread
 
+__device__ __forceinline__ float ld(const float *p) { return *p; }
+__device__ __forceinline__ float ld(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+template <typename T> __device__ __forceinline__ T to_out(float x);
+template <> __device__ __forceinline__ float to_out<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+template <typename T>
 __global__ void __launch_bounds__(kFwdQ)
-f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k,
-               const float *__restrict__ v, const float *__restrict__ bias,
-               const float *__restrict__ gate, float *__restrict__ out,
+f32_fwd_kernel(Frame f, const T *__restrict__ q, const T *__restrict__ k,
+               const T *__restrict__ v, const T *__restrict__ bias,
+               const T *__restrict__ gate, T *__restrict__ out,
                float *__restrict__ lse) {
   __shared__ float ks[kFwdK][kCMax];
   __shared__ float vs[kFwdK][kCMax];
@@ -48,7 +61,7 @@ f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k
   float qr[kCMax], acc[kCMax];
 #pragma unroll
   for (int cc = 0; cc < kCMax; ++cc) {
-    qr[cc] = (active && cc < C) ? q[px + cc] : 0.0f;
+    qr[cc] = (active && cc < C) ? ld(q + px + cc) : 0.0f;
     acc[cc] = 0.0f;
   }
   float m = -INFINITY, l = 0.0f;
@@ -60,8 +73,8 @@ f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k
       float kv = 0.0f, vv = 0.0f;
       if (y < N) {
         const int64_t py = (int64_t)r * f.sR + (int64_t)y * f.sX + (int64_t)h * C + cc;
-        kv = k[py];
-        vv = v[py];
+        kv = ld(k + py);
+        vv = ld(v + py);
       }
       ks[yy][cc] = kv;
       vs[yy][cc] = vv;
@@ -79,7 +92,7 @@ f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k
 #pragma unroll
       for (int cc = 0; cc < kCMax; ++cc)
         if (cc < C) dot = fmaf(qr[cc], ks[yy][cc], dot);
-      const float s = dot * scale + bias[hb + (int64_t)x * f.bX + (int64_t)y * f.bY];
+      const float s = dot * scale + ld(bias + hb + (int64_t)x * f.bX + (int64_t)y * f.bY);
       if (s > m) {
         const float a = expf(m - s);  // m = -inf gives 0
         l = l * a + 1.0f;
@@ -101,8 +114,8 @@ f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k
 #pragma unroll
   for (int cc = 0; cc < kCMax; ++cc) {
     if (cc < C) {
-      const float sg = 1.0f / (1.0f + expf(-gate[px + cc]));
-      out[px + cc] = sg * (acc[cc] * inv);
+      const float sg = 1.0f / (1.0f + expf(-ld(gate + px + cc)));
+      out[px + cc] = to_out<T>(sg * (acc[cc] * inv));
     }
   }
   lse[((int64_t)r * f.H + h) * N + x] = l > 0.0f ? m + logf(l) : -INFINITY;
@@ -110,10 +123,11 @@ f32_fwd_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k
 
 // du = dout * sigmoid(g) (compact, variant frame); D = sum_c dout * out;
 // dgate = dout * out * (1 - sigmoid(g)).
-__global__ void f32_bwd_pre_kernel(Frame f, const float *__restrict__ gate,
-                                   const float *__restrict__ out,
-                                   const float *__restrict__ dout, float *__restrict__ du,
-                                   float *__restrict__ D, float *__restrict__ dgate) {
+template <typename T>
+__global__ void f32_bwd_pre_kernel(Frame f, const T *__restrict__ gate,
+                                   const T *__restrict__ out,
+                                   const T *__restrict__ dout, float *__restrict__ du,
+                                   float *__restrict__ D, T *__restrict__ dgate) {
   const int64_t total = (int64_t)f.N * f.N * f.H;
   const int C = f.c;
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
@@ -125,23 +139,24 @@ __global__ void f32_bwd_pre_kernel(Frame f, const float *__restrict__ gate,
     const int64_t cx = w * C;
     float d = 0.0f;
     for (int cc = 0; cc < C; ++cc) {
-      const float sg = 1.0f / (1.0f + expf(-gate[px + cc]));
-      const float go = dout[px + cc], o = out[px + cc];
+      const float sg = 1.0f / (1.0f + expf(-ld(gate + px + cc)));
+      const float go = ld(dout + px + cc), o = ld(out + px + cc);
       du[cx + cc] = go * sg;
       d = fmaf(go, o, d);
-      dgate[px + cc] = go * o * (1.0f - sg);
+      dgate[px + cc] = to_out<T>(go * o * (1.0f - sg));
     }
     D[(r * f.H + h) * f.N + x] = d;
   }
 }
 
+template <typename T>
 __global__ void __launch_bounds__(kBwdThreads)
-f32_bwd_main_kernel(Frame f, const float *__restrict__ q, const float *__restrict__ k,
-                    const float *__restrict__ v, const float *__restrict__ bias,
+f32_bwd_main_kernel(Frame f, const T *__restrict__ q, const T *__restrict__ k,
+                    const T *__restrict__ v, const T *__restrict__ bias,
                     const float *__restrict__ lse, const float *__restrict__ du,
                     const float *__restrict__ Dv, float *__restrict__ part_dq,
                     float *__restrict__ part_dk, float *__restrict__ part_dv,
-                    float *__restrict__ part_db, float *__restrict__ dbias, int ngroups,
+                    float *__restrict__ part_db, T *__restrict__ dbias, int ngroups,
                     int rows_per_group) {
   __shared__ float Qs[kT][kCMax + 1], Us[kT][kCMax + 1], Ks[kT][kCMax + 1], Vs[kT][kCMax + 1];
   __shared__ float Ps[kT][kT + 1], Ss[kT][kT + 1];
@@ -162,7 +177,7 @@ f32_bwd_main_kernel(Frame f, const float *__restrict__ q, const float *__restric
   for (int i = 0; i < kEntries; ++i) {
     const int e = threadIdx.x + kBwdThreads * i;
     const int x = x0 + e / kT, y = y0 + e % kT;
-    bval[i] = (x < N && y < N) ? bias[hb + (int64_t)x * f.bX + (int64_t)y * f.bY] : 0.0f;
+    bval[i] = (x < N && y < N) ? ld(bias + hb + (int64_t)x * f.bX + (int64_t)y * f.bY) : 0.0f;
     dbacc[i] = 0.0f;
   }
 
@@ -173,13 +188,13 @@ f32_bwd_main_kernel(Frame f, const float *__restrict__ q, const float *__restric
       const int x = x0 + t, y = y0 + t;
       float qv = 0.0f, uv = 0.0f, kv = 0.0f, vv = 0.0f;
       if (x < N) {
-        qv = q[(int64_t)r * f.sR + (int64_t)x * f.sX + (int64_t)h * C + cc];
+        qv = ld(q + (int64_t)r * f.sR + (int64_t)x * f.sX + (int64_t)h * C + cc);
         uv = du[(((int64_t)r * N + x) * H + h) * C + cc];
       }
       if (y < N) {
         const int64_t py = (int64_t)r * f.sR + (int64_t)y * f.sX + (int64_t)h * C + cc;
-        kv = k[py];
-        vv = v[py];
+        kv = ld(k + py);
+        vv = ld(v + py);
       }
       Qs[t][cc] = qv; Us[t][cc] = uv; Ks[t][cc] = kv; Vs[t][cc] = vv;
     }
@@ -233,16 +248,10 @@ f32_bwd_main_kernel(Frame f, const float *__restrict__ q, const float *__restric
     const int x = x0 + e / kT, y = y0 + e % kT;
     if (x >= N || y >= N) continue;
     if (ngroups == 1)
-      dbias[hb + (int64_t)x * f.bX + (int64_t)y * f.bY] = dbacc[i];
+      dbias[hb + (int64_t)x * f.bX + (int64_t)y * f.bY] = to_out<T>(dbacc[i]);
     else
       part_db[((int64_t)g * H + h) * N * N + (int64_t)x * N + y] = dbacc[i];
   }
-}
-
-template <typename T> __device__ __forceinline__ T to_out(float x);
-template <> __device__ __forceinline__ float to_out<float>(float x) { return x; }
-template <> __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float x) {
-  return __float2bfloat16_rn(x);
 }
 
 template <typename T>
@@ -284,12 +293,12 @@ int grid_for(int64_t n, int threads) {
 
 }  // namespace
 
-cudaError_t launch_f32_fwd(const Frame &f, const float *q, const float *k, const float *v,
-                           const float *bias, const float *gate, float *out, float *lse,
-                           cudaStream_t stream) {
+template <typename T>
+cudaError_t launch_f32_fwd(const Frame &f, const T *q, const T *k, const T *v, const T *bias,
+                           const T *gate, T *out, float *lse, cudaStream_t stream) {
   if (f.N == 0) return cudaSuccess;
   dim3 grid((f.N + kFwdQ - 1) / kFwdQ, f.H, f.N);
-  f32_fwd_kernel<<<grid, kFwdQ, 0, stream>>>(f, q, k, v, bias, gate, out, lse);
+  f32_fwd_kernel<T><<<grid, kFwdQ, 0, stream>>>(f, q, k, v, bias, gate, out, lse);
   return cudaGetLastError();
 }
 
@@ -307,32 +316,32 @@ void f32_bwd_plan(const Frame &f, int *ntile, int *ngroups) {
   *ngroups = rows > 0 ? (f.N + rows - 1) / rows : 1;
 }
 
-cudaError_t launch_f32_bwd(const Frame &f, const float *q, const float *k, const float *v,
-                           const float *bias, const float *gate, const float *out,
-                           const float *lse, const float *dout, float *dq, float *dk,
-                           float *dv, float *dbias, float *dgate, const F32BwdScratch &s,
+template <typename T>
+cudaError_t launch_f32_bwd(const Frame &f, const T *q, const T *k, const T *v, const T *bias,
+                           const T *gate, const T *out, const float *lse, const T *dout, T *dq,
+                           T *dk, T *dv, T *dbias, T *dgate, const F32BwdScratch &s,
                            cudaStream_t stream) {
   if (f.N == 0) return cudaSuccess;
   const int64_t rows_hx = (int64_t)f.N * f.N * f.H;
-  f32_bwd_pre_kernel<<<grid_for(rows_hx, 256), 256, 0, stream>>>(f, gate, out, dout, s.du, s.D,
-                                                                  dgate);
+  f32_bwd_pre_kernel<T><<<grid_for(rows_hx, 256), 256, 0, stream>>>(f, gate, out, dout, s.du,
+                                                                     s.D, dgate);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int rows_per_group = (f.N + s.ngroups - 1) / s.ngroups;
   dim3 grid(s.ntile, s.ntile, f.H * s.ngroups);
-  f32_bwd_main_kernel<<<grid, kBwdThreads, 0, stream>>>(
+  f32_bwd_main_kernel<T><<<grid, kBwdThreads, 0, stream>>>(
       f, q, k, v, bias, lse, s.du, s.D, s.part_dq, s.part_dk, s.part_dv, s.part_db, dbias,
       s.ngroups, rows_per_group);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const float scale = 1.0f / sqrtf((float)f.c);
-  if ((e = launch_pair_reduce<float>(f, s.part_dq, s.ntile, scale, dq, stream)) != cudaSuccess)
+  if ((e = launch_pair_reduce<T>(f, s.part_dq, s.ntile, scale, dq, stream)) != cudaSuccess)
     return e;
-  if ((e = launch_pair_reduce<float>(f, s.part_dk, s.ntile, scale, dk, stream)) != cudaSuccess)
+  if ((e = launch_pair_reduce<T>(f, s.part_dk, s.ntile, scale, dk, stream)) != cudaSuccess)
     return e;
-  if ((e = launch_pair_reduce<float>(f, s.part_dv, s.ntile, 1.0f, dv, stream)) != cudaSuccess)
+  if ((e = launch_pair_reduce<T>(f, s.part_dv, s.ntile, 1.0f, dv, stream)) != cudaSuccess)
     return e;
   if (s.ngroups > 1)
-    return launch_bias_reduce<float>(f, s.part_db, s.ngroups, dbias, stream);
+    return launch_bias_reduce<T>(f, s.part_db, s.ngroups, dbias, stream);
   return cudaSuccess;
 }
 
@@ -362,5 +371,22 @@ template cudaError_t launch_bias_reduce<float>(const Frame &, const float *, int
                                                cudaStream_t);
 template cudaError_t launch_bias_reduce<__nv_bfloat16>(const Frame &, const float *, int,
                                                        __nv_bfloat16 *, cudaStream_t);
+template cudaError_t launch_f32_fwd<float>(const Frame &, const float *, const float *,
+                                           const float *, const float *, const float *, float *,
+                                           float *, cudaStream_t);
+template cudaError_t launch_f32_fwd<__nv_bfloat16>(const Frame &, const __nv_bfloat16 *,
+                                                   const __nv_bfloat16 *, const __nv_bfloat16 *,
+                                                   const __nv_bfloat16 *, const __nv_bfloat16 *,
+                                                   __nv_bfloat16 *, float *, cudaStream_t);
+template cudaError_t launch_f32_bwd<float>(const Frame &, const float *, const float *,
+                                           const float *, const float *, const float *,
+                                           const float *, const float *, const float *, float *,
+                                           float *, float *, float *, float *,
+                                           const F32BwdScratch &, cudaStream_t);
+template cudaError_t launch_f32_bwd<__nv_bfloat16>(
+    const Frame &, const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *,
+    const __nv_bfloat16 *, const __nv_bfloat16 *, const __nv_bfloat16 *, const float *,
+    const __nv_bfloat16 *, __nv_bfloat16 *, __nv_bfloat16 *, __nv_bfloat16 *, __nv_bfloat16 *,
+    __nv_bfloat16 *, const F32BwdScratch &, cudaStream_t);
 
 }  // namespace tri
