@@ -158,3 +158,29 @@ def make_block_inputs(N: int, cz: int = 128, H: int = 4, c: int = 32, batch: Opt
     out["dy"] = draw(lead + (cz,))
     out["meta"] = dict(N=N, cz=cz, H=H, c=c, batch=batch, seed=seed)
     return out
+
+
+def make_update_inputs(N: int, cz: int = 128, c: int = 128, seed: int = 0) -> dict:
+    """Draw the pair representation, the parameters of the triangle
+    multiplicative update and the gradient that flows into its output.
+
+    Draw order: z, ln_gamma, ln_beta, w_in, b_in, ln_out_gamma, ln_out_beta, w_o,
+    b_o, dy. z ~ N(0, 1) + a per-position offset N(0, 1); LayerNorm gains ~
+    1 + 0.1 N(0, 1); offsets and biases ~ 0.1 N(0, 1); w_in ~ N(0, 1/cz) (its
+    [cz][4c + cz] columns are W_ap, W_ag, W_bp, W_bg, W_g); w_o ~ N(0, 1/c); dy ~
+    N(0, 1). z, w_in, w_o and dy are bf16, the rest float32."""
+    rng = np.random.default_rng(seed)
+
+    def draw(shape, s=1.0, shift=0.0, dtype="bf16"):
+        x = rng.standard_normal(shape, dtype=np.float32) * np.float32(s) + np.float32(shift)
+        return _round(x, dtype)
+
+    z = rng.standard_normal((N, N, cz), dtype=np.float32)
+    z += rng.standard_normal((N, N, 1), dtype=np.float32)
+    p = {"ln_gamma": draw((cz,), 0.1, 1.0, "f32"), "ln_beta": draw((cz,), 0.1, 0.0, "f32"),
+         "w_in": draw((cz, 4 * c + cz), cz ** -0.5), "b_in": draw((4 * c + cz,), 0.1, 0.0, "f32"),
+         "ln_out_gamma": draw((c,), 0.1, 1.0, "f32"), "ln_out_beta": draw((c,), 0.1, 0.0, "f32"),
+         "w_o": draw((c, cz), c ** -0.5), "b_o": draw((cz,), 0.1, 0.0, "f32")}
+    dy = draw((N, N, cz))
+    return {"z": _round(z, "bf16"), "params": p, "dy": dy,
+            "meta": dict(N=N, cz=cz, c=c, seed=seed)}
