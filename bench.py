@@ -579,6 +579,83 @@ def run_trimul(args, rank, world, local):
     return line
 
 
+UPDATE_METRIC = ("triangle multiplicative update fwd+bwd TFLOP/s at N=768, cz=128, c=128 bf16 "
+                 "(both directions; LayerNorms, gated projections, contraction, output)")
+
+
+def update_flops(N: int, cz: int, c: int) -> float:
+    """Matmul FLOPs of one forward + backward of the update (2 per multiply-add):
+    the input projection x W_in and its two gradients, the contraction and its
+    two, the output projection and its two."""
+    R, pgw = N * N, 4 * c + cz
+    return 3 * 2.0 * R * cz * pgw + 3 * 2.0 * N ** 3 * c + 3 * 2.0 * R * c * cz
+
+
+def run_trimul_update(args, rank, world, local):
+    """One step: forward and backward of the full triangle multiplicative update,
+    outgoing and incoming, N=768, cz=c=128."""
+    import triangle_attention_b200 as ta
+    N, cz, c = 768, 128, 128
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    d = tri_inputs.make_update_inputs(N, cz=cz, c=c, seed=21 + rank)
+    z, dy = d["z"].to(dev), d["dy"].to(dev)
+    params = {k: v.to(dev) for k, v in d["params"].items()}
+    prob = ta.MulUpdateProblem(N, cz, c, ta.OUTGOING, 1e-5)
+    nsaved, nws = ta.mul_update_sizes(prob)
+    ws = ta.workspace(nws, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for direction in (ta.OUTGOING, ta.INCOMING):
+            y, saved = ta.mul_update_fwd(z, params, direction, ws=ws)
+            ta.mul_update_bwd(z, params, saved, dy, direction, ws=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    if ta.get_status(ws):
+        raise RuntimeError("device status set in the timed region")
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
+    flops_step = 2 * update_flops(N, cz, c)
+    peaks = load_peaks()
+    achieved = flops_step / (ms * 1e-3) / 1e12
+    return {"metric": UPDATE_METRIC, "value": whole_job_tflops(world, flops_step, ms),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded inputs and random-init parameters, tri_inputs)",
+            "config": {"workload": "trimul_update_n768_cz128_c128", "N": N, "cz": cz, "c": c,
+                       "directions": ["outgoing", "incoming"],
+                       "l2": "inputs larger than L2 (saved activations 1.7 GB per direction)",
+                       "parallelism": "independent replica per GPU"},
+            "roofline": {"bound": "tensor", "kernel": "whole step (every kernel of the update)",
+                         "achieved": achieved, "peak": tensor_peak(peaks, clk)[0], "unit": UNIT,
+                         "frac": achieved / tensor_peak(peaks, clk)[0], "traffic": None,
+                         "peak_source": tensor_peak(peaks, clk)[1]},
+            "clocks": clk,
+            # per direction: forward 8 kernels (2 LayerNorms, 2 products, the
+            # contraction, 2 elementwise, a transpose); backward 19 (2 products, 2
+            # weight gradients with their sums, 2 contraction products, 2 LayerNorm
+            # backwards with their sums, 2 column sums with their sums, 2 elementwise,
+            # a transpose)
+            "gpu_launches": 2 * (8 + 19) * args.steps}
+
+
 BLOCK_METRIC = ("triangle-attention block fwd+bwd TFLOP/s at N=768, cz=128, H=4, c=32 bf16 "
                 "(LayerNorm, projections, attention, output projection)")
 
@@ -791,10 +868,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["attention", "trimul", "block", "proj"],
+    ap.add_argument("--op", choices=["attention", "trimul", "trimul_update", "block", "proj"],
                     default="attention",
-                    help="attention (the default line), the triangle multiplication, the "
-                         "whole block around the attention, or its projection stages alone")
+                    help="attention (the default line), the triangle multiplication "
+                         "contraction, the full triangle multiplicative update, the whole "
+                         "block around the attention, or its projection stages alone")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(tri_inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -816,6 +894,8 @@ def main():
     try:
         if args.op == "trimul":
             line = run_trimul(args, rank, world, local)
+        elif args.op == "trimul_update":
+            line = run_trimul_update(args, rank, world, local)
         elif args.op == "block":
             line = run_block(args, rank, world, local)
         elif args.op == "proj":

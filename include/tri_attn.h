@@ -391,6 +391,73 @@ tri_attn_status tri_mul_bwd(const tri_mul_problem *prob, const void *a, const vo
                             const void *dt, void *da, void *db, void *workspace,
                             size_t workspace_bytes, tri_attn_stream_t stream);
 
+/*
+ * The full triangle multiplicative update around the contraction, forward and
+ * backward ("TurboPairFormer accelera fino a 1,73x l'addestramento di OpenFold3
+ * nei test", sections "Dove si impiega il tempo" and "Benchmark di
+ * addestramento", name it beside triangle attention; the pages print no
+ * formula, the standard AlphaFold-family form is taken). Per pair position of
+ * z [N][N][cz] (bf16):
+ *   x = LayerNorm(z)                                   (over cz, biased variance)
+ *   [ap | ag | bp | bg | gl] = x W_in + b_in           W_in [cz][4c + cz]
+ *   a = sigmoid(ag) ap,  b = sigmoid(bg) bp            [N][N][c]
+ *   t = the outgoing or incoming contraction of a and b (tri_mul_fwd)
+ *   y = sigmoid(gl) (LayerNorm_out(t) W_o + b_o)       W_o [c][cz], y [N][N][cz] bf16
+ * Limits: cz and c in {64, 128, 192, 256}, N a multiple of 8
+ * (TRI_ATTN_ERR_UNSUPPORTED otherwise), eps > 0.
+ */
+typedef struct {
+    int64_t N;          /* residues */
+    int32_t cz;         /* channels of z and y */
+    int32_t c;          /* channels of a, b and t */
+    int32_t direction;  /* tri_mul_direction */
+    float eps;          /* epsilon of both LayerNorms */
+} tri_mul_update_problem;
+
+/* Parameters (device, caller-owned, 16-byte aligned). */
+typedef struct {
+    const float *ln_gamma, *ln_beta;          /* fp32 [cz] */
+    const void *w_in;                          /* bf16 [cz][4c + cz]: W_ap W_ag W_bp W_bg W_g */
+    const float *b_in;                         /* fp32 [4c + cz] */
+    const float *ln_out_gamma, *ln_out_beta;   /* fp32 [c] */
+    const void *w_o;                           /* bf16 [c][cz] */
+    const float *b_o;                          /* fp32 [cz] */
+} tri_mul_update_params;
+
+/* Parameter gradients (device, fp32, the shapes of the parameters). */
+typedef struct {
+    float *ln_gamma, *ln_beta, *w_in, *b_in, *ln_out_gamma, *ln_out_beta, *w_o, *b_o;
+} tri_mul_update_grads;
+
+/*
+ * Bytes of the activations the forward keeps for the backward (`saved`) and of
+ * the scratch either call needs (`workspace`, the larger of the two calls').
+ */
+tri_attn_status tri_mul_update_sizes(const tri_mul_update_problem *prob, size_t *saved_bytes,
+                                     size_t *workspace_bytes);
+
+/*
+ * Forward: reads z, writes y and the saved activations (caller-owned, at least
+ * saved_bytes, kept unchanged until the backward has run). Returns before the
+ * work completes; the workspace's first word is the status word
+ * (tri_attn_get_status).
+ */
+tri_attn_status tri_mul_update_fwd(const tri_mul_update_problem *prob,
+                                   const tri_mul_update_params *params, const void *z, void *y,
+                                   void *saved, size_t saved_bytes, void *workspace,
+                                   size_t workspace_bytes, tri_attn_stream_t stream);
+
+/*
+ * Backward of L = sum(dy * y): dz (bf16, shape of z) and every parameter
+ * gradient (overwritten, fp32, summed over the pair positions in a fixed
+ * order). `saved` is what the forward of the same z and parameters wrote.
+ */
+tri_attn_status tri_mul_update_bwd(const tri_mul_update_problem *prob,
+                                   const tri_mul_update_params *params, const void *z,
+                                   const void *saved, size_t saved_bytes, const void *dy,
+                                   void *dz, const tri_mul_update_grads *grads, void *workspace,
+                                   size_t workspace_bytes, tri_attn_stream_t stream);
+
 /* ------------------------------------------ LayerNorm and projections --
  *
  * The steps either side of the attention. The pages put LayerNorm at 14% of

@@ -86,6 +86,23 @@ class MulProblem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("C", ctypes.c_int32), ("direction", ctypes.c_int32)]
 
 
+class MulUpdateProblem(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("cz", ctypes.c_int32), ("c", ctypes.c_int32),
+                ("direction", ctypes.c_int32), ("eps", ctypes.c_float)]
+
+
+MUL_UPDATE_PARAMS = ("ln_gamma", "ln_beta", "w_in", "b_in", "ln_out_gamma", "ln_out_beta",
+                     "w_o", "b_o")
+
+
+class MulUpdateParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in MUL_UPDATE_PARAMS]
+
+
+class MulUpdateGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in MUL_UPDATE_PARAMS]
+
+
 class ProjProblem(ctypes.Structure):
     _fields_ = [("rows", ctypes.c_int64), ("batch", ctypes.c_int32), ("cz", ctypes.c_int32),
                 ("H", ctypes.c_int32), ("c", ctypes.c_int32), ("eps", ctypes.c_float),
@@ -134,6 +151,12 @@ def lib():
         L.tri_mul_workspace_size.argtypes = [MP, ctypes.POINTER(sz)]
         L.tri_mul_fwd.argtypes = [MP, P, P, P, P, sz, P]
         L.tri_mul_bwd.argtypes = [MP, P, P, P, P, P, P, sz, P]
+        UP = ctypes.POINTER(MulUpdateProblem)
+        L.tri_mul_update_sizes.argtypes = [UP, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.tri_mul_update_fwd.argtypes = [UP, ctypes.POINTER(MulUpdateParams), P, P, P, sz, P,
+                                         sz, P]
+        L.tri_mul_update_bwd.argtypes = [UP, ctypes.POINTER(MulUpdateParams), P, P, sz, P, P,
+                                         ctypes.POINTER(MulUpdateGrads), P, sz, P]
         JP = ctypes.POINTER(ProjProblem)
         L.tri_proj_workspace_size.argtypes = [JP, ctypes.POINTER(sz)]
         L.tri_proj_in_fwd.argtypes = [JP] + [P] * 13 + [P, sz, P]
@@ -145,7 +168,8 @@ def lib():
                   L.tri_attn_kernel_launches, L.tri_attn_read_status, L.tri_attn_get_status,
                   L.tri_attn_fwd_rows, L.tri_attn_bwd_rows, L.tri_attn_dbias_reduce,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
-                  L.tri_mul_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
+                  L.tri_mul_bwd, L.tri_mul_update_sizes, L.tri_mul_update_fwd,
+                  L.tri_mul_update_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
                   L.tri_proj_in_bwd, L.tri_proj_out_fwd, L.tri_proj_out_bwd):
             f.restype = ctypes.c_int
         _lib = L
@@ -503,6 +527,97 @@ class TriangleMultiplication(torch.autograd.Function):
             for i in range(a.shape[0]):
                 mul_bwd(a[i], b[i], dt[i], ctx.direction, grads=(da[i], db[i]))
         return da, db, None
+
+
+# --------------------------------------- full triangle multiplicative update --
+
+def _update_problem(z: torch.Tensor, params: dict, direction: int, eps: float):
+    if z.dim() != 3 or z.shape[0] != z.shape[1] or z.dtype != torch.bfloat16:
+        raise ValueError("the update takes a bf16 pair tensor [N, N, cz]")
+    N, cz = z.shape[0], z.shape[2]
+    c = (params["w_in"].shape[1] - cz) // 4
+    return MulUpdateProblem(N, cz, c, direction, eps)
+
+
+def _update_params(params: dict) -> MulUpdateParams:
+    _contig(*[params[n] for n in MUL_UPDATE_PARAMS])
+    return MulUpdateParams(*[params[n].data_ptr() for n in MUL_UPDATE_PARAMS])
+
+
+def mul_update_sizes(prob: MulUpdateProblem) -> tuple:
+    saved, ws = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    _check(lib().tri_mul_update_sizes(ctypes.byref(prob), ctypes.byref(saved), ctypes.byref(ws)),
+           "tri_mul_update_sizes")
+    return saved.value, ws.value
+
+
+def mul_update_fwd(z, params: dict, direction: int = OUTGOING, eps: float = 1e-5, ws=None,
+                   stream=None) -> tuple:
+    """The full triangle multiplicative update, bf16 [N, N, cz] -> [N, N, cz].
+    params: ln_gamma, ln_beta [cz], w_in [cz, 4c + cz] (bf16; W_ap W_ag W_bp W_bg
+    W_g), b_in [4c + cz], ln_out_gamma, ln_out_beta [c], w_o [c, cz] (bf16), b_o
+    [cz]; float32 unless marked. Returns (y, saved): saved holds the activations
+    the backward reads."""
+    _contig(z)
+    prob = _update_problem(z, params, direction, eps)
+    nsaved, nws = mul_update_sizes(prob)
+    saved = workspace(nsaved, z.device)
+    if ws is None:
+        ws = workspace(nws, z.device)
+    y = torch.empty_like(z)
+    pp = _update_params(params)
+    _check(lib().tri_mul_update_fwd(ctypes.byref(prob), ctypes.byref(pp), _p(z), _p(y),
+                                    _p(saved), saved.numel(), _p(ws), ws.numel(),
+                                    _stream(stream)), "tri_mul_update_fwd")
+    return y, saved
+
+
+def mul_update_bwd(z, params: dict, saved, dy, direction: int = OUTGOING, eps: float = 1e-5,
+                   ws=None, stream=None) -> tuple:
+    """(dz, grads) of L = sum(dy * y) for mul_update_fwd; grads maps every
+    parameter name to its float32 gradient."""
+    _contig(z, dy, saved)
+    prob = _update_problem(z, params, direction, eps)
+    _, nws = mul_update_sizes(prob)
+    if ws is None:
+        ws = workspace(nws, z.device)
+    dz = torch.empty_like(z)
+    grads = {n: torch.empty(params[n].shape, dtype=torch.float32, device=z.device)
+             for n in MUL_UPDATE_PARAMS}
+    gg = MulUpdateGrads(*[grads[n].data_ptr() for n in MUL_UPDATE_PARAMS])
+    pp = _update_params(params)
+    _check(lib().tri_mul_update_bwd(ctypes.byref(prob), ctypes.byref(pp), _p(z), _p(saved),
+                                    saved.numel(), _p(dy), _p(dz), ctypes.byref(gg), _p(ws),
+                                    ws.numel(), _stream(stream)), "tri_mul_update_bwd")
+    return dz, grads
+
+
+class TriangleMultiplicativeUpdate(torch.autograd.Function):
+    """y = TriangleMultiplicativeUpdate.apply(z, direction, eps, *params) with the
+    parameters in MUL_UPDATE_PARAMS order; gradients for z and every parameter
+    (cast to each parameter's dtype)."""
+
+    @staticmethod
+    def forward(ctx, z, direction, eps, *plist):
+        params = dict(zip(MUL_UPDATE_PARAMS, plist))
+        y, saved = mul_update_fwd(z, params, direction, eps)
+        ctx.direction, ctx.eps = direction, eps
+        ctx.save_for_backward(z, saved, *plist)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        z, saved, *plist = ctx.saved_tensors
+        params = dict(zip(MUL_UPDATE_PARAMS, plist))
+        dz, grads = mul_update_bwd(z, params, saved, dy.contiguous(), ctx.direction, ctx.eps)
+        return (dz, None, None) + tuple(grads[n].to(params[n].dtype) for n in MUL_UPDATE_PARAMS)
+
+
+def triangle_multiplicative_update(z, params: dict, direction: int = OUTGOING,
+                                   eps: float = 1e-5) -> torch.Tensor:
+    """Differentiable full triangle multiplicative update (see mul_update_fwd)."""
+    return TriangleMultiplicativeUpdate.apply(z, direction, eps,
+                                              *[params[n] for n in MUL_UPDATE_PARAMS])
 
 
 # ------------------------------------------------ LayerNorm and projections --

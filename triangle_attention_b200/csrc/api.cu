@@ -15,6 +15,7 @@
 #include "bf16.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "mul_update.cuh"
 #include "proj.cuh"
 
 namespace {
@@ -1291,6 +1292,321 @@ tri_attn_status tri_proj_out_bwd(const tri_proj_problem *prob, const void *o, co
   if (e != cudaSuccess) return cuda_status(e);
   segs[1] = colsum_segment(cpart, cz, db_o);
   return cuda_status(tri::launch_ordered_sums(segs, 2, stream));
+}
+
+// ----------------------------------------- triangle multiplicative update --
+
+namespace {
+
+struct MulUpdSaved {
+  __nv_bfloat16 *x, *pg, *a_cm, *b_cm, *t_pm, *u, *h;
+  float *stats, *stats_o;
+};
+
+struct MulUpdWs {
+  int32_t *status;
+  __nv_bfloat16 *zero_wb, *zero_bias, *bias_scratch;   // the LayerNorm kernels' bias head
+  __nv_bfloat16 *t_cm;                                 // forward
+  __nv_bfloat16 *dh, *dpg, *dt_pm, *dt_cm, *da_cm, *db_cm;   // backward
+  float *du, *dx, *part;
+};
+
+tri_attn_status check_mul_update(const tri_mul_update_problem *p) {
+  if (!p) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->N < 0 || p->N > kMaxN || !(p->eps > 0.0f)) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->direction != TRI_MUL_OUTGOING && p->direction != TRI_MUL_INCOMING)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  auto channels_ok = [](int v) { return v == 64 || v == 128 || v == 192 || v == 256; };
+  if (!channels_ok(p->cz) || !channels_ok(p->c) || p->N % 8 != 0)
+    return TRI_ATTN_ERR_UNSUPPORTED;
+  return TRI_ATTN_OK;
+}
+
+size_t carve_mul_update_saved(const tri_mul_update_problem *p, void *base, MulUpdSaved *out) {
+  Carver c(base);
+  MulUpdSaved s{};
+  const size_t R = (size_t)p->N * p->N, cz = p->cz, ch = p->c, pgw = 4 * ch + cz;
+  s.x = static_cast<__nv_bfloat16 *>(c.take(2 * R * cz));
+  s.stats = static_cast<float *>(c.take(8 * R));
+  s.pg = static_cast<__nv_bfloat16 *>(c.take(2 * R * pgw));
+  s.a_cm = static_cast<__nv_bfloat16 *>(c.take(2 * R * ch));
+  s.b_cm = static_cast<__nv_bfloat16 *>(c.take(2 * R * ch));
+  s.t_pm = static_cast<__nv_bfloat16 *>(c.take(2 * R * ch));
+  s.u = static_cast<__nv_bfloat16 *>(c.take(2 * R * ch));
+  s.stats_o = static_cast<float *>(c.take(8 * R));
+  s.h = static_cast<__nv_bfloat16 *>(c.take(2 * R * cz));
+  if (out) *out = s;
+  return c.off;
+}
+
+// A common head (status word, the zero bias head of the LayerNorm kernels),
+// then the forward's buffers and the backward's sharing one region.
+size_t carve_mul_update_ws(const tri_mul_update_problem *p, void *base, MulUpdWs *out) {
+  Carver c(base);
+  MulUpdWs w{};
+  const int64_t R = p->N * p->N, cz = p->cz, ch = p->c, pgw = 4 * ch + cz;
+  w.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
+  w.zero_wb = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)std::max(cz, ch)));
+  w.zero_bias = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)R));
+  w.bias_scratch = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)R));
+  const size_t head = c.off;
+  // forward
+  w.t_cm = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * ch)));
+  const size_t fwd_end = c.off;
+  // backward, from the same offset
+  c.off = head;
+  w.dh = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * cz)));
+  w.dpg = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * pgw)));
+  w.dt_pm = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * ch)));
+  w.dt_cm = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * ch)));
+  w.da_cm = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * ch)));
+  w.db_cm = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)(R * ch)));
+  w.du = static_cast<float *>(c.take(4 * (size_t)(R * ch)));
+  w.dx = static_cast<float *>(c.take(4 * (size_t)(R * cz)));
+  const int64_t blocks = tri::proj_partials();
+  int64_t part = std::max<int64_t>(blocks * 3 * std::max(cz, ch), blocks * pgw);
+  if (R > 0) {
+    part = std::max(part, weight_grad_partials(cz, pgw, R));
+    part = std::max(part, weight_grad_partials(ch, cz, R));
+  }
+  w.part = static_cast<float *>(c.take(4 * (size_t)part));
+  if (out) *out = w;
+  return std::max(fwd_end, c.off);
+}
+
+// One LayerNorm over `ch` channels through the projection kernels, with a
+// single bias head of zeros whose output is discarded.
+tri::ProjArgs ln_args(const MulUpdWs &w, int64_t R, int ch, float eps, const void *z,
+                      const float *gamma, const float *beta, __nv_bfloat16 *x, float *stats) {
+  tri::ProjArgs a{};
+  a.rows = R;
+  a.rows_per = R;
+  a.cz = ch;
+  a.H = 1;
+  a.eps = eps;
+  a.z = static_cast<const __nv_bfloat16 *>(z);
+  a.gamma = gamma;
+  a.beta = beta;
+  a.w_b = w.zero_wb;
+  a.x = x;
+  a.stats = stats;
+  a.bias = w.bias_scratch;
+  a.dbias = w.zero_bias;
+  a.part = w.part;
+  a.status = w.status;
+  return a;
+}
+
+// D [M][Nn] = X Y^T with X [M][K] K-major and Y as stored (MN-major [K][Nn] or
+// K-major [Nn][K]); bf16 output with an optional column bias, or fp32.
+tri_attn_status product(const void *x, const void *y, bool y_mn, void *out, bool f32, int64_t M,
+                        int64_t Nn, int64_t K, const float *bias, int32_t *status,
+                        cudaStream_t stream) {
+  tri::GemmMaps xs, ys;
+  tri::GemmOuts outs;
+  if (!encode_operand(&xs.map[0], x, false, M, K, 1) ||
+      !encode_operand(&ys.map[0], y, y_mn, Nn, K, 1) ||
+      !encode_stack(&outs.map[0], out, f32, Nn, M, 1, f32 ? 32 : 64, 32))
+    return TRI_ATTN_ERR_CUDA;
+  tri::GemmArgs args{};
+  args.M = (int)M;
+  args.Nn = (int)Nn;
+  args.K = (int)K;
+  args.batch = 1;
+  args.nouts = 1;
+  args.cols_per_out = (int)Nn;
+  args.k_per_x = 1 << 30;
+  args.col_bias = bias;
+  args.col_bias_from = 0;
+  args.status = status;
+  return cuda_status(tri::launch_gemm_tc(false, y_mn, f32, xs, ys, outs, args, stream));
+}
+
+tri_attn_status mul_update_begin(const tri_mul_update_problem *p,
+                                 const tri_mul_update_params *w, const void *saved,
+                                 size_t saved_bytes, void *ws, size_t ws_bytes) {
+  tri_attn_status st = check_mul_update(p);
+  if (st != TRI_ATTN_OK) return st;
+  if (!w) return TRI_ATTN_ERR_INVALID_ARG;
+  for (const void *q : {(const void *)w->ln_gamma, (const void *)w->ln_beta, w->w_in,
+                        (const void *)w->b_in, (const void *)w->ln_out_gamma,
+                        (const void *)w->ln_out_beta, w->w_o, (const void *)w->b_o})
+    TRI_CHECK_PTR(q);
+  if (!ws || !aligned16(ws) || ws_bytes < carve_mul_update_ws(p, nullptr, nullptr))
+    return TRI_ATTN_ERR_WORKSPACE;
+  if (!saved || !aligned16(saved) || saved_bytes < carve_mul_update_saved(p, nullptr, nullptr))
+    return TRI_ATTN_ERR_WORKSPACE;
+  return TRI_ATTN_OK;
+}
+
+}  // namespace
+
+tri_attn_status tri_mul_update_sizes(const tri_mul_update_problem *prob, size_t *saved_bytes,
+                                     size_t *workspace_bytes) {
+  tri_attn_status st = check_mul_update(prob);
+  if (st != TRI_ATTN_OK) return st;
+  if (!saved_bytes || !workspace_bytes) return TRI_ATTN_ERR_INVALID_ARG;
+  *saved_bytes = carve_mul_update_saved(prob, nullptr, nullptr);
+  *workspace_bytes = carve_mul_update_ws(prob, nullptr, nullptr);
+  return TRI_ATTN_OK;
+}
+
+tri_attn_status tri_mul_update_fwd(const tri_mul_update_problem *prob,
+                                   const tri_mul_update_params *params, const void *z, void *y,
+                                   void *saved, size_t saved_bytes, void *workspace,
+                                   size_t workspace_bytes, tri_attn_stream_t stream_) {
+  tri_attn_status st =
+      mul_update_begin(prob, params, saved, saved_bytes, workspace, workspace_bytes);
+  if (st != TRI_ATTN_OK) return st;
+  if (prob->N == 0) return TRI_ATTN_OK;
+  TRI_CHECK_PTR(z);
+  TRI_CHECK_PTR(y);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  MulUpdSaved s;
+  MulUpdWs w;
+  carve_mul_update_saved(prob, saved, &s);
+  carve_mul_update_ws(prob, workspace, &w);
+  const int64_t R = prob->N * prob->N, cz = prob->cz, ch = prob->c, pgw = 4 * ch + cz;
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.zero_wb, 0, 2 * (size_t)std::max(cz, ch), stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  // x = LayerNorm(z)
+  tri::ProjArgs a = ln_args(w, R, (int)cz, prob->eps, z, params->ln_gamma, params->ln_beta,
+                            s.x, s.stats);
+  if ((st = cuda_status(tri::launch_ln_fwd(a, stream))) != TRI_ATTN_OK) return st;
+  // [ap | ag | bp | bg | gl] = x W_in + b_in
+  if ((st = product(s.x, params->w_in, true, s.pg, false, R, pgw, cz, params->b_in, w.status,
+                    stream)) != TRI_ATTN_OK)
+    return st;
+  // a, b channel-major; t = their contraction (channel-major), then pair-major
+  if ((st = cuda_status(tri::launch_gate_in_fwd(s.pg, R, (int)ch, pgw, s.a_cm, s.b_cm,
+                                                stream))) != TRI_ATTN_OK)
+    return st;
+  const tri_mul_problem mp{prob->N, (int32_t)ch, prob->direction};
+  const bool mn = prob->direction == TRI_MUL_INCOMING;
+  if ((st = mul_product(&mp, s.a_cm, mn, s.b_cm, mn, w.t_cm, w.status, stream)) != TRI_ATTN_OK)
+    return st;
+  if ((st = cuda_status(tri::launch_transpose(w.t_cm, ch, R, s.t_pm, stream))) != TRI_ATTN_OK)
+    return st;
+  // u = LayerNorm_out(t); h = u W_o + b_o; y = sigmoid(gl) h
+  a = ln_args(w, R, (int)ch, prob->eps, s.t_pm, params->ln_out_gamma, params->ln_out_beta, s.u,
+              s.stats_o);
+  if ((st = cuda_status(tri::launch_ln_fwd(a, stream))) != TRI_ATTN_OK) return st;
+  if ((st = product(s.u, params->w_o, true, s.h, false, R, cz, ch, params->b_o, w.status,
+                    stream)) != TRI_ATTN_OK)
+    return st;
+  return cuda_status(tri::launch_out_fwd(s.pg, pgw, (int)(4 * ch), s.h, R, (int)cz,
+                                         static_cast<__nv_bfloat16 *>(y), stream));
+}
+
+tri_attn_status tri_mul_update_bwd(const tri_mul_update_problem *prob,
+                                   const tri_mul_update_params *params, const void *z,
+                                   const void *saved, size_t saved_bytes, const void *dy,
+                                   void *dz, const tri_mul_update_grads *grads, void *workspace,
+                                   size_t workspace_bytes, tri_attn_stream_t stream_) {
+  tri_attn_status st =
+      mul_update_begin(prob, params, saved, saved_bytes, workspace, workspace_bytes);
+  if (st != TRI_ATTN_OK) return st;
+  if (!grads) return TRI_ATTN_ERR_INVALID_ARG;
+  for (const void *q : {(const void *)grads->ln_gamma, (const void *)grads->ln_beta,
+                        (const void *)grads->w_in, (const void *)grads->b_in,
+                        (const void *)grads->ln_out_gamma, (const void *)grads->ln_out_beta,
+                        (const void *)grads->w_o, (const void *)grads->b_o})
+    TRI_CHECK_PTR(q);
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int64_t R = prob->N * prob->N, cz = prob->cz, ch = prob->c, pgw = 4 * ch + cz;
+  if (R == 0) {
+    // no pair positions: every parameter gradient is an empty sum
+    for (auto t : {std::make_pair(grads->ln_gamma, cz), std::make_pair(grads->ln_beta, cz),
+                   std::make_pair(grads->w_in, cz * pgw), std::make_pair(grads->b_in, pgw),
+                   std::make_pair(grads->ln_out_gamma, ch), std::make_pair(grads->ln_out_beta, ch),
+                   std::make_pair(grads->w_o, ch * cz), std::make_pair(grads->b_o, cz)})
+      if ((st = zero_f32(t.first, (size_t)t.second, stream)) != TRI_ATTN_OK) return st;
+    return TRI_ATTN_OK;
+  }
+  TRI_CHECK_PTR(z);
+  TRI_CHECK_PTR(dy);
+  TRI_CHECK_PTR(dz);
+  MulUpdSaved s;
+  MulUpdWs w;
+  carve_mul_update_saved(prob, const_cast<void *>(saved), &s);
+  carve_mul_update_ws(prob, workspace, &w);
+  const ProjWs pw{w.status, w.dx, w.part};
+  const int64_t blocks = tri::proj_partials();
+  cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.zero_wb, 0, 2 * (size_t)std::max(cz, ch), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.zero_bias, 0, 2 * (size_t)R, stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  // dh = dy sigmoid(gl); dgl into the last cz columns of dpg
+  if ((st = cuda_status(tri::launch_out_bwd(static_cast<const __nv_bfloat16 *>(dy), s.pg, pgw,
+                                            (int)(4 * ch), s.h, R, (int)cz, w.dh, w.dpg,
+                                            stream))) != TRI_ATTN_OK)
+    return st;
+  // dW_o = u^T dh, db_o = column sums of dh, du = dh W_o^T (fp32)
+  const void *dh_list[1] = {w.dh};
+  if ((st = weight_grad(s.u, dh_list, 1, ch, cz, R, grads->w_o, pw, stream)) != TRI_ATTN_OK)
+    return st;
+  e = tri::launch_colsum(w.dh, R, (int)cz, w.part, stream);
+  if (e == cudaSuccess) {
+    const tri::SumSeg seg = colsum_segment(w.part, cz, grads->b_o);
+    e = tri::launch_ordered_sums(&seg, 1, stream);
+  }
+  if ((st = cuda_status(e)) != TRI_ATTN_OK) return st;
+  if ((st = product(w.dh, params->w_o, false, w.du, true, R, ch, cz, nullptr, w.status,
+                    stream)) != TRI_ATTN_OK)
+    return st;
+  // LayerNorm_out backward: dt (pair-major), dgamma_o, dbeta_o
+  tri::ProjArgs a = ln_args(w, R, (int)ch, prob->eps, s.t_pm, params->ln_out_gamma, nullptr,
+                            s.u, s.stats_o);
+  a.dx = w.du;
+  a.dz = w.dt_pm;
+  e = tri::launch_ln_bwd(a, stream);
+  if (e == cudaSuccess) {
+    const tri::SumSeg segs[2] = {{w.part, blocks, 3 * ch, ch, grads->ln_out_gamma, ch, ch},
+                                 {w.part + ch, blocks, 3 * ch, ch, grads->ln_out_beta, ch, ch}};
+    e = tri::launch_ordered_sums(segs, 2, stream);
+  }
+  if (e == cudaSuccess) e = tri::launch_transpose(w.dt_pm, R, ch, w.dt_cm, stream);
+  if ((st = cuda_status(e)) != TRI_ATTN_OK) return st;
+  // the contraction's backward (as tri_mul_bwd), then the gates': dpg columns 0 .. 4c
+  const tri_mul_problem mp{prob->N, (int32_t)ch, prob->direction};
+  if (prob->direction == TRI_MUL_OUTGOING) {
+    st = mul_product(&mp, w.dt_cm, false, s.b_cm, true, w.da_cm, w.status, stream);
+    if (st == TRI_ATTN_OK)
+      st = mul_product(&mp, w.dt_cm, true, s.a_cm, true, w.db_cm, w.status, stream);
+  } else {
+    st = mul_product(&mp, s.b_cm, false, w.dt_cm, false, w.da_cm, w.status, stream);
+    if (st == TRI_ATTN_OK)
+      st = mul_product(&mp, s.a_cm, false, w.dt_cm, true, w.db_cm, w.status, stream);
+  }
+  if (st != TRI_ATTN_OK) return st;
+  if ((st = cuda_status(tri::launch_gate_in_bwd(w.da_cm, w.db_cm, s.pg, R, (int)ch, pgw, w.dpg,
+                                                stream))) != TRI_ATTN_OK)
+    return st;
+  // db_in = column sums of dpg; dW_in = x^T dpg; dx = dpg W_in^T (fp32)
+  e = tri::launch_colsum_strided(w.dpg, R, pgw, (int)pgw, w.part, stream);
+  if (e == cudaSuccess) {
+    const tri::SumSeg seg = colsum_segment(w.part, pgw, grads->b_in);
+    e = tri::launch_ordered_sums(&seg, 1, stream);
+  }
+  if ((st = cuda_status(e)) != TRI_ATTN_OK) return st;
+  const void *dpg_list[1] = {w.dpg};
+  if ((st = weight_grad(s.x, dpg_list, 1, cz, pgw, R, grads->w_in, pw, stream)) != TRI_ATTN_OK)
+    return st;
+  if ((st = product(w.dpg, params->w_in, false, w.dx, true, R, cz, pgw, nullptr, w.status,
+                    stream)) != TRI_ATTN_OK)
+    return st;
+  // LayerNorm backward: dz, dgamma, dbeta
+  a = ln_args(w, R, (int)cz, prob->eps, z, params->ln_gamma, nullptr, s.x, s.stats);
+  a.dx = w.dx;
+  a.dz = static_cast<__nv_bfloat16 *>(dz);
+  e = tri::launch_ln_bwd(a, stream);
+  if (e == cudaSuccess) {
+    const tri::SumSeg segs[2] = {{w.part, blocks, 3 * cz, cz, grads->ln_gamma, cz, cz},
+                                 {w.part + cz, blocks, 3 * cz, cz, grads->ln_beta, cz, cz}};
+    e = tri::launch_ordered_sums(segs, 2, stream);
+  }
+  return cuda_status(e);
 }
 
 }  // extern "C"
