@@ -207,6 +207,17 @@ typedef struct {
  */
 #define TRI_ATTN_OPT_ONCHIP_SUMS 0x1u
 
+/*
+ * flags bit of tri_attn_fwd_ex: compute one key pair in four of the softmax
+ * exponentials on the FMA pipe (tri_attn_check_exp2 gives the method and its
+ * error bound) instead of the MUFU unit, whose 16 results per clock per SM set
+ * the floor of the exponentials of the step. Tensor-core shapes only (the
+ * CUDA-core forward ignores it); results differ from the default in the last
+ * bits of the affected probabilities. The backward rejects it
+ * (TRI_ATTN_ERR_INVALID_ARG).
+ */
+#define TRI_ATTN_OPT_EXP2_SPLIT 0x2u
+
 /* tri_attn_fwd with options (opts may be NULL: same as tri_attn_fwd). */
 tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, const void *k,
                                 const void *v, const void *bias, const void *gate,
@@ -350,6 +361,18 @@ tri_attn_status tri_attn_get_status(const void *workspace, tri_attn_stream_t str
  */
 tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
                                             tri_attn_stream_t stream);
+
+/*
+ * Diagnostic of the forward's two exp2 evaluations (no counterpart on the
+ * pages): for each of the n fp32 exponents x (device), y_fma receives the
+ * FMA-pipe polynomial evaluation that TRI_ATTN_OPT_EXP2_SPLIT uses (Cody-Waite
+ * reduction, degree-4 minimax polynomial, relative error below 2.7e-6 for
+ * -125 <= x <= 126, inputs below -125 treated as -125) and y_mufu the hardware
+ * approximation (ex2.approx.ftz). Device buffers of n floats, caller-owned; one
+ * kernel on `stream`. TRI_ATTN_ERR_INVALID_ARG for n < 0 or NULL pointers.
+ */
+tri_attn_status tri_attn_check_exp2(const float *x, float *y_fma, float *y_mufu, int64_t n,
+                                    tri_attn_stream_t stream);
 
 /* ------------------------------------------------ triangle multiplication --
  *

@@ -51,21 +51,25 @@ class LaunchOpts(ctypes.Structure):
 
 
 OPT_ONCHIP_SUMS = 0x1
+OPT_EXP2_SPLIT = 0x2
 
 
 def launch_opts(main_start=None, main_stop=None, residual=None,
-                onchip_sums: bool = False) -> LaunchOpts:
+                onchip_sums: bool = False, exp2_split: bool = False) -> LaunchOpts:
     """Options: torch.cuda.Event objects recorded around the main kernel, the
     bf16 rounding residual of `out` (a tensor shaped like out) that the
-    forward writes and the backward uses for D and dgate, and (backward only)
-    the on-chip summation of the tile contributions (TRI_ATTN_OPT_ONCHIP_SUMS)."""
+    forward writes and the backward uses for D and dgate, (backward only) the
+    on-chip summation of the tile contributions (TRI_ATTN_OPT_ONCHIP_SUMS) and
+    (forward only) one exponential pair in four on the FMA pipe
+    (TRI_ATTN_OPT_EXP2_SPLIT)."""
     def handle(ev):
         if ev is None:
             return None
         if not ev.cuda_event:            # torch creates the event lazily
             ev.record()
         return ctypes.c_void_p(ev.cuda_event)
-    return LaunchOpts(ctypes.sizeof(LaunchOpts), OPT_ONCHIP_SUMS if onchip_sums else 0,
+    flags = (OPT_ONCHIP_SUMS if onchip_sums else 0) | (OPT_EXP2_SPLIT if exp2_split else 0)
+    return LaunchOpts(ctypes.sizeof(LaunchOpts), flags,
                       handle(main_start), handle(main_stop),
                       None if residual is None else ctypes.c_void_p(residual.data_ptr()))
 
@@ -142,6 +146,7 @@ def lib():
                                                ctypes.POINTER(ctypes.c_int32)]
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.tri_attn_get_status.argtypes = [P, P]
+        L.tri_attn_check_exp2.argtypes = [P, P, P, ctypes.c_int64, P]
         i64 = ctypes.c_int64
         L.tri_attn_fwd_rows.argtypes = [PP, i64, i64, P, P, P, P, P, P, P, P, P, sz, P]
         L.tri_attn_bwd_rows.argtypes = [PP, i64, i64] + [P] * 15 + [sz, P]
@@ -167,6 +172,7 @@ def lib():
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
                   L.tri_attn_kernel_launches, L.tri_attn_read_status, L.tri_attn_get_status,
                   L.tri_attn_fwd_rows, L.tri_attn_bwd_rows, L.tri_attn_dbias_reduce,
+                  L.tri_attn_check_exp2,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
                   L.tri_mul_bwd, L.tri_mul_update_sizes, L.tri_mul_update_fwd,
                   L.tri_mul_update_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
@@ -403,6 +409,15 @@ def get_status(ws: torch.Tensor, stream=None) -> int:
     if code == 4:
         _check(code, "tri_attn_get_status")
     return code
+
+
+def check_exp2(x: torch.Tensor, stream=None) -> tuple:
+    """(FMA-pipe exp2, MUFU exp2) of the fp32 device tensor x, elementwise."""
+    _contig(x)
+    y_fma, y_mufu = torch.empty_like(x), torch.empty_like(x)
+    _check(lib().tri_attn_check_exp2(_p(x), _p(y_fma), _p(y_mufu), x.numel(), _stream(stream)),
+           "tri_attn_check_exp2")
+    return y_fma, y_mufu
 
 
 def check_wait_timeout(ws: torch.Tensor, stream=None) -> int:

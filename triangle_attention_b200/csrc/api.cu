@@ -435,7 +435,7 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
                          int64_t row0, int64_t row_count) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  st = check_opts(prob, opts, 0u);
+  st = check_opts(prob, opts, TRI_ATTN_OPT_EXP2_SPLIT);
   if (st != TRI_ATTN_OK) return st;
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0)
@@ -480,6 +480,7 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
   a.H = f.H;
   a.row0 = f.row0;
   a.row_end = f.row_end;
+  a.exp2_split = (opts && (opts->flags & TRI_ATTN_OPT_EXP2_SPLIT)) ? 1 : 0;
   a.x_inner = x_inner ? 1 : 0;
   a.scale = 1.0f / sqrtf((float)prob->c);
   a.sR = f.sR;
@@ -850,6 +851,13 @@ tri_attn_status tri_attn_get_status(const void *workspace, tri_attn_stream_t str
   int32_t v = 0;
   const tri_attn_status st = tri_attn_read_status(workspace, &v, stream);
   return st != TRI_ATTN_OK ? st : static_cast<tri_attn_status>(v);
+}
+
+tri_attn_status tri_attn_check_exp2(const float *x, float *y_fma, float *y_mufu, int64_t n,
+                                    tri_attn_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y_fma || !y_mufu))) return TRI_ATTN_ERR_INVALID_ARG;
+  return cuda_status(
+      tri::launch_exp2_eval(x, y_fma, y_mufu, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,

@@ -26,6 +26,7 @@ struct FwdMaps {
 struct FwdArgs {
   int N, H;
   int row0, row_end;                 // attention rows of this launch (multiples of 8)
+  int exp2_split;                    // host-side: one key pair in four takes the FMA-pipe exp2
   int x_inner;                       // dimension order of the pair maps (see above)
   float scale;                       // c^-1/2
   int64_t sR, sX;                    // pair strides of the variant frame (elements)

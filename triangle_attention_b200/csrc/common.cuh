@@ -36,6 +36,9 @@ __device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
 
 // Diagnostic kernel: a bounded wait that nothing satisfies (see selftest.cu).
 cudaError_t launch_unsatisfied_wait(int32_t *status, cudaStream_t stream);
+// Diagnostic kernel: both device exp2 evaluations of x[0..n) (see selftest.cu).
+cudaError_t launch_exp2_eval(const float *x, float *y_fma, float *y_mufu, int64_t n,
+                             cudaStream_t stream);
 
 __host__ __device__ inline int64_t pair_elems(const Frame &f) {
   return (int64_t)f.N * f.N * f.H * f.c;

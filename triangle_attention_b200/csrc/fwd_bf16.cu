@@ -127,13 +127,23 @@ __device__ __forceinline__ void exponents32(uint32_t (&u)[32], const uint8_t *br
 }
 
 // Probabilities of 32 keys from their exponents: bf16 pairs into pk, running
-// sums into sa/sb. MASKED: keys whose bit in mword is clear give 0.
-template <bool MASKED>
+// sums into sa/sb. MASKED: keys whose bit in mword is clear give 0. POLY > 0:
+// every POLY-th key pair takes the FMA-pipe exp2 instead of the MUFU one.
+template <bool MASKED, int POLY>
 __device__ __forceinline__ void probs32(const uint32_t (&u)[32], uint32_t mword, uint64_t &sa,
                                         uint64_t &sb, uint32_t (&pk)[16]) {
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    float p0 = ex2_approx(__uint_as_float(u[e])), p1 = ex2_approx(__uint_as_float(u[e + 1]));
+    float p0, p1;
+    if (POLY > 0 && (e / 2) % POLY == POLY - 1) {
+      const float2 pp =
+          f2unpack(exp2_fma2(f2pack(__uint_as_float(u[e]), __uint_as_float(u[e + 1]))));
+      p0 = pp.x;
+      p1 = pp.y;
+    } else {
+      p0 = ex2_approx(__uint_as_float(u[e]));
+      p1 = ex2_approx(__uint_as_float(u[e + 1]));
+    }
     if (MASKED) {
       if (!((mword >> e) & 1u)) p0 = 0.0f;
       if (!((mword >> (e + 1)) & 1u)) p1 = 0.0f;
@@ -144,6 +154,7 @@ __device__ __forceinline__ void probs32(const uint32_t (&u)[32], uint32_t mword,
   }
 }
 
+template <int POLY>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
@@ -390,8 +401,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           // P (bf16 pairs) of keys 32*c32.. goes to columns 16*c32.. of this S
           // buffer, whose S values were already read into registers.
           exponents32(u, brow, row, c32, c1x2, l2e2, nm2);
-          if (full_tile) probs32<false>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
-          else probs32<true>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
+          if (full_tile) probs32<false, POLY>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
+          else probs32<true, POLY>(u, c32 ? mk1 : mk0, sum_a, sum_b, pk);
           tmem_st16(sbuf + 16 * c32, pk);
         }
         const float2 sa = f2unpack(add2(sum_a, sum_b));
@@ -478,15 +489,22 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 int fwd_bf16_rows_per_cta() { return kRows; }
 int fwd_bf16_key_tile() { return kBN; }
 
-cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream) {
-  if (args.N == 0) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel,
+template <int POLY>
+cudaError_t launch_fwd_poly(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(fwd_bf16_kernel<POLY>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((args.N + kBM - 1) / kBM, args.H, (args.row_end - args.row0 + kRows - 1) / kRows);
-  fwd_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k, maps.v, maps.bias,
-                                                           args);
+  fwd_bf16_kernel<POLY><<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k, maps.v,
+                                                                 maps.bias, args);
   return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_bf16(const FwdMaps &maps, const FwdArgs &args, cudaStream_t stream) {
+  if (args.N == 0) return cudaSuccess;
+  // the exp2 split: one key pair in four on the FMA pipe
+  return args.exp2_split ? launch_fwd_poly<4>(maps, args, stream)
+                         : launch_fwd_poly<0>(maps, args, stream);
 }
 
 }  // namespace tri

@@ -556,6 +556,29 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a pair of fp32 exponents on the FMA and integer pipes, for the share
+// of the softmax exponentials kept off the MUFU unit. Cody and Waite's range
+// reduction: j = round(x) (adding 1.5 * 2^23 rounds to an integer in the low
+// mantissa bits) and f = x - j in [-1/2, 1/2], both exact in fp32; 2^f by the
+// degree-4 polynomial of least maximum relative error on [-1/2, 1/2] (Remez
+// exchange; coefficients and the 2.7e-6 bound from gen_exp2_poly.py in this
+// directory); 2^j added to the exponent field. x is clamped below at -125 so the
+// result stays a normal number (about 2^-125 for anything smaller).
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  const float2 xs = f2unpack(x2);
+  const uint64_t x = f2pack(fmaxf(xs.x, -125.0f), fmaxf(xs.y, -125.0f));
+  const uint64_t t = add2(x, f2pack(12582912.0f, 12582912.0f));
+  const uint64_t j = add2(t, f2pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = fma2(j, f2pack(-1.0f, -1.0f), x);
+  uint64_t p = fma2(f, f2pack(0x1.3997d6p-7f, 0x1.3997d6p-7f), f2pack(0x1.ca1440p-5f, 0x1.ca1440p-5f));
+  p = fma2(p, f, f2pack(0x1.ec06dap-3f, 0x1.ec06dap-3f));
+  p = fma2(p, f, f2pack(0x1.62e0dcp-1f, 0x1.62e0dcp-1f));
+  p = fma2(p, f, f2pack(0x1.ffffe8p-1f, 0x1.ffffe8p-1f));
+  const float2 pp = f2unpack(p), tt = f2unpack(t);
+  return f2pack(__int_as_float(__float_as_int(pp.x) + (__float_as_int(tt.x) << 23)),
+                __int_as_float(__float_as_int(pp.y) + (__float_as_int(tt.y) << 23)));
+}
+
 // Three-input maximum (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
