@@ -30,14 +30,20 @@
  * query).
  *
  * Layout (all row-major, c fastest, no padding):
- *   q, k, v, gate, out, dout, dq, dk, dv, dgate : [N, N, H, c]
- *   bias, dbias                                 : [H, N, N]
- *   lse                                         : float32 [N, H, N]
- *   mask                                        : uint8, row stride
- *                                                 mask_row_stride (0: one key
- *                                                 mask [N] shared by every row;
- *                                                 N: a full [N, N] mask); NULL
- *                                                 means every key takes part.
+ *   q, k, v, gate, out, dout, dq, dk, dv, dgate : [B, N, N, H, c]
+ *   bias, dbias                                 : [B, H, N, N]
+ *   lse                                         : float32 [B, N, H, N]
+ *   mask                                        : uint8 [B, N] (mask_row_stride
+ *                                                 0: one key mask per problem,
+ *                                                 shared by its rows) or
+ *                                                 [B, N, N] (mask_row_stride N);
+ *                                                 NULL means every key takes part.
+ * B = batch (1 for a single problem, the leading dimension then absent); the B
+ * problems are independent. On the tensor-core path they share one launch of
+ * each kernel (attention row r of problem b is row b*N + r of the launch); the
+ * CUDA-core kernels take them one after another. The row-shard calls take
+ * B = 1 only; the on-chip-sum option applies to B = 1 (a batch takes the
+ * default backward); B*N is limited like N.
  *
  * Types. dtype BF16: every tensor above except lse and mask is bfloat16. With
  * c == 32 and N % 8 == 0 the contractions run on the tensor cores with fp32
@@ -106,6 +112,9 @@ typedef struct {
     int32_t dtype;            /* tri_attn_dtype                                 */
     int32_t variant;          /* tri_attn_variant                               */
     int64_t mask_row_stride;  /* 0 or N (ignored when mask is NULL)             */
+    int32_t batch;            /* independent problems of this size, stacked   */
+                              /* along a leading dimension (0 is taken as 1)  */
+    int32_t reserved;         /* must be 0                                    */
 } tri_attn_problem;
 
 /* Library version, (major << 16) | minor. */
@@ -307,7 +316,7 @@ tri_attn_status tri_attn_dbias_reduce(const float *partials, int32_t count, int6
  * library. Every GPU on which the library is used holds that array until the
  * process exits. A problem whose tri_attn_fwd_workspace_size() exceeds it is
  * rejected with TRI_ATTN_ERR_WORKSPACE before anything is enqueued (starting
- * node: any size up to the N limit; ending node: H*N*N*2 bytes must also fit).
+ * node: any size up to the N limit; ending node: B*H*N*N*2 bytes must also fit).
  *
  * The first call in a CUDA context looks up the array's device address with
  * that context's device current and keeps it, keyed by the context's unique

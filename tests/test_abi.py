@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import triangle_attention_b200 as ta
 from triangle_attention_b200 import build as tbuild
@@ -172,6 +173,66 @@ def test_onchip_sum_option_on_the_host(lib):
     assert rc == 0
     pair = 768 * 768 * 4 * 32
     assert nb >= 2 * pair + 8 * 768 * 768 * 4 + 8 * 4 * 3 * 36 * 128 * 32 * 2
+
+
+def test_batch_on_the_host(lib):
+    """The batch field: validation, workspace growth, the calls that take one
+    problem only, and launch counts (no CUDA call is made)."""
+    def B(batch, reserved=0, **kw):
+        p = P(**kw)
+        p.batch, p.reserved = batch, reserved
+        return p
+    assert ws_size(lib, B(-1))[0] == 1
+    assert ws_size(lib, B(2, reserved=1))[0] == 1
+    assert ws_size(lib, B(65, N=1024))[0] == 1           # B*N above the N limit
+    assert ws_size(lib, B(64, N=1024))[0] == 0
+    # batch 0 and 1 are the same problem
+    assert ws_size(lib, B(0)) == ws_size(lib, B(1))
+    # an ending-node batch holds a transposed bias per problem
+    rc1, n1 = ws_size(lib, B(1, variant=ta.ENDING))
+    rc3, n3 = ws_size(lib, B(3, variant=ta.ENDING))
+    assert rc1 == rc3 == 0 and n3 - n1 >= 2 * 2 * 4 * 64 * 64
+    # the backward's scratch (dU, D, tile contributions) grows with the batch
+    rc, nb1 = ws_size(lib, B(1, N=256), "bwd")
+    rc, nb3 = ws_size(lib, B(3, N=256), "bwd")
+    pair = 256 * 256 * 4 * 32
+    assert nb3 - nb1 >= 2 * (2 * pair + 4 * 256 * 256 * 4 + 3 * 2 * 2 * pair)
+    # row shards take one problem only
+    fake = ctypes.c_void_p(4096)
+    z = None
+    prob = B(2)
+    assert lib.tri_attn_fwd_rows(ctypes.byref(prob), 0, 8, *([fake] * 5), z, fake, fake, fake,
+                                 ctypes.c_size_t(1 << 40), z) == 2
+    assert lib.tri_attn_bwd_rows(ctypes.byref(prob), 0, 8, *([fake] * 5), z, *([fake] * 9),
+                                 ctypes.c_size_t(1 << 40), z) == 2
+    # launches: the tensor-core path runs a batch in one problem's launches; the
+    # CUDA-core kernels take the problems in turn; the on-chip-sum option falls
+    # back to the default backward for a batch
+    n = ctypes.c_int32(0)
+    for bwd in (0, 1):
+        assert lib.tri_attn_kernel_launches(ctypes.byref(B(3)), bwd, 0, ctypes.byref(n)) == 0
+        tc = n.value
+        assert lib.tri_attn_kernel_launches(ctypes.byref(B(1)), bwd, 0, ctypes.byref(n)) == 0
+        assert n.value == tc
+    assert lib.tri_attn_kernel_launches(ctypes.byref(B(3, c=16)), 0, 0, ctypes.byref(n)) == 0
+    assert n.value == 3
+    assert lib.tri_attn_kernel_launches(ctypes.byref(B(2, N=768)), 2, 0, ctypes.byref(n)) == 0
+    assert n.value == 4
+
+
+def test_problem_of_batched_tensors():
+    q = torch.empty((3, 16, 16, 2, 32), dtype=torch.bfloat16)
+    p = ta.problem(q, torch.ones((3, 16), dtype=torch.uint8), ta.STARTING)
+    assert (p.N, p.H, p.c, p.batch, p.mask_row_stride) == (16, 2, 32, 3, 0)
+    p = ta.problem(q, torch.ones((3, 16, 16), dtype=torch.uint8), ta.ENDING)
+    assert (p.batch, p.mask_row_stride) == (3, 16)
+    assert ta.problem(q[0], None, ta.STARTING).batch == 1
+    with pytest.raises(ValueError):
+        ta.problem(q, torch.ones((2, 16), dtype=torch.uint8), ta.STARTING)
+    with pytest.raises(ValueError):
+        ta.problem(q, torch.ones((16,), dtype=torch.uint8), ta.STARTING)
+    with pytest.raises(ValueError):
+        ta.problem(torch.empty((3, 16, 15, 2, 32)), None, ta.STARTING)
 
 
 def test_read_status_rejects_null(lib):

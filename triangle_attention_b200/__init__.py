@@ -116,7 +116,8 @@ class ProjProblem(ctypes.Structure):
 class Problem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("H", ctypes.c_int32), ("c", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("variant", ctypes.c_int32),
-                ("mask_row_stride", ctypes.c_int64)]
+                ("mask_row_stride", ctypes.c_int64), ("batch", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 def lib():
@@ -191,18 +192,26 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def problem(q: torch.Tensor, mask: Optional[torch.Tensor], variant: int) -> Problem:
-    if q.dim() != 4 or q.shape[0] != q.shape[1]:
-        raise ValueError(f"pair tensors must be [N, N, H, c], got {tuple(q.shape)}")
-    N, _, H, c = q.shape
+    """The problem of pair tensors [N, N, H, c], or of a batch [B, N, N, H, c]
+    (mask None, [N] or [N, N] unbatched; None, [B, N] or [B, N, N] batched)."""
+    if q.dim() not in (4, 5) or q.shape[-4] != q.shape[-3]:
+        raise ValueError(f"pair tensors must be [N, N, H, c] or [B, N, N, H, c], "
+                         f"got {tuple(q.shape)}")
+    N, _, H, c = q.shape[-4:]
+    B = q.shape[0] if q.dim() == 5 else 1
+    lead = q.dim() - 4
     stride = 0
     if mask is not None:
-        if mask.dim() == 1:
+        if mask.dim() - lead == 1 and mask.shape[-1] == N:
             stride = 0
-        elif mask.dim() == 2:
+        elif mask.dim() - lead == 2 and tuple(mask.shape[-2:]) == (N, N):
             stride = N
         else:
-            raise ValueError("mask must be [N] (shared by every row) or [N, N]")
-    return Problem(N, H, c, _dtype_code(q), variant, stride)
+            raise ValueError("mask must be [N] (shared by every row) or [N, N], with the "
+                             "pair tensors' leading batch dimension if they have one")
+        if lead and mask.shape[0] != B:
+            raise ValueError(f"mask batch {mask.shape[0]} != {B}")
+    return Problem(N, H, c, _dtype_code(q), variant, stride, B, 0)
 
 
 def _p(t: Optional[torch.Tensor]):
@@ -260,17 +269,18 @@ def _contig(*ts):
 
 def fwd(q, k, v, bias, gate, mask=None, variant: int = STARTING, out=None, lse=None, ws=None,
         stream=None, opts: Optional[LaunchOpts] = None, residual=None):
-    """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N].
-    residual (bf16 path): a tensor shaped like out that receives out's rounding
-    residual, for the compensated backward."""
+    """Forward. Returns (out, lse); out has q's dtype, lse is float32 [N, H, N]
+    ([B, N, H, N] for a batch [B, N, N, H, c], whose B problems share each
+    launch). residual (bf16 path): a tensor shaped like out that receives
+    out's rounding residual, for the compensated backward."""
     _contig(q, k, v, bias, gate, mask, residual)
     opts = _with_residual(opts, residual)
     prob = problem(q, mask, variant)
-    N, _, H, _ = q.shape
+    N, _, H, _ = q.shape[-4:]
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((N, H, N), dtype=torch.float32, device=q.device)
+        lse = torch.empty(q.shape[:-4] + (N, H, N), dtype=torch.float32, device=q.device)
     if ws is None:
         ws = workspace(fwd_workspace_size(prob), q.device)
     _check(lib().tri_attn_fwd_ex(ctypes.byref(prob), _p(q), _p(k), _p(v), _p(bias), _p(gate),
@@ -461,52 +471,27 @@ def mul_bwd(a, b, dt, direction: int = OUTGOING, grads=None, ws=None, stream=Non
     return da, db
 
 
-def _attention_fwd(q, k, v, bias, gate, mask, variant):
-    """fwd, unbatched or over a leading batch dimension (each element in turn)."""
-    if q.dim() == 4:
-        return fwd(q, k, v, bias, gate, mask, variant)
-    out = torch.empty_like(q)
-    B, N, _, H, _ = q.shape
-    lse = torch.empty((B, N, H, N), dtype=torch.float32, device=q.device)
-    for i in range(B):
-        fwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i], variant,
-            out=out[i], lse=lse[i])
-    return out, lse
-
-
-def _attention_bwd(q, k, v, bias, gate, mask, out, lse, dout, variant):
-    """bwd, unbatched or over a leading batch dimension."""
-    if q.dim() == 4:
-        return bwd(q, k, v, bias, gate, mask, out, lse, dout, variant)
-    dq, dk, dv, dgate = (torch.empty_like(t) for t in (q, k, v, gate))
-    dbias = torch.empty_like(bias)
-    for i in range(q.shape[0]):
-        bwd(q[i], k[i], v[i], bias[i], gate[i], None if mask is None else mask[i], out[i],
-            lse[i], dout[i], variant, grads=(dq[i], dk[i], dv[i], dbias[i], dgate[i]))
-    return dq, dk, dv, dbias, dgate
-
-
 class TriangleAttention(torch.autograd.Function):
     """out = TriangleAttention.apply(q, k, v, bias, gate, mask, variant).
 
     Unbatched: q, k, v, gate [N, N, H, c], bias [H, N, N], mask None, [N] or
     [N, N]. Batched: a leading batch dimension on every tensor (q [B, N, N, H,
     c], bias [B, H, N, N], mask None, [B, N] or [B, N, N]); each batch element
-    is an independent problem, run in turn on the current stream."""
+    is an independent problem, and the B problems share each kernel launch."""
 
     @staticmethod
     def forward(ctx, q, k, v, bias, gate, mask=None, variant=STARTING):
         ctx.mask = mask
         ctx.variant = variant
-        out, lse = _attention_fwd(q, k, v, bias, gate, mask, variant)
+        out, lse = fwd(q, k, v, bias, gate, mask, variant)
         ctx.save_for_backward(q, k, v, bias, gate, out, lse)
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, bias, gate, out, lse = ctx.saved_tensors
-        dq, dk, dv, dbias, dgate = _attention_bwd(q, k, v, bias, gate, ctx.mask, out, lse,
-                                                  dout.contiguous(), ctx.variant)
+        dq, dk, dv, dbias, dgate = bwd(q, k, v, bias, gate, ctx.mask, out, lse,
+                                       dout.contiguous(), ctx.variant)
         return dq, dk, dv, dbias, dgate, None, None
 
 
@@ -748,7 +733,7 @@ class TriangleAttentionBlock(torch.autograd.Function):
                 eps=1e-5):
         z = z.contiguous()
         x, stats, q, k, v, g, bias = proj_in_fwd(z, gamma, beta, w_qkvg, b_g, w_b, eps)
-        o, lse = _attention_fwd(q, k, v, bias, g, mask, variant)
+        o, lse = fwd(q, k, v, bias, g, mask, variant)
         y = proj_out_fwd(o, w_o, b_o)
         ctx.eps, ctx.mask, ctx.variant = eps, mask, variant
         ctx.save_for_backward(z, gamma, w_qkvg, w_b, w_o, x, stats, q, k, v, g, bias, o, lse)
@@ -758,8 +743,7 @@ class TriangleAttentionBlock(torch.autograd.Function):
     def backward(ctx, dy):
         z, gamma, w_qkvg, w_b, w_o, x, stats, q, k, v, g, bias, o, lse = ctx.saved_tensors
         do, dw_o, db_o = proj_out_bwd(o, w_o, dy.contiguous())
-        dq, dk, dv, dbias, dg = _attention_bwd(q, k, v, bias, g, ctx.mask, o, lse, do,
-                                               ctx.variant)
+        dq, dk, dv, dbias, dg = bwd(q, k, v, bias, g, ctx.mask, o, lse, do, ctx.variant)
         dz, dgamma, dbeta, dw_qkvg, db_g, dw_b = proj_in_bwd(z, gamma, w_qkvg, w_b, x, stats, dq,
                                                              dk, dv, dg, dbias, ctx.eps)
         return dz, dgamma, dbeta, dw_qkvg, db_g, dw_b, dw_o, db_o, None, None, None

@@ -6,6 +6,7 @@
 #include <cstdint>
 #include <cstring>
 #include <algorithm>
+#include <type_traits>
 #include <utility>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -37,14 +38,21 @@ tri_attn_status check_problem(const tri_attn_problem *p) {
   if (p->variant != TRI_ATTN_STARTING && p->variant != TRI_ATTN_ENDING)
     return TRI_ATTN_ERR_INVALID_ARG;
   if (p->mask_row_stride != 0 && p->mask_row_stride != p->N) return TRI_ATTN_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->reserved != 0 || (int64_t)std::max(p->batch, 1) * p->N > kMaxN)
+    return TRI_ATTN_ERR_INVALID_ARG;
   if (p->c > 64) return TRI_ATTN_ERR_UNSUPPORTED;
   return TRI_ATTN_OK;
 }
 
+// Problems in the batch (0 is taken as 1).
+int64_t batch_of(const tri_attn_problem *p) { return p->batch > 1 ? p->batch : 1; }
+
 // bf16 problems the tensor-core kernels take (head dimension 32, N a multiple of
 // 8); every other problem runs on the CUDA-core kernels.
 bool tc_shape(const tri_attn_problem *p) {
-  return p->dtype == TRI_ATTN_BF16 && p->c == 32 && p->N % 8 == 0;
+  // (the backward grid's third dimension counts heads x row groups x problems)
+  return p->dtype == TRI_ATTN_BF16 && p->c == 32 && p->N % 8 == 0 &&
+         (int64_t)p->H * batch_of(p) * tri::bwd_bf16_max_groups((int)p->N, p->H) <= 65535;
 }
 
 Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status) {
@@ -68,8 +76,9 @@ Frame make_frame(const tri_attn_problem *p, const uint8_t *mask, int32_t *status
   f.mask = mask;
   f.mask_stride = mask ? p->mask_row_stride : 0;
   f.status = status;
+  f.B = (int)batch_of(p);
   f.row0 = 0;
-  f.row_end = (int)p->N;
+  f.row_end = (int)(p->N * f.B);     // attention rows of every problem of the batch, in order
   return f;
 }
 
@@ -87,8 +96,27 @@ struct Carver {
   }
 };
 
+// Elements between consecutive problems of a batch.
+struct ProblemStrides {
+  int64_t pair, bias, lse, mask;
+};
+ProblemStrides problem_strides(const tri_attn_problem *p, bool has_mask) {
+  const int64_t N = p->N;
+  const int64_t es = p->dtype == TRI_ATTN_F32 ? 4 : 2;
+  return {N * N * p->H * p->c * es, (int64_t)p->H * N * N * es, N * p->H * N,
+          has_mask ? (p->mask_row_stride == N ? N * N : N) : 0};
+}
+// `base` advanced by `bytes` (pair and bias offsets are in bytes).
+template <typename T> T *at(T *base, int64_t bytes) {
+  return reinterpret_cast<T *>(reinterpret_cast<
+      typename std::conditional<std::is_const<T>::value, const char, char>::type *>(base) +
+                               bytes);
+}
+
+// Rows of packed key bits: one per attention row of every problem (a per-row
+// mask), else one per problem.
 int64_t mask_rows(const tri_attn_problem *p, bool has_mask) {
-  return (has_mask && p->mask_row_stride == p->N) ? p->N : 1;
+  return (has_mask && p->mask_row_stride == p->N) ? p->N * batch_of(p) : batch_of(p);
 }
 
 int64_t mask_words_per_row(const tri_attn_problem *p) { return ((p->N + 127) / 128) * 4; }
@@ -105,10 +133,11 @@ size_t carve_fwd(const tri_attn_problem *p, void *ws, bool per_row_mask, FwdWs *
   FwdWs w{};
   w.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
   if (tc_shape(p)) {
-    const int64_t rows = per_row_mask ? p->N : 1;
+    const int64_t rows = (per_row_mask ? p->N : 1) * batch_of(p);
     w.mask_bits = static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
     if (p->variant == TRI_ATTN_ENDING)
-      w.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * p->N * p->N));
+      w.biasT = static_cast<__nv_bfloat16 *>(
+          c.take(2 * (size_t)p->H * p->N * p->N * batch_of(p)));
   }
   if (out) *out = w;
   return c.off;
@@ -153,11 +182,13 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
   w.fw.status = static_cast<int32_t *>(c.take(sizeof(int32_t)));
   const size_t pair = (size_t)p->N * p->N * p->H * p->c;
   const size_t nn = (size_t)p->N * p->N;
+  const size_t B = (size_t)batch_of(p);
   if (tc_shape(p)) {
-    const int64_t rows = per_row_mask ? p->N : 1;
+    const int64_t rows = (per_row_mask ? p->N : 1) * (int64_t)B;
     w.fw.mask_bits =
         static_cast<uint32_t *>(c.take(sizeof(uint32_t) * rows * mask_words_per_row(p)));
-    w.tc = onchip && tri::bwd_tc_plan((int)p->N, p->H, sm_count(), &w.ntile, &w.ngroups, &w.ghl);
+    w.tc = onchip && B == 1 &&
+           tri::bwd_tc_plan((int)p->N, p->H, sm_count(), &w.ntile, &w.ngroups, &w.ghl);
     if (w.tc) {
       const int64_t gh = (int64_t)w.ngroups * p->H, nb = w.ntile;
       w.du = c.take(2 * pair);
@@ -168,13 +199,15 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
       w.flags = static_cast<int32_t *>(c.take(4 * (size_t)w.nflags));
     } else {
       if (p->variant == TRI_ATTN_ENDING)
-        w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn));
+        w.fw.biasT = static_cast<__nv_bfloat16 *>(c.take(2 * (size_t)p->H * nn * B));
+      // planned per problem, so that a problem of a batch is summed in the same
+      // order as the same problem alone
       tri::bwd_bf16_plan((int)p->N, p->H, (int)p->N, &w.ntile, &w.ngroups);
-      w.du = c.take(2 * pair);
-      w.D = static_cast<float *>(c.take(4 * nn * p->H));
-      w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
-      w.bpart_k = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
-      w.bpart_v = static_cast<__nv_bfloat16 *>(c.take(2 * pair * (size_t)w.ntile));
+      w.du = c.take(2 * pair * B);
+      w.D = static_cast<float *>(c.take(4 * nn * p->H * B));
+      w.bpart_q = static_cast<__nv_bfloat16 *>(c.take(2 * pair * B * (size_t)w.ntile));
+      w.bpart_k = static_cast<__nv_bfloat16 *>(c.take(2 * pair * B * (size_t)w.ntile));
+      w.bpart_v = static_cast<__nv_bfloat16 *>(c.take(2 * pair * B * (size_t)w.ntile));
     }
   } else {
     tri::f32_bwd_plan(make_frame(p, nullptr, nullptr), &w.ntile, &w.ngroups);
@@ -188,7 +221,7 @@ size_t carve_bwd(const tri_attn_problem *p, void *ws, bool per_row_mask, bool on
     // per-group dbias sums: also taken by a row-shard call, whose groups split
     // fewer rows but never number more than bwd_bf16_max_groups
     w.part_db = static_cast<float *>(
-        c.take(4 * nn * p->H * (size_t)tri::bwd_bf16_max_groups((int)p->N, p->H)));
+        c.take(4 * nn * p->H * B * (size_t)tri::bwd_bf16_max_groups((int)p->N, p->H)));
   } else {
     w.part_db = w.ngroups > 1
                     ? static_cast<float *>(c.take(4 * nn * p->H * (size_t)w.ngroups))
@@ -206,6 +239,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
+  // The driver's encoder wants a current context on this host thread, which a
+  // thread whose first CUDA work is a call into this library (a fresh thread,
+  // or a worker whose allocations all came from a cache) may not have yet:
+  // bind the runtime's primary context of the thread's current device.
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
   static EncodeTiledFn fn = nullptr;
   if (!fn) {
     void *ptr = nullptr;
@@ -218,28 +260,30 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// A pair tensor [.., .., H, 32] bf16 seen through the frame; dimensions by
-// increasing stride (c, h, then the smaller of x/r), box = one 128 x 32 tile.
+// A batch of pair tensors [batch][.., .., H, 32] bf16 seen through the frame;
+// dimensions by increasing stride (c, h, the smaller of x/r, the larger, the
+// problem), box = one 128 x 32 tile. The problem is a dimension of its own so
+// that a tile reaching past N reads zeros, not the next problem.
 bool encode_pair(CUtensorMap *m, const void *base, int64_t N, int64_t H, int64_t sR, int64_t sX,
-                 bool x_inner, uint32_t box_rows = 128) {
+                 bool x_inner, uint32_t box_rows = 128, int64_t batch = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[4] = {32, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)N};
-  cuuint64_t strides[3] = {64, (cuuint64_t)((x_inner ? sX : sR) * 2),
-                           (cuuint64_t)((x_inner ? sR : sX) * 2)};
-  cuuint32_t box[4] = {32, 1, x_inner ? box_rows : 1u, x_inner ? 1u : box_rows};
-  cuuint32_t es[4] = {1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+  cuuint64_t dims[5] = {32, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)batch};
+  cuuint64_t strides[4] = {64, (cuuint64_t)((x_inner ? sX : sR) * 2),
+                           (cuuint64_t)((x_inner ? sR : sX) * 2), (cuuint64_t)(N * N * H * 64)};
+  cuuint32_t box[5] = {32, 1, x_inner ? box_rows : 1u, x_inner ? 1u : box_rows, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
 }
 
 // Bias [H, N, N] bf16 in the variant frame (y fastest), box 64 keys x 128 queries.
-bool encode_bias(CUtensorMap *m, const void *base, int64_t N, int64_t H) {
+bool encode_bias(CUtensorMap *m, const void *base, int64_t N, int64_t H, int64_t batch = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)H};
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)N, (cuuint64_t)(H * batch)};
   cuuint64_t strides[2] = {(cuuint64_t)(N * 2), (cuuint64_t)(N * N * 2)};
   cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t es[3] = {1, 1, 1};
@@ -447,19 +491,32 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
   TRI_CHECK_PTR(q); TRI_CHECK_PTR(k); TRI_CHECK_PTR(v); TRI_CHECK_PTR(bias);
   TRI_CHECK_PTR(gate); TRI_CHECK_PTR(out); TRI_CHECK_PTR(lse);
   Frame f = make_frame(prob, mask, w.status);
+  const bool whole = row_count < 0;                  // every row of every problem
+  if (whole) row_count = f.row_end;
   f.row0 = (int)row0;
   f.row_end = (int)(row0 + row_count);
   if (row_count == 0) return TRI_ATTN_OK;
 
   if (!tc_shape(prob)) {
-    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic)
-    if (row0 != 0 || row_count != prob->N) return TRI_ATTN_ERR_UNSUPPORTED;
+    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic), one
+    // problem of the batch after another
+    if (!whole) return TRI_ATTN_ERR_UNSUPPORTED;
     cudaError_t e = cudaMemsetAsync(w.status, 0, sizeof(int32_t), stream);
     if (e == cudaSuccess) e = mark(opts, true, stream);
-    if (e == cudaSuccess)
+    const ProblemStrides ps = problem_strides(prob, mask != nullptr);
+    for (int64_t b = 0; e == cudaSuccess && b < batch_of(prob); ++b) {
+      Frame fb = make_frame(prob, mask ? mask + b * ps.mask : nullptr, w.status);
+      fb.B = 1;
+      fb.row_end = f.N;
       e = prob->dtype == TRI_ATTN_F32
-              ? core_fwd<float>(f, q, k, v, bias, gate, out, lse, stream)
-              : core_fwd<__nv_bfloat16>(f, q, k, v, bias, gate, out, lse, stream);
+              ? core_fwd<float>(fb, at(q, b * ps.pair), at(k, b * ps.pair), at(v, b * ps.pair),
+                                at(bias, b * ps.bias), at(gate, b * ps.pair), at(out, b * ps.pair),
+                                lse + b * ps.lse, stream)
+              : core_fwd<__nv_bfloat16>(fb, at(q, b * ps.pair), at(k, b * ps.pair),
+                                        at(v, b * ps.pair), at(bias, b * ps.bias),
+                                        at(gate, b * ps.pair), at(out, b * ps.pair),
+                                        lse + b * ps.lse, stream);
+    }
     if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
@@ -470,10 +527,11 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
   tri::FwdMaps maps;
   const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.biasT : bias;
   const uint32_t kv_rows = (uint32_t)tri::fwd_bf16_key_tile();
-  if (!encode_pair(&maps.q, q, prob->N, prob->H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.k, k, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows) ||
-      !encode_pair(&maps.v, v, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows) ||
-      !encode_bias(&maps.bias, bias_frame, prob->N, prob->H))
+  const int64_t B = f.B;
+  if (!encode_pair(&maps.q, q, prob->N, prob->H, f.sR, f.sX, x_inner, 128, B) ||
+      !encode_pair(&maps.k, k, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows, B) ||
+      !encode_pair(&maps.v, v, prob->N, prob->H, f.sR, f.sX, x_inner, kv_rows, B) ||
+      !encode_bias(&maps.bias, bias_frame, prob->N, prob->H, B))
     return TRI_ATTN_ERR_CUDA;
   tri::FwdArgs a;
   a.N = f.N;
@@ -490,13 +548,14 @@ tri_attn_status fwd_impl(const tri_attn_problem *prob, const void *q, const void
   a.out_res = static_cast<__nv_bfloat16 *>(opt_residual(opts));
   a.lse = lse;
   a.mask_bits = w.mask_bits;
-  a.mask_bits_stride = rows > 1 ? words : 0;
+  a.mask_bits_stride = words;
+  a.mask_per_row = per_row ? 1 : 0;
   a.status = w.status;
   cudaError_t e =
       tri::launch_mask_bits(f, w.mask_bits, rows, words, w.status, nullptr, 0, stream);
   if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
-    e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.biasT, f.N, f.H,
-                                   stream);
+    e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.biasT, f.N,
+                                   f.H * f.B, stream);
   if (e == cudaSuccess) e = mark(opts, true, stream);
   if (e == cudaSuccess) e = tri::launch_fwd_bf16(maps, a, stream);
   if (e == cudaSuccess) e = mark(opts, false, stream);
@@ -511,7 +570,7 @@ tri_attn_status tri_attn_fwd_ex(const tri_attn_problem *prob, const void *q, con
                                 size_t workspace_bytes, tri_attn_stream_t stream,
                                 const tri_attn_launch_opts *opts) {
   return fwd_impl(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes, stream,
-                  opts, 0, prob ? prob->N : 0);
+                  opts, 0, -1);
 }
 
 tri_attn_status tri_attn_fwd(const tri_attn_problem *prob, const void *q, const void *k,
@@ -557,13 +616,16 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
     TRI_CHECK_PTR(dbias);
   }
   Frame f = make_frame(prob, mask, w.fw.status);
+  const bool whole = row_count < 0;                  // every row of every problem
+  if (whole) row_count = f.row_end;
   f.row0 = (int)row0;
   f.row_end = (int)(row0 + row_count);
-  const bool shard = dbias_partial != nullptr || row0 != 0 || row_count != prob->N;
+  const bool shard = dbias_partial != nullptr || !whole;
   if (row_count == 0) return TRI_ATTN_OK;
 
   if (!tc_shape(prob)) {
-    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic)
+    // CUDA-core kernels (fp32, or bf16 storage with fp32 arithmetic), one
+    // problem of the batch after another on the same scratch
     if (shard) return TRI_ATTN_ERR_UNSUPPORTED;
     tri::F32BwdScratch s;
     s.du = static_cast<float *>(w.du);
@@ -576,12 +638,22 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
     s.ngroups = w.ngroups;
     cudaError_t e = cudaMemsetAsync(w.fw.status, 0, sizeof(int32_t), stream);
     if (e == cudaSuccess) e = mark(opts, true, stream);
-    if (e == cudaSuccess)
+    const ProblemStrides ps = problem_strides(prob, mask != nullptr);
+    for (int64_t b = 0; e == cudaSuccess && b < batch_of(prob); ++b) {
+      Frame fb = make_frame(prob, mask ? mask + b * ps.mask : nullptr, w.fw.status);
+      fb.B = 1;
+      fb.row_end = f.N;
+      const int64_t o = b * ps.pair;
       e = prob->dtype == TRI_ATTN_F32
-              ? core_bwd<float>(f, q, k, v, bias, gate, out, lse, dout, dq, dk, dv, dbias, dgate,
-                                s, stream)
-              : core_bwd<__nv_bfloat16>(f, q, k, v, bias, gate, out, lse, dout, dq, dk, dv,
-                                        dbias, dgate, s, stream);
+              ? core_bwd<float>(fb, at(q, o), at(k, o), at(v, o), at(bias, b * ps.bias),
+                                at(gate, o), at(out, o), lse + b * ps.lse, at(dout, o), at(dq, o),
+                                at(dk, o), at(dv, o), at(dbias, b * ps.bias), at(dgate, o), s,
+                                stream)
+              : core_bwd<__nv_bfloat16>(fb, at(q, o), at(k, o), at(v, o), at(bias, b * ps.bias),
+                                        at(gate, o), at(out, o), lse + b * ps.lse, at(dout, o),
+                                        at(dq, o), at(dk, o), at(dv, o), at(dbias, b * ps.bias),
+                                        at(dgate, o), s, stream);
+    }
     if (e == cudaSuccess) e = mark(opts, false, stream);
     return cuda_status(e);
   }
@@ -651,18 +723,23 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
 
   const void *bias_frame = prob->variant == TRI_ATTN_ENDING ? w.fw.biasT : bias;
   tri::BwdMaps maps;
-  if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.v, v, N, H, f.sR, f.sX, x_inner) ||
-      !encode_pair(&maps.du, w.du, N, H, N * H * 32, H * 32, true) ||
-      !encode_bias(&maps.bias, bias_frame, N, H))
+  const int64_t B = f.B;
+  if (!encode_pair(&maps.q, q, N, H, f.sR, f.sX, x_inner, 128, B) ||
+      !encode_pair(&maps.k, k, N, H, f.sR, f.sX, x_inner, 128, B) ||
+      !encode_pair(&maps.v, v, N, H, f.sR, f.sX, x_inner, 128, B) ||
+      !encode_pair(&maps.du, w.du, N, H, N * H * 32, H * 32, true, 128, B) ||
+      !encode_bias(&maps.bias, bias_frame, N, H, B))
     return TRI_ATTN_ERR_CUDA;
-  // row groups of this call's rows (the whole problem unless a row shard)
+  // row groups of each problem's rows (a row shard's rows when B = 1), planned
+  // as for the problem alone: each problem of a batch gets the results, bit for
+  // bit, that a call on it alone gives
+  const int64_t rows_per_problem = whole ? N : row_count;
   int ntile = w.ntile, ngroups = w.ngroups;
-  tri::bwd_bf16_plan(f.N, f.H, (int)row_count, &ntile, &ngroups);
+  tri::bwd_bf16_plan(f.N, f.H, (int)rows_per_problem, &ntile, &ngroups);
   tri::BwdArgs a;
   a.N = f.N;
   a.H = f.H;
+  a.B = f.B;
   a.row0 = f.row0;
   a.row_end = f.row_end;
   a.x_inner = x_inner ? 1 : 0;
@@ -673,7 +750,8 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
   a.lse = lse;
   a.D = w.D;
   a.mask_bits = w.fw.mask_bits;
-  a.mask_bits_stride = rows > 1 ? words : 0;
+  a.mask_bits_stride = words;
+  a.mask_per_row = per_row ? 1 : 0;
   a.part_q = w.bpart_q;
   a.part_k = w.bpart_k;
   a.part_v = w.bpart_v;
@@ -683,14 +761,14 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
   a.bX = f.bX;
   a.bY = f.bY;
   a.ngroups = ngroups;
-  a.rows_per_group = (int)((row_count + ngroups - 1) / ngroups);
+  a.rows_per_group = (int)((rows_per_problem + ngroups - 1) / ngroups);
   a.status = w.fw.status;
 
   cudaError_t e = tri::launch_mask_bits(f, w.fw.mask_bits, rows, words, w.fw.status, nullptr,
                                         0, stream);
   if (e == cudaSuccess && prob->variant == TRI_ATTN_ENDING)
     e = tri::launch_bias_transpose(static_cast<const __nv_bfloat16 *>(bias), w.fw.biasT, f.N,
-                                   f.H, stream);
+                                   f.H * f.B, stream);
   if (e == cudaSuccess)
     e = tri::launch_bwd_pre_bf16(f, static_cast<const __nv_bfloat16 *>(gate),
                                  static_cast<const __nv_bfloat16 *>(out),
@@ -706,10 +784,13 @@ tri_attn_status bwd_impl(const tri_attn_problem *prob, const void *q, const void
                                         static_cast<__nv_bfloat16 *>(dq),
                                         static_cast<__nv_bfloat16 *>(dk),
                                         static_cast<__nv_bfloat16 *>(dv), stream);
+  // the per-group sums are [group][B*H][N][N]: the reduction sees B*H heads
+  Frame fh = f;
+  fh.H = f.H * f.B;
   if (e == cudaSuccess && dbias_partial)
-    e = tri::launch_bias_reduce<float>(f, w.part_db, ngroups, dbias_partial, stream);
+    e = tri::launch_bias_reduce<float>(fh, w.part_db, ngroups, dbias_partial, stream);
   else if (e == cudaSuccess && ngroups > 1)
-    e = tri::launch_bias_reduce<__nv_bfloat16>(f, w.part_db, ngroups,
+    e = tri::launch_bias_reduce<__nv_bfloat16>(fh, w.part_db, ngroups,
                                                static_cast<__nv_bfloat16 *>(dbias), stream);
   return cuda_status(e);
 }
@@ -723,7 +804,7 @@ tri_attn_status tri_attn_bwd_ex(const tri_attn_problem *prob, const void *q, con
                                 void *dgate, void *workspace, size_t workspace_bytes,
                                 tri_attn_stream_t stream, const tri_attn_launch_opts *opts) {
   return bwd_impl(prob, q, k, v, bias, gate, mask, out, lse, dout, dq, dk, dv, dbias, nullptr,
-                  dgate, workspace, workspace_bytes, stream, opts, 0, prob ? prob->N : 0);
+                  dgate, workspace, workspace_bytes, stream, opts, 0, -1);
 }
 
 namespace {
@@ -743,7 +824,7 @@ tri_attn_status tri_attn_fwd_rows(const tri_attn_problem *prob, int64_t row_begi
                                   tri_attn_stream_t stream) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  if (!tc_shape(prob)) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!tc_shape(prob) || batch_of(prob) != 1) return TRI_ATTN_ERR_UNSUPPORTED;
   st = check_rows(prob, row_begin, row_count);
   if (st != TRI_ATTN_OK) return st;
   return fwd_impl(prob, q, k, v, bias, gate, mask, out, lse, workspace, workspace_bytes, stream,
@@ -759,7 +840,7 @@ tri_attn_status tri_attn_bwd_rows(const tri_attn_problem *prob, int64_t row_begi
                                   tri_attn_stream_t stream) {
   tri_attn_status st = check_problem(prob);
   if (st != TRI_ATTN_OK) return st;
-  if (!tc_shape(prob)) return TRI_ATTN_ERR_UNSUPPORTED;
+  if (!tc_shape(prob) || batch_of(prob) != 1) return TRI_ATTN_ERR_UNSUPPORTED;
   st = check_rows(prob, row_begin, row_count);
   if (st != TRI_ATTN_OK) return st;
   if (!dbias_partial && prob->N > 0) return TRI_ATTN_ERR_INVALID_ARG;
@@ -778,6 +859,7 @@ tri_attn_status tri_attn_dbias_reduce(const float *partials, int32_t count, int6
   Frame f{};
   f.N = (int)N;
   f.H = H;
+  f.B = 1;
   f.bX = N;
   f.bY = 1;
   return cuda_status(tri::launch_bias_reduce<__nv_bfloat16>(
@@ -805,12 +887,14 @@ tri_attn_status tri_attn_kernel_launches(const tri_attn_problem *prob, int backw
   int32_t n = 0;
   if (prob->N > 0) {
     if (!tc_shape(prob)) {
+      // one problem of the batch after another
+      const int32_t B = (int32_t)batch_of(prob);
       if (!backward) {
-        n = 1;
+        n = B;
       } else {
         BwdWs w;
         carve_bwd(prob, nullptr, false, false, &w);
-        n = 5 + (w.ngroups > 1 ? 1 : 0);  // pre, main, three reductions, dbias reduction
+        n = B * (5 + (w.ngroups > 1 ? 1 : 0));  // pre, main, three reductions, dbias reduction
       }
     } else {
       const int ending = prob->variant == TRI_ATTN_ENDING ? 1 : 0;

@@ -12,12 +12,13 @@
 namespace tri {
 
 // ------------------------------------------------------------------ forward --
-// Pair-tensor maps list their dimensions by increasing stride: (c, h, x, r)
+// Pair-tensor maps list their dimensions by increasing stride: (c, h, x, r, b)
 // when the query index has the smaller stride (x_inner = 1, starting node),
-// else (c, h, r, x); the box is 32 channels x 1 head x 128 queries x 1 row, so
-// a tile lands in shared memory as 128 rows of 64 bytes (64-byte swizzle).
-// The bias map is (y, x, h) in the variant frame, box (64, 128, 1), 128-byte
-// swizzle.
+// else (c, h, r, x, b), b the problem of a batch; the box is 32 channels x 1
+// head x 128 queries x 1 row x 1 problem, so a tile lands in shared memory as
+// 128 rows of 64 bytes (64-byte swizzle). The bias map is (y, x, b*H + h) in
+// the variant frame, box (64, 128, 1), 128-byte swizzle. Attention rows of the
+// batch count on across problems: row b*N + r is row r of problem b.
 struct FwdMaps {
   CUtensorMap q, k, v;
   CUtensorMap bias;
@@ -35,7 +36,8 @@ struct FwdArgs {
   __nv_bfloat16 *out_res;            // rounding residual of out (bf16) or null
   float *lse;
   const uint32_t *mask_bits;         // [rows][ceil(N/128)*4] key bits, 0 beyond N
-  int64_t mask_bits_stride;          // words per attention row (0: shared by all rows)
+  int64_t mask_bits_stride;          // words per row of bits
+  int mask_per_row;                  // 1: a row of bits per attention row, 0: one per problem
   int32_t *status;
 };
 
@@ -51,20 +53,21 @@ struct BwdMaps {
 };
 
 struct BwdArgs {
-  int N, H;
-  int row0, row_end;                 // attention rows of this launch
+  int N, H, B;                       // B problems of N x N pairs and H heads
+  int row0, row_end;                 // attention rows of this launch (of the batch)
   int x_inner;
   int nb;                            // tiles per axis, ceil(N / 128)
   float scale;
   int64_t sR, sX;                    // pair strides of the variant frame (outputs)
-  const float *lse;                  // [N, H, N] natural log
-  const float *D;                    // [N, H, N] sum_c dout * out
+  const float *lse;                  // [B*N, H, N] natural log
+  const float *D;                    // [B*N, H, N] sum_c dout * out
   const uint32_t *mask_bits;
-  int64_t mask_bits_stride;
-  // bf16 tile contributions, [tile][row][H][2][N][16] (16-channel halves):
+  int64_t mask_bits_stride;          // words per row of bits
+  int mask_per_row;                  // 1: a row of bits per attention row, 0: one per problem
+  // bf16 tile contributions, [tile][B*N rows][H][2][N][16] (16-channel halves):
   // part_q over key tiles yb, part_k and part_v over query tiles xb
   __nv_bfloat16 *part_q, *part_k, *part_v;
-  float *part_db;                    // [ngroups][H, N, N] variant frame (used when dbias is null)
+  float *part_db;                    // [ngroups][B*H, N, N] variant frame (used when dbias is null)
   __nv_bfloat16 *dbias;              // final dbias (one row group covering every row), else null
   int64_t bX, bY;                    // dbias strides of the variant frame
   int ngroups, rows_per_group;

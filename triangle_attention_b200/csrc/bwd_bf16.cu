@@ -218,10 +218,13 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = a.N, H = a.H;
   const int xb = blockIdx.x, yb = blockIdx.y;
-  const int h = blockIdx.z % H, g = blockIdx.z / H;
-  const int r0 = a.row0 + g * a.rows_per_group;
-  const int r1 = min(a.row_end, r0 + a.rows_per_group);
+  // blockIdx.z = (problem pb, row group g, head h), h fastest; rows count on
+  // across the problems of a batch (row pb*N + r is row r of problem pb)
+  const int h = blockIdx.z % H, g = (blockIdx.z / H) % a.ngroups, pb = blockIdx.z / H / a.ngroups;
+  const int r0 = a.row0 + pb * N + g * a.rows_per_group;
+  const int r1 = min(min(a.row_end, (pb + 1) * N), r0 + a.rows_per_group);
   const int T = max(0, r1 - r0);
+  const int rb0 = r0 - pb * N;        // r0's row inside its problem
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -261,9 +264,9 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int s = 0; s < kStages; ++s) armed[s] = -1;
       bool ok = true;
       mbar_arrive_expect_tx(&ctl.bias_full, kSqTileBytes);
-      tma_load_3d(smem + kOffBias, &tm_b, &ctl.bias_full, yb * kBN, xb * kBM, h);
+      tma_load_3d(smem + kOffBias, &tm_b, &ctl.bias_full, yb * kBN, xb * kBM, pb * H + h);
       tma_load_3d(smem + kOffBias + kSqTileBytes / 2, &tm_b, &ctl.bias_full, yb * kBN + 64,
-                  xb * kBM, h);
+                  xb * kBM, pb * H + h);
       // lse and D rows of this query tile: min(128, N - x0) floats (N % 8 == 0)
       const uint32_t row_bytes = (uint32_t)min(kBM, N - xb * kBM) * 4u;
       for (int it = 0; it < T; ++it) {
@@ -273,38 +276,40 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           ok = false;
           break;
         }
-        const int r = r0 + it;
+        const int r = r0 + it, rb = rb0 + it;
         uint8_t *in = smem + kOffIn + st * kStageBytes;
         mbar_arrive_expect_tx(&ctl.in_full[st], 4 * kPairTileBytes + 2 * row_bytes + 16);
         if (a.x_inner) {
-          tma_load_4d(in, &tm_q, &ctl.in_full[st], 0, h, xb * kBM, r);
-          tma_load_4d(in + 2 * kPairTileBytes, &tm_k, &ctl.in_full[st], 0, h, yb * kBN, r);
-          tma_load_4d(in + 3 * kPairTileBytes, &tm_v, &ctl.in_full[st], 0, h, yb * kBN, r);
+          tma_load_5d(in, &tm_q, &ctl.in_full[st], 0, h, xb * kBM, rb, pb);
+          tma_load_5d(in + 2 * kPairTileBytes, &tm_k, &ctl.in_full[st], 0, h, yb * kBN, rb, pb);
+          tma_load_5d(in + 3 * kPairTileBytes, &tm_v, &ctl.in_full[st], 0, h, yb * kBN, rb, pb);
         } else {
-          tma_load_4d(in, &tm_q, &ctl.in_full[st], 0, h, r, xb * kBM);
-          tma_load_4d(in + 2 * kPairTileBytes, &tm_k, &ctl.in_full[st], 0, h, r, yb * kBN);
-          tma_load_4d(in + 3 * kPairTileBytes, &tm_v, &ctl.in_full[st], 0, h, r, yb * kBN);
+          tma_load_5d(in, &tm_q, &ctl.in_full[st], 0, h, rb, xb * kBM, pb);
+          tma_load_5d(in + 2 * kPairTileBytes, &tm_k, &ctl.in_full[st], 0, h, rb, yb * kBN, pb);
+          tma_load_5d(in + 3 * kPairTileBytes, &tm_v, &ctl.in_full[st], 0, h, rb, yb * kBN, pb);
         }
-        tma_load_4d(in + kPairTileBytes, &tm_du, &ctl.in_full[st], 0, h, xb * kBM, r);
+        tma_load_5d(in + kPairTileBytes, &tm_du, &ctl.in_full[st], 0, h, xb * kBM, rb, pb);
         const int64_t lo = ((int64_t)r * H + h) * N + xb * kBM;
         uint8_t *rd = smem + kOffRow + st * kRowBytes;
         bulk_load(rd + kStLse, a.lse + lo, row_bytes, &ctl.in_full[st]);
         bulk_load(rd + kStD, a.D + lo, row_bytes, &ctl.in_full[st]);
-        bulk_load(rd + kStMask, a.mask_bits + (int64_t)r * a.mask_bits_stride + yb * 4, 16,
+        bulk_load(rd + kStMask,
+                  a.mask_bits + (int64_t)(a.mask_per_row ? r : pb) * a.mask_bits_stride + yb * 4,
+                  16,
                   &ctl.in_full[st]);
         armed[st] = it / kStages;
         if (kL2Ahead > 0 && it + kL2Ahead < T) {
-          const int rp = r + kL2Ahead;
+          const int rp = r + kL2Ahead, rbp = rb + kL2Ahead;
           if (a.x_inner) {
-            tma_prefetch_l2_4d(&tm_q, 0, h, xb * kBM, rp);
-            tma_prefetch_l2_4d(&tm_k, 0, h, yb * kBN, rp);
-            tma_prefetch_l2_4d(&tm_v, 0, h, yb * kBN, rp);
+            tma_prefetch_l2_5d(&tm_q, 0, h, xb * kBM, rbp, pb);
+            tma_prefetch_l2_5d(&tm_k, 0, h, yb * kBN, rbp, pb);
+            tma_prefetch_l2_5d(&tm_v, 0, h, yb * kBN, rbp, pb);
           } else {
-            tma_prefetch_l2_4d(&tm_q, 0, h, rp, xb * kBM);
-            tma_prefetch_l2_4d(&tm_k, 0, h, rp, yb * kBN);
-            tma_prefetch_l2_4d(&tm_v, 0, h, rp, yb * kBN);
+            tma_prefetch_l2_5d(&tm_q, 0, h, rbp, xb * kBM, pb);
+            tma_prefetch_l2_5d(&tm_k, 0, h, rbp, yb * kBN, pb);
+            tma_prefetch_l2_5d(&tm_v, 0, h, rbp, yb * kBN, pb);
           }
-          tma_prefetch_l2_4d(&tm_du, 0, h, xb * kBM, rp);
+          tma_prefetch_l2_5d(&tm_du, 0, h, xb * kBM, rbp, pb);
           const int64_t lp = ((int64_t)rp * H + h) * N + xb * kBM;
           bulk_prefetch_l2(a.lse + lp, row_bytes);
           bulk_prefetch_l2(a.D + lp, row_bytes);
@@ -419,7 +424,7 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // be summed over query tiles). Contributions are stored piece-major,
     // [t][r][h][j&1][i][16] (t the tile summed over, i the query or key): a lane
     // writes its 16 channels with one 32-byte store and a warp store covers 1 KB.
-    const int64_t pair = (int64_t)N * N * H * kC;
+    const int64_t pair = (int64_t)a.B * N * N * H * kC;   // one tile's contributions
     // piece j's 16-channel plane of row r in one tensor's contributions
     auto piece_base = [&](int j, int r) -> __nv_bfloat16 * {
       __nv_bfloat16 *buf = j < 2 ? a.part_q : j < 4 ? a.part_k : a.part_v;
@@ -529,7 +534,7 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (ok && T > 0) ok = drain(T - 1);
     // the pair-bias gradient block: summed over every row of the group
     if (ok && x < N) {
-      const int64_t hb = (int64_t)h * N * N;
+      const int64_t hb = ((int64_t)pb * H + h) * N * N;
       const int y0 = yb * kBN + kbase;
 #pragma unroll
       for (int e = 0; e < kKeys; e += 2) {
@@ -542,7 +547,7 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (a.dbias)
               a.dbias[hb + (int64_t)x * a.bX + (int64_t)y * a.bY] = __float2bfloat16_rn(val);
             else
-              a.part_db[((int64_t)g * H + h) * N * N + (int64_t)x * N + y] = val;
+              a.part_db[(((int64_t)g * a.B + pb) * H + h) * N * N + (int64_t)x * N + y] = val;
           }
         }
       }
@@ -583,7 +588,7 @@ cudaError_t launch_bwd_bf16(const BwdMaps &maps, const BwdArgs &args, cudaStream
   cudaError_t e = cudaFuncSetAttribute(bwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(args.nb, args.nb, args.H * args.ngroups);
+  dim3 grid(args.nb, args.nb, args.H * args.ngroups * args.B);
   bwd_bf16_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k, maps.v, maps.du,
                                                            maps.bias, args);
   return cudaGetLastError();

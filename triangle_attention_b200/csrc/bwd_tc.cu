@@ -355,15 +355,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t *rb = smem + kOffRow + st * kRowBytes;
         mbar_arrive_expect_tx(&ctl.in_full[st], kStageBytes + lse_bytes + 16);
         if (a.x_inner) {
-          tma_load_4d(in, &tm_q, &ctl.in_full[st], 0, h, X * kT, r);
-          tma_load_4d(in + 2 * kTileBytes, &tm_k, &ctl.in_full[st], 0, h, Y * kT, r);
-          tma_load_4d(in + 3 * kTileBytes, &tm_v, &ctl.in_full[st], 0, h, Y * kT, r);
+          tma_load_5d(in, &tm_q, &ctl.in_full[st], 0, h, X * kT, r, 0);
+          tma_load_5d(in + 2 * kTileBytes, &tm_k, &ctl.in_full[st], 0, h, Y * kT, r, 0);
+          tma_load_5d(in + 3 * kTileBytes, &tm_v, &ctl.in_full[st], 0, h, Y * kT, r, 0);
         } else {
-          tma_load_4d(in, &tm_q, &ctl.in_full[st], 0, h, r, X * kT);
-          tma_load_4d(in + 2 * kTileBytes, &tm_k, &ctl.in_full[st], 0, h, r, Y * kT);
-          tma_load_4d(in + 3 * kTileBytes, &tm_v, &ctl.in_full[st], 0, h, r, Y * kT);
+          tma_load_5d(in, &tm_q, &ctl.in_full[st], 0, h, r, X * kT, 0);
+          tma_load_5d(in + 2 * kTileBytes, &tm_k, &ctl.in_full[st], 0, h, r, Y * kT, 0);
+          tma_load_5d(in + 3 * kTileBytes, &tm_v, &ctl.in_full[st], 0, h, r, Y * kT, 0);
         }
-        tma_load_4d(in + kTileBytes, &tm_du, &ctl.in_full[st], 0, h, X * kT, r);
+        tma_load_5d(in + kTileBytes, &tm_du, &ctl.in_full[st], 0, h, X * kT, r, 0);
         bulk_load(rb, a.LD + ((int64_t)r * H + h) * (N / 2) + X * (kT / 2), lse_bytes,
                   &ctl.in_full[st]);
         bulk_load(rb + kLDBytes, a.mask_bits + (int64_t)r * a.mask_bits_stride + Y * 4, 16,
@@ -376,15 +376,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int rp = r + kStages + 1;
         if (rp < r1) {
           if (a.x_inner) {
-            tma_prefetch_l2_4d(&tm_q, 0, h, X * kT, rp);
-            tma_prefetch_l2_4d(&tm_k, 0, h, Y * kT, rp);
-            tma_prefetch_l2_4d(&tm_v, 0, h, Y * kT, rp);
+            tma_prefetch_l2_5d(&tm_q, 0, h, X * kT, rp, 0);
+            tma_prefetch_l2_5d(&tm_k, 0, h, Y * kT, rp, 0);
+            tma_prefetch_l2_5d(&tm_v, 0, h, Y * kT, rp, 0);
           } else {
-            tma_prefetch_l2_4d(&tm_q, 0, h, rp, X * kT);
-            tma_prefetch_l2_4d(&tm_k, 0, h, rp, Y * kT);
-            tma_prefetch_l2_4d(&tm_v, 0, h, rp, Y * kT);
+            tma_prefetch_l2_5d(&tm_q, 0, h, rp, X * kT, 0);
+            tma_prefetch_l2_5d(&tm_k, 0, h, rp, Y * kT, 0);
+            tma_prefetch_l2_5d(&tm_v, 0, h, rp, Y * kT, 0);
           }
-          tma_prefetch_l2_4d(&tm_du, 0, h, X * kT, rp);
+          tma_prefetch_l2_5d(&tm_du, 0, h, X * kT, rp, 0);
         }
       }
       // every copy this thread started lands before the CTA exits

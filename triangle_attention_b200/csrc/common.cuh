@@ -23,9 +23,11 @@ struct Frame {
   const uint8_t *mask;
   int64_t mask_stride;
   int32_t *status;  // device status word, never null inside a launch
-  // attention rows [row0, row_end) of the variant frame that this call computes
-  // (0 and N unless the caller asked for a row shard)
+  // attention rows [row0, row_end) of the variant frame that this call computes:
+  // rows of B stacked problems count on, row b*N + r being row r of problem b
+  // (0 and B*N unless the caller asked for a row shard)
   int row0, row_end;
+  int B;  // problems in the batch (the CUDA-core kernels take one at a time)
 };
 
 // Record a device-side failure (first writer wins; the value never goes back

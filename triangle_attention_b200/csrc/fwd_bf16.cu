@@ -169,8 +169,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int lane = threadIdx.x & 31;
   const int N = a.N;
   const int xb = blockIdx.x, h = blockIdx.y;
-  const int r0 = a.row0 + blockIdx.z * kRows;
+  const int r0 = a.row0 + blockIdx.z * kRows;   // row of the stacked problems
   const int nrows = min(kRows, a.row_end - r0);
+  // problem of these rows and the first one's row inside it (N % 8 == 0, so the
+  // 8 rows of a CTA belong to one problem)
+  const int pb = r0 / N;
+  const int rb0 = r0 - pb * N;
   const int nkb = (N + kBN - 1) / kBN;
   const int T = nkb * kRows;        // (key tile, row) steps, row fastest
 
@@ -218,9 +222,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int rr = 0; rr < kRows; ++rr) {
         uint8_t *dst = smem + kOffQ + rr * kQTileBytes;
         if (a.x_inner)
-          tma_load_4d(dst, &tm_q, &ctl.q_full, 0, h, xb * kBM, r0 + rr);
+          tma_load_5d(dst, &tm_q, &ctl.q_full, 0, h, xb * kBM, rb0 + rr, pb);
         else
-          tma_load_4d(dst, &tm_q, &ctl.q_full, 0, h, r0 + rr, xb * kBM);
+          tma_load_5d(dst, &tm_q, &ctl.q_full, 0, h, rb0 + rr, xb * kBM, pb);
       }
       int it = 0;
       for (int kb = 0; kb < nkb && ok; ++kb) {
@@ -231,7 +235,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mbar_arrive_expect_tx(&ctl.bias_full[bb], kBiasTileBytes);
         tma_load_3d(smem + kOffB + bb * kBiasTileBytes, &tm_b, &ctl.bias_full[bb], kb * kBN,
-                    xb * kBM, h);
+                    xb * kBM, pb * a.H + h);
         armed_b[bb] = kb >> 1;
         for (int rr = 0; rr < kRows; ++rr, ++it) {
           const int st = it % kStages;
@@ -244,15 +248,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           uint8_t *kd = smem + kOffK + st * kKVTileBytes;
           uint8_t *vd = smem + kOffV + st * kKVTileBytes;
           if (a.x_inner) {
-            tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
-            tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, kb * kBN, r0 + rr);
+            tma_load_5d(kd, &tm_k, &ctl.kv_full[st], 0, h, kb * kBN, rb0 + rr, pb);
+            tma_load_5d(vd, &tm_v, &ctl.kv_full[st], 0, h, kb * kBN, rb0 + rr, pb);
           } else {
-            tma_load_4d(kd, &tm_k, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
-            tma_load_4d(vd, &tm_v, &ctl.kv_full[st], 0, h, r0 + rr, kb * kBN);
+            tma_load_5d(kd, &tm_k, &ctl.kv_full[st], 0, h, rb0 + rr, kb * kBN, pb);
+            tma_load_5d(vd, &tm_v, &ctl.kv_full[st], 0, h, rb0 + rr, kb * kBN, pb);
           }
           // the 4 key-bit words of the 128 keys around this tile (16-byte aligned)
           bulk_load(smem + kOffMask + st * 16,
-                    a.mask_bits + (int64_t)(r0 + rr) * a.mask_bits_stride + (kb >> 1) * 4, 16,
+                    a.mask_bits + (int64_t)(a.mask_per_row ? r0 + rr : pb) * a.mask_bits_stride +
+                        (kb >> 1) * 4,
+                    16,
                     &ctl.kv_full[st]);
           armed_kv[st] = it / kStages;
         }
@@ -447,7 +453,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       const float l = l_r[0];
       const float inv = l > 0.0f ? rcp_approx(l) : 0.0f;
-      const int64_t off = (int64_t)r * a.sR + (int64_t)x * a.sX + (int64_t)h * kC;
+      const int64_t off = (int64_t)pb * N * N * a.H * kC + (int64_t)(rb0 + rr) * a.sR +
+                          (int64_t)x * a.sX + (int64_t)h * kC;
       const uint4 *gp = reinterpret_cast<const uint4 *>(a.gate + off);
       uint4 *op = reinterpret_cast<uint4 *>(a.out + off);
       uint4 *rp = a.out_res ? reinterpret_cast<uint4 *>(a.out_res + off) : nullptr;

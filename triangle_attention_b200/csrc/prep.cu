@@ -18,8 +18,10 @@ int blocks_for(int64_t n, int threads) {
   return (int)(b < 1 ? 1 : b);
 }
 
-// One word = 32 keys of one attention row; bit j set when key 32*w + j exists
-// and takes part. Also resets the call's status word.
+// One word = 32 keys of one row of the mask; bit j set when key 32*w + j exists
+// and takes part. The mask's rows are N bytes apart: one per attention row of
+// every problem (a per-row mask) or one per problem. Also resets the call's
+// status word.
 __global__ void mask_bits_kernel(Frame f, uint32_t *__restrict__ bits, int64_t rows,
                                  int64_t words_per_row, int32_t *status,
                                  int32_t *__restrict__ zero, int64_t nzero) {
@@ -35,7 +37,7 @@ __global__ void mask_bits_kernel(Frame f, uint32_t *__restrict__ bits, int64_t r
     uint32_t b = 0;
     for (int j = 0; j < 32; ++j) {
       const int64_t y = y0 + j;
-      if (y < f.N && (!f.mask || f.mask[r * f.mask_stride + y] != 0)) b |= 1u << j;
+      if (y < f.N && (!f.mask || f.mask[r * f.N + y] != 0)) b |= 1u << j;
     }
     bits[w] = b;
   }
@@ -61,9 +63,10 @@ __device__ __forceinline__ float sigmoid_fast(float g) {
   return rcp_approx(1.0f + ex2_approx(-g * 1.4426950408889634f));
 }
 
-// One thread per 8 channels (16 bytes) of one (storage row a, storage column b,
-// head h), so a warp reads 512 contiguous bytes of each tensor per load; the
-// four threads of one (a, b, h) sum their parts of D with two shuffles.
+// One thread per 8 channels (16 bytes) of one (problem p, storage row a, storage
+// column b, head h), so a warp reads 512 contiguous bytes of each tensor per
+// load; the four threads of one (p, a, b, h) sum their parts of D with two
+// shuffles. Rows r of problem p count as attention row p*N + r of the batch.
 __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ gate,
                                     const __nv_bfloat16 *__restrict__ out,
                                     const __nv_bfloat16 *__restrict__ out_res,
@@ -72,7 +75,7 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
                                     __nv_bfloat16 *__restrict__ dgate,
                                     const float *__restrict__ lse, float *__restrict__ LD,
                                     int ending) {
-  const int64_t total = (int64_t)f.N * f.N * f.H * 4;
+  const int64_t total = (int64_t)f.B * f.N * f.N * f.H * 4;
   const unsigned group = 0xfu << (threadIdx.x & 28);   // the 4 lanes of one (a, b, h)
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
        w += (int64_t)gridDim.x * blockDim.x) {
@@ -80,8 +83,9 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
     const int64_t e = w >> 2;                                  // (a, b, h)
     const int h = (int)(e % f.H);
     const int64_t b = (e / f.H) % f.N;
-    const int64_t aa = e / ((int64_t)f.H * f.N);
-    const int64_t r = ending ? b : aa;
+    const int64_t pa = e / ((int64_t)f.H * f.N);              // p*N + a
+    const int64_t aa = pa % f.N;
+    const int64_t r = pa - aa + (ending ? b : aa);             // row of the batch
     const int64_t x = ending ? aa : b;
     if (r < f.row0 || r >= f.row_end) continue;      // another call's row shard
     const int64_t so = w * 8;                                  // storage offset
@@ -137,9 +141,10 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
                                            float scale, __nv_bfloat16 *__restrict__ dq,
                                            __nv_bfloat16 *__restrict__ dk,
                                            __nv_bfloat16 *__restrict__ dv) {
-  const int64_t pair = (int64_t)f.N * f.N * f.H * 32;
-  // 16-byte groups per attention row of one tensor and tile; rows are outermost,
-  // so this call's row shard is one contiguous range of groups
+  const int64_t pair = (int64_t)f.N * f.N * f.H * 32;          // one problem
+  const int64_t tile = pair * f.B;                               // one tile's contributions
+  // 16-byte groups per attention row of one tensor and tile; rows (of the
+  // batch) are outermost, so this call's row shard is one contiguous range
   const int64_t per_row = (int64_t)f.N * f.H * 4;
   const int64_t first = (int64_t)f.row0 * per_row;
   const int64_t per = (int64_t)(f.row_end - f.row0) * per_row;
@@ -158,7 +163,7 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
       uint4 v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u)
-        if (t0 + u < nb) v[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (t0 + u) * pair));
+        if (t0 + u < nb) v[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (t0 + u) * tile));
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         if (t0 + u >= nb) break;
@@ -176,8 +181,9 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
     const int half = (int)((gidx >> 1) / f.N % 2);
     const int h = (int)((gidx >> 1) / ((int64_t)f.N * 2) % f.H);
     const int64_t r = (gidx >> 1) / ((int64_t)f.N * 2 * f.H);
-    __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + r * f.sR + i * f.sX +
-                         (int64_t)h * 32 + half * 16 + c8 * 8;
+    const int64_t p = r / f.N;                                     // problem of row r
+    __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + p * pair +
+                         (r - p * f.N) * f.sR + i * f.sX + (int64_t)h * 32 + half * 16 + c8 * 8;
     *reinterpret_cast<uint4 *>(dst) =
         make_uint4(pack_bf16(acc[0] * sc, acc[1] * sc), pack_bf16(acc[2] * sc, acc[3] * sc),
                    pack_bf16(acc[4] * sc, acc[5] * sc), pack_bf16(acc[6] * sc, acc[7] * sc));
@@ -218,7 +224,7 @@ cudaError_t launch_bwd_pre_bf16(const Frame &f, const __nv_bfloat16 *gate,
                                 const __nv_bfloat16 *dout,
                                 __nv_bfloat16 *du, float *D, __nv_bfloat16 *dgate,
                                 const float *lse, float *LD, cudaStream_t stream) {
-  const int64_t total = (int64_t)f.N * f.N * f.H * 4;
+  const int64_t total = (int64_t)f.B * f.N * f.N * f.H * 4;
   if (total == 0) return cudaSuccess;
   const int ending = f.variant == 1 ? 1 : 0;
   bwd_pre_bf16_kernel<<<blocks_for(total, 256), 256, 0, stream>>>(f, gate, out, out_res, dout,

@@ -104,12 +104,12 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, uint64_t
       : "memory");
 }
 
-__device__ __forceinline__ void tma_load_4d(void *dst, const void *map, uint64_t *bar, int c0,
-                                            int c1, int c2, int c3) {
+__device__ __forceinline__ void tma_load_5d(void *dst, const void *map, uint64_t *bar, int c0,
+                                            int c1, int c2, int c3, int c4) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
 
@@ -137,10 +137,10 @@ __device__ __forceinline__ void bulk_wait_all() {
 }
 
 // Prefetch of a 4-D tensor-map tile into L2 (no shared memory, no barrier).
-__device__ __forceinline__ void tma_prefetch_l2_4d(const void *map, int c0, int c1, int c2,
-                                                   int c3) {
-  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global [%0, {%1, %2, %3, %4}];" ::"l"(map),
-               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+__device__ __forceinline__ void tma_prefetch_l2_5d(const void *map, int c0, int c1, int c2,
+                                                   int c3, int c4) {
+  asm volatile("cp.async.bulk.prefetch.tensor.5d.L2.global [%0, {%1, %2, %3, %4, %5}];" ::"l"(map),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
                : "memory");
 }
 
