@@ -176,6 +176,155 @@ __global__ void colsum_strided_kernel(const __nv_bfloat16 *__restrict__ m, int64
   }
 }
 
+// ------------------------------------------------ 64 x 64 tiled versions --
+// For shapes whose both sides are multiples of 64 (every shape of the update:
+// c is a multiple of 64 and R = N*N with N % 8 == 0). A tile moves through
+// shared memory as [64 channels][32 position pairs] words, each word the bf16
+// values of two consecutive positions: warp w reads (or writes) channels
+// 8w .. 8w+7 of 64 positions with one 16-byte access per position, and the
+// channel-major side moves 16 bytes (8 positions) per access, eight lanes
+// covering 128 contiguous bytes. Both shared-memory passes are free of bank
+// conflicts. Arithmetic and rounding are those of the kernels above.
+constexpr int kT = 64;
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ float lo_of(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_of(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 8 bf16 of a uint4 as floats
+__device__ __forceinline__ void unpack8(const uint4 v, float (&o)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    o[2 * e] = lo_of(w[e]);
+    o[2 * e + 1] = hi_of(w[e]);
+  }
+}
+
+__global__ void __launch_bounds__(256) gate_in_fwd_tiled(const __nv_bfloat16 *__restrict__ pg,
+                                                         int64_t R, int c, int64_t ldpg,
+                                                         __nv_bfloat16 *__restrict__ a_cm,
+                                                         __nv_bfloat16 *__restrict__ b_cm) {
+  __shared__ __align__(16) uint32_t ta[kT][kT / 2], tb[kT][kT / 2];
+  const int64_t p0 = (int64_t)blockIdx.x * kT;
+  const int ch0 = blockIdx.y * kT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cg = ch0 + warp * 8;
+  float av[2][8], bv[2][8];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const __nv_bfloat16 *row = pg + (p0 + 2 * lane + k) * ldpg + cg;
+    float ap[8], ag[8], bp[8], bg[8];
+    unpack8(*reinterpret_cast<const uint4 *>(row), ap);
+    unpack8(*reinterpret_cast<const uint4 *>(row + c), ag);
+    unpack8(*reinterpret_cast<const uint4 *>(row + 2 * c), bp);
+    unpack8(*reinterpret_cast<const uint4 *>(row + 3 * c), bg);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      av[k][e] = sigm(ag[e]) * ap[e];
+      bv[k][e] = sigm(bg[e]) * bp[e];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    ta[warp * 8 + e][lane] = pack2(av[0][e], av[1][e]);
+    tb[warp * 8 + e][lane] = pack2(bv[0][e], bv[1][e]);
+  }
+  __syncthreads();
+  for (int it = threadIdx.x; it < 2 * kT * 8; it += 256) {
+    const int tns = it / (kT * 8), chl = (it / 8) % kT, k = it % 8;
+    const uint4 v = *reinterpret_cast<const uint4 *>(&(tns ? tb : ta)[chl][4 * k]);
+    *reinterpret_cast<uint4 *>((tns ? b_cm : a_cm) + (int64_t)(ch0 + chl) * R + p0 + 8 * k) = v;
+  }
+}
+
+__global__ void __launch_bounds__(256) gate_in_bwd_tiled(const __nv_bfloat16 *__restrict__ da_cm,
+                                                         const __nv_bfloat16 *__restrict__ db_cm,
+                                                         const __nv_bfloat16 *__restrict__ pg,
+                                                         int64_t R, int c, int64_t ldpg,
+                                                         __nv_bfloat16 *__restrict__ dpg) {
+  __shared__ __align__(16) uint32_t ta[kT][kT / 2], tb[kT][kT / 2];
+  const int64_t p0 = (int64_t)blockIdx.x * kT;
+  const int ch0 = blockIdx.y * kT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int it = threadIdx.x; it < 2 * kT * 8; it += 256) {
+    const int tns = it / (kT * 8), chl = (it / 8) % kT, k = it % 8;
+    const uint4 v = *reinterpret_cast<const uint4 *>((tns ? db_cm : da_cm) +
+                                                     (int64_t)(ch0 + chl) * R + p0 + 8 * k);
+    *reinterpret_cast<uint4 *>(&(tns ? tb : ta)[chl][4 * k]) = v;
+  }
+  __syncthreads();
+  const int cg = ch0 + warp * 8;
+  uint32_t dw[8], ew[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    dw[e] = ta[warp * 8 + e][lane];
+    ew[e] = tb[warp * 8 + e][lane];
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int64_t off = (p0 + 2 * lane + k) * ldpg + cg;
+    float ap[8], ag[8], bp[8], bg[8];
+    unpack8(*reinterpret_cast<const uint4 *>(pg + off), ap);
+    unpack8(*reinterpret_cast<const uint4 *>(pg + off + c), ag);
+    unpack8(*reinterpret_cast<const uint4 *>(pg + off + 2 * c), bp);
+    unpack8(*reinterpret_cast<const uint4 *>(pg + off + 3 * c), bg);
+    uint32_t o0[4], o1[4], o2[4], o3[4];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      float r0[2], r1[2], r2[2], r3[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float da = k ? hi_of(dw[e + u]) : lo_of(dw[e + u]);
+        const float db = k ? hi_of(ew[e + u]) : lo_of(ew[e + u]);
+        const float sa = sigm(ag[e + u]), sb = sigm(bg[e + u]);
+        r0[u] = da * sa;
+        r1[u] = da * ap[e + u] * sa * (1.0f - sa);
+        r2[u] = db * sb;
+        r3[u] = db * bp[e + u] * sb * (1.0f - sb);
+      }
+      o0[e / 2] = pack2(r0[0], r0[1]);
+      o1[e / 2] = pack2(r1[0], r1[1]);
+      o2[e / 2] = pack2(r2[0], r2[1]);
+      o3[e / 2] = pack2(r3[0], r3[1]);
+    }
+    *reinterpret_cast<uint4 *>(dpg + off) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    *reinterpret_cast<uint4 *>(dpg + off + c) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    *reinterpret_cast<uint4 *>(dpg + off + 2 * c) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+    *reinterpret_cast<uint4 *>(dpg + off + 3 * c) = make_uint4(o3[0], o3[1], o3[2], o3[3]);
+  }
+}
+
+// out [cols][rows] = in [rows][cols]^T, both sides multiples of 64; the bits
+// move unchanged (two rows' values of one column per shared-memory word).
+__global__ void __launch_bounds__(256) transpose_tiled(const __nv_bfloat16 *__restrict__ in,
+                                                       int64_t rows, int64_t cols,
+                                                       __nv_bfloat16 *__restrict__ out) {
+  __shared__ __align__(16) uint32_t t[kT][kT / 2];
+  const int64_t col_tiles = cols / kT;
+  const int64_t r0 = ((int64_t)blockIdx.x / col_tiles) * kT;
+  const int64_t c0 = ((int64_t)blockIdx.x % col_tiles) * kT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const __nv_bfloat16 *src = in + (r0 + 2 * lane) * cols + c0 + 8 * warp;
+  const uint4 va = *reinterpret_cast<const uint4 *>(src);
+  const uint4 vb = *reinterpret_cast<const uint4 *>(src + cols);
+  const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    t[warp * 8 + e][lane] = __byte_perm(wa[e / 2], wb[e / 2], (e & 1) ? 0x7632 : 0x5410);
+  __syncthreads();
+  for (int it = threadIdx.x; it < kT * 8; it += 256) {
+    const int chl = it / 8, k = it % 8;
+    *reinterpret_cast<uint4 *>(out + (c0 + chl) * rows + r0 + 8 * k) =
+        *reinterpret_cast<const uint4 *>(&t[chl][4 * k]);
+  }
+}
+
+bool tiled_shape(int64_t a, int64_t b) { return a % kT == 0 && b % kT == 0; }
+
 int blocks_for(int64_t n) {
   int64_t b = (n + 255) / 256;
   if (b > 148 * 16) b = 148 * 16;
@@ -187,6 +336,11 @@ int blocks_for(int64_t n) {
 cudaError_t launch_gate_in_fwd(const __nv_bfloat16 *pg, int64_t R, int c, int64_t ldpg,
                                __nv_bfloat16 *a_cm, __nv_bfloat16 *b_cm, cudaStream_t stream) {
   if (R == 0) return cudaSuccess;
+  if (tiled_shape(R, c) && ldpg % 8 == 0 && R / kT <= 0x7fffffffLL) {
+    gate_in_fwd_tiled<<<dim3((unsigned)(R / kT), c / kT), 256, 0, stream>>>(pg, R, c, ldpg, a_cm,
+                                                                            b_cm);
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)((R + kTile - 1) / kTile), c / kTile);
   gate_in_fwd_kernel<<<grid, dim3(kTile, 8), 0, stream>>>(pg, R, c, ldpg, a_cm, b_cm);
   return cudaGetLastError();
@@ -196,6 +350,11 @@ cudaError_t launch_gate_in_bwd(const __nv_bfloat16 *da_cm, const __nv_bfloat16 *
                                const __nv_bfloat16 *pg, int64_t R, int c, int64_t ldpg,
                                __nv_bfloat16 *dpg, cudaStream_t stream) {
   if (R == 0) return cudaSuccess;
+  if (tiled_shape(R, c) && ldpg % 8 == 0 && R / kT <= 0x7fffffffLL) {
+    gate_in_bwd_tiled<<<dim3((unsigned)(R / kT), c / kT), 256, 0, stream>>>(da_cm, db_cm, pg, R,
+                                                                            c, ldpg, dpg);
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)((R + kTile - 1) / kTile), c / kTile);
   gate_in_bwd_kernel<<<grid, dim3(kTile, 8), 0, stream>>>(da_cm, db_cm, pg, R, c, ldpg, dpg);
   return cudaGetLastError();
@@ -204,6 +363,11 @@ cudaError_t launch_gate_in_bwd(const __nv_bfloat16 *da_cm, const __nv_bfloat16 *
 cudaError_t launch_transpose(const __nv_bfloat16 *in, int64_t rows, int64_t cols,
                              __nv_bfloat16 *out, cudaStream_t stream) {
   if (rows == 0 || cols == 0) return cudaSuccess;
+  if (tiled_shape(rows, cols) && (rows / kT) * (cols / kT) <= 0x7fffffffLL) {
+    transpose_tiled<<<(unsigned)((rows / kT) * (cols / kT)), 256, 0, stream>>>(in, rows, cols,
+                                                                               out);
+    return cudaGetLastError();
+  }
   const int64_t tiles = ((cols + kTile - 1) / kTile) * ((rows + kTile - 1) / kTile);
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   transpose_kernel<<<(unsigned)tiles, dim3(kTile, 8), 0, stream>>>(in, rows, cols, out);
