@@ -178,29 +178,54 @@ __global__ void colsum_strided_kernel(const __nv_bfloat16 *__restrict__ m, int64
 
 // ------------------------------------------------ 64 x 64 tiled versions --
 // For shapes whose both sides are multiples of 64 (every shape of the update:
-// c is a multiple of 64 and R = N*N with N % 8 == 0). A tile moves through
-// shared memory as [64 channels][32 position pairs] words, each word the bf16
-// values of two consecutive positions: warp w reads (or writes) channels
-// 8w .. 8w+7 of 64 positions with one 16-byte access per position, and the
-// channel-major side moves 16 bytes (8 positions) per access, eight lanes
-// covering 128 contiguous bytes. Both shared-memory passes are free of bank
-// conflicts. Arithmetic and rounding are those of the kernels above.
+// c is a multiple of 64 and R = N*N with N % 8 == 0). A tile of 64 positions x
+// 64 channels passes through shared memory as [channel][position] bf16. On the
+// position-major side a thread takes 16 channels (32 contiguous bytes, a whole
+// sector) of one position per tensor; on the channel-major side 16 bytes (8
+// positions), eight lanes covering 128 contiguous bytes. Both shared-memory
+// passes are free of bank conflicts. Arithmetic and rounding are those of the
+// kernels above.
 constexpr int kT = 64;
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
 }
-__device__ __forceinline__ float lo_of(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float hi_of(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint16_t bits_of(float v) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  return *reinterpret_cast<const uint16_t *>(&b);
+}
+__device__ __forceinline__ float from_bits(uint16_t v) {
+  return __uint_as_float((uint32_t)v << 16);
+}
 
-// 8 bf16 of a uint4 as floats
+// 16 bf16 (32 bytes at p) as floats
+__device__ __forceinline__ void load16(const __nv_bfloat16 *p, float (&o)[16]) {
+  const uint4 v0 = *reinterpret_cast<const uint4 *>(p);
+  const uint4 v1 = *reinterpret_cast<const uint4 *>(p + 8);
+  const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    o[2 * e] = __uint_as_float(w[e] << 16);
+    o[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+  }
+}
+// 16 floats rounded to bf16 into 32 bytes at p (one 32-byte store)
+__device__ __forceinline__ void store16(__nv_bfloat16 *p, const float (&v)[16]) {
+  uint32_t w[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) w[e] = pack2(v[2 * e], v[2 * e + 1]);
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+// 8 bf16 (16 bytes) of a shared-memory row as a uint4
 __device__ __forceinline__ void unpack8(const uint4 v, float (&o)[8]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    o[2 * e] = lo_of(w[e]);
-    o[2 * e + 1] = hi_of(w[e]);
+    o[2 * e] = __uint_as_float(w[e] << 16);
+    o[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
   }
 }
 
@@ -208,35 +233,29 @@ __global__ void __launch_bounds__(256) gate_in_fwd_tiled(const __nv_bfloat16 *__
                                                          int64_t R, int c, int64_t ldpg,
                                                          __nv_bfloat16 *__restrict__ a_cm,
                                                          __nv_bfloat16 *__restrict__ b_cm) {
-  __shared__ __align__(16) uint32_t ta[kT][kT / 2], tb[kT][kT / 2];
+  __shared__ __align__(16) uint16_t ta[kT][kT], tb[kT][kT];
   const int64_t p0 = (int64_t)blockIdx.x * kT;
   const int ch0 = blockIdx.y * kT;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cg = ch0 + warp * 8;
-  float av[2][8], bv[2][8];
+  const int pl = threadIdx.x & (kT - 1), g = threadIdx.x / kT;   // position, 16-channel group
+  const __nv_bfloat16 *row = pg + (p0 + pl) * ldpg + ch0 + 16 * g;
+  {
+    float ap[16], ag[16];
+    load16(row, ap);
+    load16(row + c, ag);
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const __nv_bfloat16 *row = pg + (p0 + 2 * lane + k) * ldpg + cg;
-    float ap[8], ag[8], bp[8], bg[8];
-    unpack8(*reinterpret_cast<const uint4 *>(row), ap);
-    unpack8(*reinterpret_cast<const uint4 *>(row + c), ag);
-    unpack8(*reinterpret_cast<const uint4 *>(row + 2 * c), bp);
-    unpack8(*reinterpret_cast<const uint4 *>(row + 3 * c), bg);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      av[k][e] = sigm(ag[e]) * ap[e];
-      bv[k][e] = sigm(bg[e]) * bp[e];
-    }
+    for (int e = 0; e < 16; ++e) ta[16 * g + e][pl] = bits_of(sigm(ag[e]) * ap[e]);
   }
+  {
+    float bp[16], bg[16];
+    load16(row + 2 * c, bp);
+    load16(row + 3 * c, bg);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    ta[warp * 8 + e][lane] = pack2(av[0][e], av[1][e]);
-    tb[warp * 8 + e][lane] = pack2(bv[0][e], bv[1][e]);
+    for (int e = 0; e < 16; ++e) tb[16 * g + e][pl] = bits_of(sigm(bg[e]) * bp[e]);
   }
   __syncthreads();
   for (int it = threadIdx.x; it < 2 * kT * 8; it += 256) {
     const int tns = it / (kT * 8), chl = (it / 8) % kT, k = it % 8;
-    const uint4 v = *reinterpret_cast<const uint4 *>(&(tns ? tb : ta)[chl][4 * k]);
+    const uint4 v = *reinterpret_cast<const uint4 *>(&(tns ? tb : ta)[chl][8 * k]);
     *reinterpret_cast<uint4 *>((tns ? b_cm : a_cm) + (int64_t)(ch0 + chl) * R + p0 + 8 * k) = v;
   }
 }
@@ -246,55 +265,45 @@ __global__ void __launch_bounds__(256) gate_in_bwd_tiled(const __nv_bfloat16 *__
                                                          const __nv_bfloat16 *__restrict__ pg,
                                                          int64_t R, int c, int64_t ldpg,
                                                          __nv_bfloat16 *__restrict__ dpg) {
-  __shared__ __align__(16) uint32_t ta[kT][kT / 2], tb[kT][kT / 2];
+  __shared__ __align__(16) uint16_t ta[kT][kT], tb[kT][kT];
   const int64_t p0 = (int64_t)blockIdx.x * kT;
   const int ch0 = blockIdx.y * kT;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int it = threadIdx.x; it < 2 * kT * 8; it += 256) {
     const int tns = it / (kT * 8), chl = (it / 8) % kT, k = it % 8;
     const uint4 v = *reinterpret_cast<const uint4 *>((tns ? db_cm : da_cm) +
                                                      (int64_t)(ch0 + chl) * R + p0 + 8 * k);
-    *reinterpret_cast<uint4 *>(&(tns ? tb : ta)[chl][4 * k]) = v;
+    *reinterpret_cast<uint4 *>(&(tns ? tb : ta)[chl][8 * k]) = v;
   }
   __syncthreads();
-  const int cg = ch0 + warp * 8;
-  uint32_t dw[8], ew[8];
+  const int pl = threadIdx.x & (kT - 1), g = threadIdx.x / kT;
+  const int64_t off = (p0 + pl) * ldpg + ch0 + 16 * g;
+  {
+    float ap[16], ag[16], r0[16], r1[16];
+    load16(pg + off, ap);
+    load16(pg + off + c, ag);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    dw[e] = ta[warp * 8 + e][lane];
-    ew[e] = tb[warp * 8 + e][lane];
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int64_t off = (p0 + 2 * lane + k) * ldpg + cg;
-    float ap[8], ag[8], bp[8], bg[8];
-    unpack8(*reinterpret_cast<const uint4 *>(pg + off), ap);
-    unpack8(*reinterpret_cast<const uint4 *>(pg + off + c), ag);
-    unpack8(*reinterpret_cast<const uint4 *>(pg + off + 2 * c), bp);
-    unpack8(*reinterpret_cast<const uint4 *>(pg + off + 3 * c), bg);
-    uint32_t o0[4], o1[4], o2[4], o3[4];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      float r0[2], r1[2], r2[2], r3[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const float da = k ? hi_of(dw[e + u]) : lo_of(dw[e + u]);
-        const float db = k ? hi_of(ew[e + u]) : lo_of(ew[e + u]);
-        const float sa = sigm(ag[e + u]), sb = sigm(bg[e + u]);
-        r0[u] = da * sa;
-        r1[u] = da * ap[e + u] * sa * (1.0f - sa);
-        r2[u] = db * sb;
-        r3[u] = db * bp[e + u] * sb * (1.0f - sb);
-      }
-      o0[e / 2] = pack2(r0[0], r0[1]);
-      o1[e / 2] = pack2(r1[0], r1[1]);
-      o2[e / 2] = pack2(r2[0], r2[1]);
-      o3[e / 2] = pack2(r3[0], r3[1]);
+    for (int e = 0; e < 16; ++e) {
+      const float da = from_bits(ta[16 * g + e][pl]);
+      const float sa = sigm(ag[e]);
+      r0[e] = da * sa;
+      r1[e] = da * ap[e] * sa * (1.0f - sa);
     }
-    *reinterpret_cast<uint4 *>(dpg + off) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-    *reinterpret_cast<uint4 *>(dpg + off + c) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
-    *reinterpret_cast<uint4 *>(dpg + off + 2 * c) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
-    *reinterpret_cast<uint4 *>(dpg + off + 3 * c) = make_uint4(o3[0], o3[1], o3[2], o3[3]);
+    store16(dpg + off, r0);
+    store16(dpg + off + c, r1);
+  }
+  {
+    float bp[16], bg[16], r2[16], r3[16];
+    load16(pg + off + 2 * c, bp);
+    load16(pg + off + 3 * c, bg);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float db = from_bits(tb[16 * g + e][pl]);
+      const float sb = sigm(bg[e]);
+      r2[e] = db * sb;
+      r3[e] = db * bp[e] * sb * (1.0f - sb);
+    }
+    store16(dpg + off + 2 * c, r2);
+    store16(dpg + off + 3 * c, r3);
   }
 }
 
@@ -325,6 +334,44 @@ __global__ void __launch_bounds__(256) transpose_tiled(const __nv_bfloat16 *__re
 
 bool tiled_shape(int64_t a, int64_t b) { return a % kT == 0 && b % kT == 0; }
 
+// colsum_strided_kernel with 8 columns per thread and 16 rows of 16-byte loads in
+// flight; each column is still summed over the block's rows in row order, so
+// the partial sums are bit-identical to the one-column-per-thread form.
+__global__ void colsum_strided_vec(const __nv_bfloat16 *__restrict__ m, int64_t rows, int64_t ld,
+                                   int cols, float *__restrict__ part) {
+  const int64_t span = (rows + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = (int64_t)blockIdx.x * span;
+  const int64_t r1 = r0 + span < rows ? r0 + span : rows;
+  const int col = threadIdx.x * 8;
+  if (col >= cols) return;
+  float s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s[e] = 0.0f;
+  constexpr int kAhead = 16;
+  int64_t r = r0;
+  for (; r + kAhead <= r1; r += kAhead) {
+    uint4 v[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u)
+      v[u] = *reinterpret_cast<const uint4 *>(m + (r + u) * ld + col);
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+      float x[8];
+      unpack8(v[u], x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[e] += x[e];
+    }
+  }
+  for (; r < r1; ++r) {
+    float x[8];
+    unpack8(*reinterpret_cast<const uint4 *>(m + r * ld + col), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s[e] += x[e];
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[(int64_t)blockIdx.x * cols + col + e] = s[e];
+}
+
 int blocks_for(int64_t n) {
   int64_t b = (n + 255) / 256;
   if (b > 148 * 16) b = 148 * 16;
@@ -350,7 +397,8 @@ cudaError_t launch_gate_in_bwd(const __nv_bfloat16 *da_cm, const __nv_bfloat16 *
                                const __nv_bfloat16 *pg, int64_t R, int c, int64_t ldpg,
                                __nv_bfloat16 *dpg, cudaStream_t stream) {
   if (R == 0) return cudaSuccess;
-  if (tiled_shape(R, c) && ldpg % 8 == 0 && R / kT <= 0x7fffffffLL) {
+  if (tiled_shape(R, c) && ldpg % 16 == 0 && (reinterpret_cast<uintptr_t>(dpg) & 31) == 0 &&
+      R / kT <= 0x7fffffffLL) {
     gate_in_bwd_tiled<<<dim3((unsigned)(R / kT), c / kT), 256, 0, stream>>>(da_cm, db_cm, pg, R,
                                                                             c, ldpg, dpg);
     return cudaGetLastError();
@@ -393,6 +441,11 @@ cudaError_t launch_out_bwd(const __nv_bfloat16 *dy, const __nv_bfloat16 *pg, int
 
 cudaError_t launch_colsum_strided(const __nv_bfloat16 *m, int64_t rows, int64_t ld, int cols,
                                   float *part, cudaStream_t stream) {
+  if (cols % 8 == 0 && ld % 8 == 0 && cols <= 8 * 1024) {
+    const int threads = ((cols / 8 + 31) / 32) * 32;
+    colsum_strided_vec<<<kProjBlocks, threads, 0, stream>>>(m, rows, ld, cols, part);
+    return cudaGetLastError();
+  }
   colsum_strided_kernel<<<kProjBlocks, 256, 0, stream>>>(m, rows, ld, cols, part);
   return cudaGetLastError();
 }
