@@ -794,6 +794,44 @@ PROJ_METRIC = ("LayerNorm + projection stages fwd+bwd GB/s (algorithmic HBM byte
                "cz=128, H=4, c=32 bf16")
 
 
+def run_mma_rate(args, rank, world, local):
+    """Cycles per tcgen05.mma instruction (M=128, K=16, bf16, fp32 accumulator) by N
+    and operand form, one CTA per SM issuing back to back, and the tensor-pipe floor
+    they set for the attention step at N=768, H=4, c=32 (every instruction of the
+    forward and backward main kernels issued back to back, nothing else)."""
+    import triangle_attention_b200 as ta
+    torch.cuda.set_device(local)
+    ta.probe_mma(128, 0, instructions=1024)                 # warm-up
+    forms = [(32, 0, "K-major A and B (S = Q K^T form)"), (64, 0, "K-major A and B"),
+             (128, 0, "K-major A and B"), (256, 0, "K-major A and B"),
+             (32, 1, "MN-major A and B (dV = P^T dU, dK = dS^T Q form)"),
+             (32, 2, "A from tensor memory (O += P V form)")]
+    rows, cyc = [], {}
+    for n, layout, form in forms:
+        c = ta.probe_mma(n, layout, instructions=16384)
+        cyc[(n, layout)] = c
+        rows.append({"n": n, "layout": layout, "form": form, "cycles_per_instruction": c,
+                     "mac_per_cycle_per_sm": 128 * n * 16 / c,
+                     "frac_of_dense": 128 * n * 16 / c / 4096})
+    N, H = 768, 4
+    nb = N // 128
+    # backward, per 128 x 128 block and attention row: S and dP (2 + 2 at N = 128),
+    # dV, dK, dQ (8 each at N = 32, K = 128 in steps of 16)
+    bwd_block = 4 * cyc[(128, 0)] + 24 * cyc[(32, 1)]
+    # forward, per 64-key step of 128 queries: S (2 at N = 64), O += P V (4 at N = 32)
+    fwd_step = 2 * cyc[(64, 0)] + 4 * cyc[(32, 2)]
+    bwd_units, fwd_units = nb * nb * N * H, nb * (N // 64) * N * H
+    ghz = 1.965
+    floor = {"backward_cycles_per_block_row": bwd_block, "forward_cycles_per_step": fwd_step,
+             "backward_ms": bwd_units / SMS * bwd_block / ghz / 1e6,
+             "forward_ms": fwd_units / SMS * fwd_step / ghz / 1e6}
+    floor["step_ms"] = floor["backward_ms"] + floor["forward_ms"]
+    return {"metric": "tcgen05.mma cycles per instruction (M=128, K=16, bf16, fp32 accumulate)",
+            "unit": "cycles", "n_gpus": 1, "rows": rows,
+            "tensor_floor_n768_h4_c32_at_1965mhz": floor,
+            "config": {"workload": "mma_issue_rate", "ctas": SMS, "instructions": 16384}}
+
+
 def run_proj(args, rank, world, local):
     """One step: the four projection calls around the attention (input side
     forward and backward, output side forward and backward) at N=768, cz=128,
@@ -876,7 +914,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["attention", "trimul", "trimul_update", "block", "proj"],
+    ap.add_argument("--op", choices=["attention", "trimul", "trimul_update", "block", "proj",
+                                     "mma_rate"],
                     default="attention",
                     help="attention (the default line), the triangle multiplication "
                          "contraction, the full triangle multiplicative update, the whole "
@@ -908,6 +947,8 @@ def main():
             line = run_block(args, rank, world, local)
         elif args.op == "proj":
             line = run_proj(args, rank, world, local)
+        elif args.op == "mma_rate":
+            line = run_mma_rate(args, rank, world, local)
         else:
             line = run_ours(args, rank, world, local, w)
         if rank == 0:

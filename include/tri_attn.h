@@ -383,6 +383,27 @@ tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_by
 tri_attn_status tri_attn_check_exp2(const float *x, float *y_fma, float *y_mufu, int64_t n,
                                     tri_attn_stream_t stream);
 
+/*
+ * Diagnostic of the tensor-core instruction the kernels are built from (no
+ * counterpart on the pages): tcgen05.mma kind::f16, bf16 operands, fp32
+ * accumulator in tensor memory, M = 128 and K = 16 per instruction, N = n in
+ * {32, 64, 128, 256}. Each of `ctas` CTAs (1 .. 1024; one per SM when ctas is
+ * the SM count) issues `instructions` (1 .. 2^24, rounded up to a multiple of 8)
+ * instructions back to back
+ * into one accumulator and writes the SM clock cycles from the first issue to
+ * their completion to cycles[cta] (device, caller-owned, `ctas` entries).
+ * layout 0: both operands K-major with the 64-byte swizzle (the S = Q K^T form);
+ * layout 1: both MN-major (the dV = P^T dU form); layout 2: A read from tensor
+ * memory, B MN-major (the O += P V form); layouts 1 and 2 take n = 32. The
+ * shared-memory operands are zeros; the tensor-memory one is whatever the
+ * columns hold (the timing does not depend on the values). *status (device int32) is set to 0, or to
+ * TRI_ATTN_ERR_TIMEOUT if the completion did not come within the bounded wait.
+ * TRI_ATTN_ERR_INVALID_ARG for other n, layout or counts, or NULL pointers.
+ */
+tri_attn_status tri_attn_probe_mma(int32_t n, int32_t layout, int32_t ctas, int32_t instructions,
+                                   unsigned long long *cycles, int32_t *status,
+                                   tri_attn_stream_t stream);
+
 /* ------------------------------------------------ triangle multiplication --
  *
  * The contraction at the core of the triangle multiplicative update, the other

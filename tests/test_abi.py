@@ -235,6 +235,14 @@ def test_problem_of_batched_tensors():
         ta.problem(torch.empty((3, 16, 15, 2, 32)), None, ta.STARTING)
 
 
+def test_probe_mma_rejects_bad_arguments(lib):
+    fake = ctypes.c_void_p(4096)
+    for args in [(48, 0, 1, 1), (32, 3, 1, 1), (64, 1, 1, 1), (64, 2, 1, 1), (32, 0, 0, 1), (32, 0, 1, 0),
+                 (32, 0, 2000, 1)]:
+        assert lib.tri_attn_probe_mma(*args, fake, fake, None) == 1, args
+    assert lib.tri_attn_probe_mma(32, 0, 1, 1, None, fake, None) == 1
+
+
 def test_read_status_rejects_null(lib):
     v = ctypes.c_int32(0)
     assert lib.tri_attn_read_status(None, ctypes.byref(v), None) == 1

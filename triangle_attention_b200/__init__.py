@@ -148,6 +148,7 @@ def lib():
         L.tri_attn_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.tri_attn_get_status.argtypes = [P, P]
         L.tri_attn_check_exp2.argtypes = [P, P, P, ctypes.c_int64, P]
+        L.tri_attn_probe_mma.argtypes = [ctypes.c_int32] * 4 + [P, P, P]
         i64 = ctypes.c_int64
         L.tri_attn_fwd_rows.argtypes = [PP, i64, i64, P, P, P, P, P, P, P, P, P, sz, P]
         L.tri_attn_bwd_rows.argtypes = [PP, i64, i64] + [P] * 15 + [sz, P]
@@ -173,7 +174,7 @@ def lib():
                   L.tri_attn_bwd, L.tri_attn_fwd_ex, L.tri_attn_bwd_ex,
                   L.tri_attn_kernel_launches, L.tri_attn_read_status, L.tri_attn_get_status,
                   L.tri_attn_fwd_rows, L.tri_attn_bwd_rows, L.tri_attn_dbias_reduce,
-                  L.tri_attn_check_exp2,
+                  L.tri_attn_check_exp2, L.tri_attn_probe_mma,
                   L.tri_attn_check_wait_timeout, L.tri_mul_workspace_size, L.tri_mul_fwd,
                   L.tri_mul_bwd, L.tri_mul_update_sizes, L.tri_mul_update_fwd,
                   L.tri_mul_update_bwd, L.tri_proj_workspace_size, L.tri_proj_in_fwd,
@@ -419,6 +420,21 @@ def get_status(ws: torch.Tensor, stream=None) -> int:
     if code == 4:
         _check(code, "tri_attn_get_status")
     return code
+
+
+def probe_mma(n: int, layout: int = 0, instructions: int = 16384, ctas: int = 148,
+              device="cuda") -> float:
+    """Mean SM cycles per tcgen05.mma (M=128, K=16, N=n) issued back to back,
+    over `ctas` CTAs; raises if a completion wait ran out."""
+    cycles = torch.zeros(ctas, dtype=torch.int64, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib().tri_attn_probe_mma(n, layout, ctas, instructions, _p(cycles), _p(status),
+                                    _stream()), "tri_attn_probe_mma")
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise TriAttnError(int(status.item()), "tri_attn_probe_mma")
+    issued = (instructions + 7) // 8 * 8
+    return float(cycles.double().mean().item()) / issued
 
 
 def check_exp2(x: torch.Tensor, stream=None) -> tuple:

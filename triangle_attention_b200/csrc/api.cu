@@ -944,6 +944,17 @@ tri_attn_status tri_attn_check_exp2(const float *x, float *y_fma, float *y_mufu,
       tri::launch_exp2_eval(x, y_fma, y_mufu, n, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+tri_attn_status tri_attn_probe_mma(int32_t n, int32_t layout, int32_t ctas, int32_t instructions,
+                                   unsigned long long *cycles, int32_t *status,
+                                   tri_attn_stream_t stream) {
+  const bool n_ok = n == 32 || n == 64 || n == 128 || n == 256;
+  if (!n_ok || layout < 0 || layout > 2 || (layout != 0 && n != 32) || ctas < 1 ||
+      ctas > 1024 || instructions < 1 || instructions > (1 << 24) || !cycles || !status)
+    return TRI_ATTN_ERR_INVALID_ARG;
+  return cuda_status(tri::launch_mma_probe(n, layout, ctas, instructions, cycles, status,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 tri_attn_status tri_attn_check_wait_timeout(void *workspace, size_t workspace_bytes,
                                             tri_attn_stream_t stream) {
   if (!workspace || !aligned16(workspace) || workspace_bytes < 256)

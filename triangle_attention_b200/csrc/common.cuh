@@ -38,6 +38,9 @@ __device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
 
 // Diagnostic kernel: a bounded wait that nothing satisfies (see selftest.cu).
 cudaError_t launch_unsatisfied_wait(int32_t *status, cudaStream_t stream);
+// Diagnostic kernel: tensor-core issue rate by instruction shape (see selftest.cu).
+cudaError_t launch_mma_probe(int n, int layout, int ctas, int instructions,
+                             unsigned long long *cycles, int32_t *status, cudaStream_t stream);
 // Diagnostic kernel: both device exp2 evaluations of x[0..n) (see selftest.cu).
 cudaError_t launch_exp2_eval(const float *x, float *y_fma, float *y_mufu, int64_t n,
                              cudaStream_t stream);
