@@ -80,11 +80,14 @@ __global__ void bwd_pre_bf16_kernel(Frame f, const __nv_bfloat16 *__restrict__ g
   for (int64_t w = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w < total;
        w += (int64_t)gridDim.x * blockDim.x) {
     const int q = (int)(w & 3);                                // channels 8q .. 8q+7
-    const int64_t e = w >> 2;                                  // (a, b, h)
-    const int h = (int)(e % f.H);
-    const int64_t b = (e / f.H) % f.N;
+    const int64_t e = w >> 2;                                  // (p, a, b, h)
+    // one 64-bit division for the storage row p*N + a; the rest in 32 bits
     const int64_t pa = e / ((int64_t)f.H * f.N);              // p*N + a
-    const int64_t aa = pa % f.N;
+    const uint32_t rem = (uint32_t)(e - pa * ((int64_t)f.H * f.N));   // b*H + h
+    const int h = (int)(rem % (uint32_t)f.H);
+    const int64_t b = rem / (uint32_t)f.H;
+    const uint32_t pp = (uint32_t)pa / (uint32_t)f.N;          // B*N <= 2^16
+    const int64_t aa = (uint32_t)pa - pp * (uint32_t)f.N;
     const int64_t r = pa - aa + (ending ? b : aa);             // row of the batch
     const int64_t x = ending ? aa : b;
     if (r < f.row0 || r >= f.row_end) continue;      // another call's row shard
@@ -176,12 +179,15 @@ __global__ void partial_reduce_bf16_kernel(Frame f, const __nv_bfloat16 *__restr
       }
     }
     // gidx -> (r, h, half, i, c8) of the [r][H][2][N][16] layout
+    // one 64-bit division for the row; the rest (below N*2*H <= 2^29) in 32 bits
     const int c8 = (int)(gidx & 1);
-    const int64_t i = (gidx >> 1) % f.N;
-    const int half = (int)((gidx >> 1) / f.N % 2);
-    const int h = (int)((gidx >> 1) / ((int64_t)f.N * 2) % f.H);
-    const int64_t r = (gidx >> 1) / ((int64_t)f.N * 2 * f.H);
-    const int64_t p = r / f.N;                                     // problem of row r
+    const int64_t row_pieces = (int64_t)f.N * 2 * f.H;
+    const int64_t r = (gidx >> 1) / row_pieces;
+    const uint32_t rem = (uint32_t)((gidx >> 1) - r * row_pieces);
+    const int64_t i = rem % (uint32_t)f.N;
+    const int half = (int)((rem / (uint32_t)f.N) & 1u);
+    const int h = (int)(rem / (2u * (uint32_t)f.N));
+    const int64_t p = (uint32_t)r / (uint32_t)f.N;                // problem of row r
     __nv_bfloat16 *dst = (which == 0 ? dq : which == 1 ? dk : dv) + p * pair +
                          (r - p * f.N) * f.sR + i * f.sX + (int64_t)h * 32 + half * 16 + c8 * 8;
     *reinterpret_cast<uint4 *>(dst) =
