@@ -384,12 +384,14 @@ def run_ours(args, rank, world, local, w):
     bwd_med = statistics.median(e[2].elapsed_time(e[3]) for e in ev)
     # Each call resets its status word, so a bounded wait that ran out in an
     # earlier step of the timed region leaves no status behind; it does leave a
-    # launch that ran for the wait's whole limit (seconds against milliseconds).
-    for name, col, med in (("forward", 0, fwd_med), ("backward", 2, bwd_med)):
-        worst = max(e[col].elapsed_time(e[col + 1]) for e in ev)
-        if worst > 20 * med:
-            raise RuntimeError(f"a {name} launch in the timed region took {worst:.1f} ms "
-                               f"against a median of {med:.3f} ms: a bounded wait ran out")
+    # launch that ran for the wait's whole limit (2 s). Under a profiler (which
+    # injects itself into the process) a captured launch is slow by design.
+    if "CUDA_INJECTION64_PATH" not in os.environ:
+        for name, col, med in (("forward", 0, fwd_med), ("backward", 2, bwd_med)):
+            worst = max(e[col].elapsed_time(e[col + 1]) for e in ev)
+            if worst > 1900.0:
+                raise RuntimeError(f"a {name} launch in the timed region took {worst:.1f} ms "
+                                   f"against a median of {med:.3f} ms: a bounded wait ran out")
 
     # roofline of the dominant kernel: algorithmic FLOPs per launch / launch time
     peaks = load_peaks()
