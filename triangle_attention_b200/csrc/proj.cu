@@ -517,6 +517,8 @@ cudaError_t launch_ln_fwd_h(const ProjArgs &a, cudaStream_t stream) {
 
 cudaError_t launch_ln_fwd(const ProjArgs &a, cudaStream_t stream) {
   if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
+  // one head (the multiplicative update's LayerNorms) skips three heads' dot products
+  if (a.H == 1) return launch_ln_fwd_h<1>(a, stream);
   return a.H <= 4 ? launch_ln_fwd_h<4>(a, stream) : launch_ln_fwd_h<kMaxHeads>(a, stream);
 }
 
@@ -544,6 +546,7 @@ cudaError_t launch_ln_bwd_h(const ProjArgs &a, cudaStream_t stream) {
 
 cudaError_t launch_ln_bwd(const ProjArgs &a, cudaStream_t stream) {
   if (a.H < 1 || a.H > kMaxHeads) return cudaErrorInvalidValue;
+  if (a.H == 1) return launch_ln_bwd_h<1>(a, stream);
   return a.H <= 4 ? launch_ln_bwd_h<4>(a, stream) : launch_ln_bwd_h<kMaxHeads>(a, stream);
 }
 
