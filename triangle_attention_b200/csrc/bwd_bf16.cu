@@ -59,11 +59,15 @@ constexpr int kEltThreads = kEltGroups * 128;
 constexpr bool kPackOnIntegerPipes = false;
 // elementwise arithmetic on fp32 pairs (fma.rn.f32x2 and friends) or scalars
 constexpr bool kPairArithmetic = true;
-// chunk (of kKeys / 8) at which warpgroup wg drains the previous row's
-// gradients: two warpgroups at a time (one with two pieces, one with one), the
-// later pair early enough to leave time for the next S/dP products
-__device__ constexpr int kDrainChunk[4] = {2, 3, 2, 3};
-static_assert(kEltGroups == 4, "drain schedule written for four warpgroups");
+// chunk (of kKeys / 8) before which the elementwise warps drain the previous
+// row's gradients: the last one. The gradient products of row t-1 start only
+// when row t-1's P/dS are complete, so an earlier drain waits for them; a drain
+// after the last chunk holds back the next S/dP products. Measured at N=768:
+// last chunk 1.59 ms, staggered over chunks 2 and 3 1.74, after the row 1.70.
+// (Read per warpgroup from a table: as a compile-time constant the drain is
+// inlined into the unrolled chunk loop and the kernel spills.)
+__device__ constexpr int kDrainChunk[4] = {3, 3, 3, 3};
+static_assert(kEltGroups == 4 && kKeys / 8 == 4, "drain table written for four warpgroups");
 // the producer asks L2 for the input tiles of row it + kL2Ahead while it loads
 // row it (0: no prefetch)
 constexpr int kL2Ahead = 4;
@@ -412,8 +416,6 @@ bwd_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // 16-byte chunk chunk0 + ch of the swizzled row is at (cswz ^ ch) (chunk0 is a
     // multiple of kKeys / 8, so adding ch never carries into its bits)
     const uint32_t cswz = (uint32_t)(chunk0 ^ (row & 7));
-    // Each warpgroup drains the previous row's gradients at its own 8-key chunk,
-    // so the stores of the four warpgroups do not all leave the SM at once.
     const int drain_chunk = kDrainChunk[wg];
     static_assert((kKeys / 8 & (kKeys / 8 - 1)) == 0, "key groups must be powers of two");
 
