@@ -96,7 +96,8 @@ struct Carver {
   }
 };
 
-// Elements between consecutive problems of a batch.
+// Offsets between consecutive problems of a batch: the pair and bias tensors in
+// bytes (their element type varies), lse in floats, the mask in bytes.
 struct ProblemStrides {
   int64_t pair, bias, lse, mask;
 };
@@ -106,7 +107,7 @@ ProblemStrides problem_strides(const tri_attn_problem *p, bool has_mask) {
   return {N * N * p->H * p->c * es, (int64_t)p->H * N * N * es, N * p->H * N,
           has_mask ? (p->mask_row_stride == N ? N * N : N) : 0};
 }
-// `base` advanced by `bytes` (pair and bias offsets are in bytes).
+// `base` advanced by `bytes`.
 template <typename T> T *at(T *base, int64_t bytes) {
   return reinterpret_cast<T *>(reinterpret_cast<
       typename std::conditional<std::is_const<T>::value, const char, char>::type *>(base) +
