@@ -34,6 +34,22 @@ int main(void) {
     p.variant = TRI_ATTN_STARTING;
     CHECK(7, tri_attn_fwd(&p, fake, fake, fake, fake, fake, NULL, fake, (float *)fake, NULL, 0,
                           NULL) == TRI_ATTN_ERR_WORKSPACE);
+    {   /* a batch of 3 ending-node problems needs a transposed bias per problem; a
+           negative batch or a nonzero reserved field is refused */
+        size_t one = 0, three = 0;
+        p.variant = TRI_ATTN_ENDING;
+        p.batch = 1;
+        CHECK(14, tri_attn_fwd_workspace_size(&p, &one) == TRI_ATTN_OK);
+        p.batch = 3;
+        CHECK(15, tri_attn_fwd_workspace_size(&p, &three) == TRI_ATTN_OK &&
+                      three >= one + 2 * (size_t)2 * 4 * 64 * 64);
+        p.variant = TRI_ATTN_STARTING;
+        p.batch = -1;
+        CHECK(16, tri_attn_fwd_workspace_size(&p, &n) == TRI_ATTN_ERR_INVALID_ARG);
+        p.batch = 1; p.reserved = 5;
+        CHECK(17, tri_attn_fwd_workspace_size(&p, &n) == TRI_ATTN_ERR_INVALID_ARG);
+        p.batch = 0; p.reserved = 0;
+    }
 
     tri_mul_problem m = {64, 4, TRI_MUL_OUTGOING};
     CHECK(8, tri_mul_workspace_size(&m, &n) == TRI_ATTN_OK);
