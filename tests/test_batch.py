@@ -112,3 +112,31 @@ def test_calls_from_a_fresh_host_thread():
     assert "err" not in box, box.get("err")
     for name in OUTS:
         assert torch.equal(box["res"][name], ref[name]), name
+
+
+def test_onchip_option_with_a_batch_takes_the_default_backward():
+    """TRI_ATTN_OPT_ONCHIP_SUMS applies to single problems; a batch takes the
+    default backward and gives its bits."""
+    ds, g = draw_batch(2, 136, 2, 32, "bf16", "random:9", seed=11)
+    out, lse = ta.fwd(g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], STARTING)
+    args = (g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], out, lse, g["dout"], STARTING)
+    plain = ta.bwd(*args)
+    opt = ta.bwd(*args, opts=ta.launch_opts(onchip_sums=True))
+    torch.cuda.synchronize()
+    for a, b, name in zip(plain, opt, ("dq", "dk", "dv", "dbias", "dgate")):
+        assert torch.equal(a, b), name
+
+
+def test_exp2_split_forward_with_a_batch():
+    """The forward with one exponential pair in four on the FMA pipe runs a batch
+    in one launch too: each problem bit-identical to the same option alone."""
+    ds, g = draw_batch(3, 72, 2, 32, "bf16", "rows", seed=13)
+    opts = ta.launch_opts(exp2_split=True)
+    out, lse = ta.fwd(g["q"], g["k"], g["v"], g["bias"], g["gate"], g["mask"], ENDING, opts=opts)
+    torch.cuda.synchronize()
+    for i, d in enumerate(ds):
+        gi = to_device(d, "cuda:0")
+        o1, l1 = ta.fwd(gi["q"], gi["k"], gi["v"], gi["bias"], gi["gate"], gi["mask"], ENDING,
+                        opts=ta.launch_opts(exp2_split=True))
+        torch.cuda.synchronize()
+        assert torch.equal(out[i], o1) and torch.equal(lse[i], l1), i
